@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""Benchmark of the routed int4 MoE FFN hot path on B200.
+
+Default workload (one "step"): single-layer decode of 1 token through a MoE
+layer with 256 experts, top-8, hidden 2048, expert width 512 -- route, the
+weight-streaming expert FFN, combine.  Steps rotate over 40 resident layers
+(40 x 256 experts x 3 int4 matrices = 18.1 GB in HBM, each layer with its own
+activations and fresh router logits), so the 14.2 MB a step streams is never
+L2-resident from an earlier step (inputs larger than L2, no flush needed).
+
+Prints one JSON line (see the design doc for every key).  Multi-GPU: one process
+per GPU (torchrun), each rank an independent replica of the workload (the
+path has no exchange step), barrier + max-over-ranks timing.
+
+--impl reference times the CPU oracle (plain C, single thread) on the same
+workload: each step is one token through one layer, rotating over a small
+pool of sampled token-layers.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+E, TOPK, H, F = 256, 8, 2048, 512
+LAYERS = 40
+EXPERT_BYTES = 1769472  # packed int4 gate/up + down of one expert (36 B per 64 weights)
+METRIC = "routed-expert tokens/s + HBM GB/s (decode), TFLOP/s (prefill) vs roofline"
+WORKLOAD = ("single-layer decode: 256 experts, top-8, hidden 2048, expert width 512, 1 token per step; "
+            "steps rotate over 40 resident int4 layers (18.1 GB) with fresh router logits per layer")
+
+
+# ---------------------------------------------------------------------------- helpers
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            p = [v.strip() for v in ln.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                mx = max(mx, float(p[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, p[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def dist_max(v: float) -> float:
+    import torch
+    import torch.distributed as dist
+    if not dist.is_initialized():
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_barrier():
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------- workload
+def build_layers(L, seed, log):
+    """40 resident layers of packed int4 experts, generated and quantised on the GPU."""
+    import torch
+    import synth
+    import quantized_moe_route_b200 as moe
+    gu_b, d_b = moe.moe_w4_packed_bytes(2 * F, H), moe.moe_w4_packed_bytes(H, F)
+    chunk = 32
+    tmp = torch.empty((chunk, 2 * F, H), dtype=torch.float32, device="cuda")
+    codes = torch.empty((chunk * 2 * F, H), dtype=torch.uint8, device="cuda")
+    sc = torch.empty((chunk * 2 * F, H // 64), dtype=torch.int16, device="cuda")
+    mn = torch.empty_like(sc)
+    layers = []
+    t0 = time.time()
+    for l in range(L):
+        gu = torch.empty(E * gu_b, dtype=torch.uint8, device="cuda")
+        dn = torch.empty(E * d_b, dtype=torch.uint8, device="cuda")
+        for proj, buf, nb, (N, K), kind in ((synth.PROJ_GATE_UP, gu, gu_b, (2 * F, H), moe.MOE_W4_GATE_UP),
+                                             (synth.PROJ_DOWN, dn, d_b, (H, F), moe.MOE_W4_PLAIN)):
+            G = K // 64
+            for e0 in range(0, E, chunk):
+                w = tmp.view(-1)[: chunk * N * K].view(chunk, N, K)
+                synth.cuda_expert_weights(w, seed, l, e0, proj)
+                c = codes.view(-1)[: chunk * N * K].view(chunk * N, K)
+                s = sc.view(-1)[: chunk * N * G].view(chunk * N, G)
+                m = mn.view(-1)[: chunk * N * G].view(chunk * N, G)
+                moe.moe_quantize_w4(w.view(chunk * N, K), c, s, m)
+                for i in range(chunk):
+                    e = e0 + i
+                    moe.moe_pack_w4(c[i * N:(i + 1) * N], s[i * N:(i + 1) * N], m[i * N:(i + 1) * N], kind,
+                                    buf[e * nb:(e + 1) * nb])
+        layers.append((gu, dn, moe.make_layer(E, H, F, gu, dn)))
+    torch.cuda.synchronize()
+    del tmp, codes, sc, mn
+    log(f"built {L} layers in {time.time() - t0:.1f}s")
+    return layers
+
+
+def layer_inputs(seed, l, T):
+    import synth
+    x = synth.activations_bf16(seed, l, T, H)
+    logits = synth.router_logits(seed, l, T, E)
+    return x, logits
+
+
+def run_gpu(args, log):
+    import torch
+    import quantized_moe_route_b200 as moe
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    T = args.tokens
+    seed = 1000 + rank
+    layers = build_layers(LAYERS, seed, log)
+    k = TOPK
+    # per-layer device inputs, routing outputs and workspaces
+    xs, ls = [], []
+    uniq = []
+    for l in range(LAYERS):
+        x, lg = layer_inputs(seed, l, T)
+        xs.append(torch.from_numpy(x.view(np.int16)).to(dev))
+        ls.append(torch.from_numpy(lg).to(dev))
+        uniq.append(len(set(np.argsort(-lg, axis=1, kind="stable")[:, :k].ravel().tolist())))
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    y_rows = torch.empty((T * k, H), dtype=torch.float32, device=dev)
+    y = torch.empty((T, H), dtype=torch.int16, device=dev)
+    ws = torch.zeros(moe.moe_decode_workspace_bytes(T, k, F), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(l, ev=None):
+        moe.moe_route(ls[l], k, idx, w, stream=stream)
+        if ev is not None:
+            ev[0].record(stream)
+        moe.moe_ffn_w4a16_decode(layers[l][2], xs[l], idx, y_rows, ws, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        moe.moe_unpermute_combine(y_rows, w, y, stream=stream)
+
+    def capture(steps, first, events=None):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(steps):
+                step((first + i) % LAYERS, None if events is None else events[i])
+        return g
+
+    K, W = args.steps, args.warmup
+    # untimed warm-up (eager once, then a graph of W steps)
+    for l in range(min(W, LAYERS)):
+        step(l)
+    torch.cuda.synchronize()
+    g_warm = capture(W, 0)
+    g_main = capture(K, W)
+    g_warm.replay()
+    torch.cuda.synchronize()
+
+    dist_barrier()
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        dist_barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g_main.replay()
+        e1.record(stream)
+        e1.synchronize()
+        torch.cuda.synchronize()
+        dist_barrier()
+    ms_local = e0.elapsed_time(e1)
+    ms = dist_max(ms_local)
+    tokens = K * T * world
+    value = tokens / (ms / 1e3)
+
+    # kernel-duration pass: the same K steps with events around each FFN launch
+    evs = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+           for _ in range(K)]
+    g_prof = capture(K, W, evs)
+    g_prof.replay()
+    torch.cuda.synchronize()
+    durs = [a.elapsed_time(b) for a, b in evs]
+    dur_ms = sum(durs) / len(durs)
+    byts = [uniq[(W + i) % LAYERS] * EXPERT_BYTES + T * H * 2 + T * k * 4 + T * k * H * 4 for i in range(K)]
+    alg_bytes = sum(byts) / K
+    peak, peak_kind = peaks()
+    achieved = alg_bytes / (dur_ms / 1e3) / 1e9
+
+    # end-to-end through the C ABI with host buffers: H2D inputs, D2H output every step
+    hx = [torch.from_numpy(layer_inputs(seed, l, T)[0].view(np.int16)).pin_memory() for l in range(LAYERS)]
+    hl = [torch.from_numpy(layer_inputs(seed, l, T)[1]).pin_memory() for l in range(LAYERS)]
+    hy = torch.empty((T, H), dtype=torch.int16).pin_memory()
+    dx = torch.empty((T, H), dtype=torch.int16, device=dev)
+    dl = torch.empty((T, E), dtype=torch.float32, device=dev)
+
+    def e2e_step(l):
+        dx.copy_(hx[l], non_blocking=True)
+        dl.copy_(hl[l], non_blocking=True)
+        moe.moe_route(dl, k, idx, w, stream=stream)
+        moe.moe_ffn_w4a16_decode(layers[l][2], dx, idx, y_rows, ws, stream=stream)
+        moe.moe_unpermute_combine(y_rows, w, y, stream=stream)
+        hy.copy_(y, non_blocking=True)
+
+    ge = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        for l in range(3):
+            e2e_step(l)
+    stream.synchronize()
+    with torch.cuda.graph(ge, stream=stream):
+        with torch.cuda.stream(stream):
+            for i in range(K):
+                e2e_step((W + i) % LAYERS)
+    ge.replay()
+    torch.cuda.synchronize()
+    dist_barrier()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    ge.replay()
+    a1.record(stream)
+    a1.synchronize()
+    e2e_ms = dist_max(a0.elapsed_time(a1))
+    e2e_value = tokens / (e2e_ms / 1e3)
+
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int4 weights (f16 scale/min), bf16 activations, fp32 accumulate", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "experts": E, "top_k": k, "hidden": H, "expert_width": F,
+                   "tokens_per_step": T, "resident_layers": LAYERS, "seed": 1000,
+                   "l2": "inputs larger than L2 (18.1 GB resident, 40-layer rotation)",
+                   "parallelism": f"replicas x{world}", "graph": "CUDA graph of K steps, PDL between kernels"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "kernel": "moe::decode_kernel",
+                     "peak_kind": peak_kind, "alg_bytes_per_launch": alg_bytes,
+                     "avg_launch_us": dur_ms * 1e3},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2 + T * E * 4,
+                "d2h_bytes_per_step": T * H * 2},
+        "gpu_launches": 3 * K,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(seed, T, budget_s=args.cpu_seconds, log=log)
+    if world > 1:
+        import torch.distributed as dist
+        del g_main, g_warm, g_prof, ge
+        dist.barrier()
+        dist.destroy_process_group()
+    return out if rank == 0 else None
+
+
+# ---------------------------------------------------------------------------- CPU oracle
+def oracle_pool(seed, T, n, log, use_gpu_generator):
+    """n sampled token-layers: canonical weights of their routed experts, built
+    with the seeded generator and the oracle's own quantiser."""
+    import oracle
+    import synth
+    pool = []
+    t0 = time.time()
+    for l in range(n):
+        x, lg = layer_inputs(seed, l, T)
+        idx, _ = oracle.route(lg, TOPK)
+        experts = {}
+        for e in sorted(set(idx.ravel().tolist())):
+            if use_gpu_generator:
+                import torch
+                wg = torch.empty((1, 2 * F, H), device="cuda")
+                wd = torch.empty((1, H, F), device="cuda")
+                synth.cuda_expert_weights(wg, seed, l, e, synth.PROJ_GATE_UP)
+                synth.cuda_expert_weights(wd, seed, l, e, synth.PROJ_DOWN)
+                a, b = wg[0].cpu().numpy(), wd[0].cpu().numpy()
+            else:
+                a = synth.expert_weights(seed, l, e, synth.PROJ_GATE_UP, 2 * F, H)
+                b = synth.expert_weights(seed, l, e, synth.PROJ_DOWN, H, F)
+            experts[e] = (oracle.quantize_w4(a), oracle.quantize_w4(b))
+        pool.append((x, lg, experts))
+    log(f"oracle pool of {n} token-layers built in {time.time() - t0:.1f}s")
+    return pool
+
+
+def cpu_baseline(seed, T, budget_s, log):
+    import oracle
+    pool = oracle_pool(seed, T, 4, log, use_gpu_generator=True)
+    t0 = time.time()
+    n = 0
+    while True:
+        x, lg, experts = pool[n % len(pool)]
+        oracle.moe_forward_w4(x, lg, TOPK, experts)
+        n += 1
+        if time.time() - t0 >= budget_s:
+            break
+    dt = time.time() - t0
+    return {"value": n * T / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} token-layer steps (T={T}) over a pool of {len(pool)} sampled layers, {dt:.1f}s"}
+
+
+def run_reference(args, log):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    import oracle
+    T = args.tokens
+    pool = oracle_pool(1000, T, 4, log, use_gpu_generator=False)
+    for i in range(args.warmup):
+        x, lg, ex = pool[i % len(pool)]
+        oracle.moe_forward_w4(x, lg, TOPK, ex)
+    t0 = time.time()
+    for i in range(args.steps):
+        x, lg, ex = pool[i % len(pool)]
+        oracle.moe_forward_w4(x, lg, TOPK, ex)
+    dt = time.time() - t0
+    value = args.steps * T / dt
+    sample = f"{args.steps} token-layer steps (T={T}) rotating over {len(pool)} sampled layers"
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int4 weights (f16 scale/min), bf16 activations, fp32 accumulate", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "experts": E, "top_k": TOPK, "hidden": H, "expert_width": F,
+                   "tokens_per_step": T, "parallelism": "single CPU thread (oracle)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--tokens", type=int, default=1)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--quiet", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    def log(msg):
+        if not args.quiet:
+            print(f"[bench] {msg}", file=sys.stderr, flush=True)
+
+    if args.impl == "reference":
+        out = run_reference(args, log)
+    else:
+        out = run_gpu(args, log)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,232 @@
+/*
+ * moe.h -- C ABI of libmoe, the routed 4-bit mixture-of-experts FFN for B200
+ * (sm_100a).
+ *
+ * The operation: a token's router logits pick k of E experts by softmax and
+ * renormalised top-k; each picked expert applies a SwiGLU FFN
+ * (gate/up: H -> F, SiLU(gate) * up, down: F -> H) whose weights are stored as
+ * 4-bit codes; the k expert outputs are summed with the routing weights.
+ * Sources, by page title and section:
+ *   - "Drama 3 int4 (drama-rs format)", section "What's quantized": routed
+ *     experts are int4, asymmetric, group 64, f16 scale + min.
+ *   - "drama-rs", section "Apple Silicon (MLX)": the same values map to the
+ *     packed affine form w = q * scale + min; prefill groups rows by routed
+ *     expert; section "Footprint and speed": decode is weight streaming.
+ *   - "Drama 3 - NVFP4 routed experts", section "Quantization": 40 layers x 256
+ *     experts x 3 projections; the NVFP4 variant (E2M1 codes, E4M3 scale per 16
+ *     input channels, FP32 global scale per matrix shared by gate and up,
+ *     dynamic per-token activation scales).
+ *
+ * Conventions (every call):
+ *   - Returns moe_status; argument errors are found on the host before any
+ *     launch and nothing is enqueued then.  MOE_ERR_CUDA reports a launch
+ *     error (the CUDA error string is kept for moe_last_error_string()).
+ *   - Every array argument is a DEVICE pointer owned by the caller, unless the
+ *     comment says "host".  The library allocates no memory: calls that need
+ *     scratch take a caller workspace sized by the matching *_workspace_bytes()
+ *     query.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously; nothing synchronises.
+ *   - bf16 and f16 values travel as uint16_t bit patterns.
+ *   - Inputs must be finite; NaN logits or activations give unspecified
+ *     (but memory-safe) results.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_API __attribute__((visibility("default")))
+
+typedef void *moe_stream_t; /* a cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,       /* null pointer, negative size, k > E, ... */
+  MOE_ERR_UNSUPPORTED_SHAPE = 2, /* a size this library's kernels do not tile */
+  MOE_ERR_WORKSPACE = 3,         /* workspace missing or smaller than required */
+  MOE_ERR_CUDA = 4,              /* a CUDA launch or runtime call failed */
+  MOE_ERR_TIMEOUT = 5            /* a bounded device-side wait gave up */
+} moe_status;
+
+/* Human-readable name of a status code (static string). */
+MOE_API const char *moe_status_string(moe_status s);
+/* Text of the last CUDA error seen by this thread (static storage). */
+MOE_API const char *moe_last_error_string(void);
+/* Library version string, e.g. "moe-w4-b200 1". */
+MOE_API const char *moe_version(void);
+
+/* ======================================================================== */
+/* int4 expert weights                                                       */
+/* ======================================================================== */
+/*
+ * Canonical form of one [N][K] matrix (K = input channels):
+ *   codes u8 [N][K], values 0..15
+ *   scale f16 [N][K/64], min f16 [N][K/64]: group g of row n covers
+ *   channels [64g, 64g + 64); the weight is codes * scale + min.
+ * A gate/up pair is one canonical [2F][H] matrix: rows [0, F) gate, rows
+ * [F, 2F) up.
+ *
+ * Device ("packed") form, written by moe_pack_w4 and read by every kernel:
+ * 16-row strips, each strip a run of K/64 blocks of 576 bytes (512 bytes of
+ * codes in the register order of the decode kernel's tensor-core fragments,
+ * then 16 x {f16 scale, f16 min}).  Size: moe_w4_packed_bytes(N, K) =
+ * N * K * 9 / 16 bytes.  For kind MOE_W4_GATE_UP the gate strip i and the up
+ * strip i (same 16 features) are stored next to each other.
+ * Requirements: N % 16 == 0 (gate/up: F % 16 == 0), K % 64 == 0.
+ */
+typedef enum { MOE_W4_PLAIN = 0, MOE_W4_GATE_UP = 1 } moe_w4_kind;
+
+MOE_API size_t moe_w4_packed_bytes(int N, int K);
+
+/*
+ * Quantise fp32 weights w [N][K] to the canonical int4 form (group 64 along K,
+ * asymmetric): per group m = f16(min) rounded toward -inf, s = f16((max - m)/15)
+ * rounded toward +inf, q = clamp(rint((w - m) / s), 0, 15) in fp32 (s = 0 gives
+ * q = 0).  Outputs codes [N][K], scale [N][K/64], min [N][K/64].
+ * Source: "Drama 3 int4 (drama-rs format)", "What's quantized" (asymmetric,
+ * group 64, f16 scale + min); plain min/max instead of the page's MSE clip
+ * search.  Errors: INVALID_ARG (null, N or K < 0), UNSUPPORTED_SHAPE (K % 64).
+ */
+MOE_API moe_status moe_quantize_w4(const float *w, int N, int K, uint8_t *codes,
+                                   uint16_t *scale, uint16_t *minv, moe_stream_t stream);
+
+/* Canonical -> packed.  packed_bytes must be >= moe_w4_packed_bytes(N, K).
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE (N % 16, K % 64, GATE_UP with N % 32),
+ * WORKSPACE (packed_bytes too small). */
+MOE_API moe_status moe_pack_w4(const uint8_t *codes, const uint16_t *scale,
+                               const uint16_t *minv, int N, int K, int kind, void *packed,
+                               size_t packed_bytes, moe_stream_t stream);
+
+/* Packed -> canonical (exact inverse of moe_pack_w4). */
+MOE_API moe_status moe_unpack_w4(const void *packed, int N, int K, int kind, uint8_t *codes,
+                                 uint16_t *scale, uint16_t *minv, moe_stream_t stream);
+
+/* Packed -> dequantised fp32 [N][K] in canonical row order, each weight one
+ * fp32 fused multiply-add q * s + m (the value the oracle's dequant gives,
+ * bit for bit).  A test and debugging export; kernels never materialise it. */
+MOE_API moe_status moe_dequant_w4(const void *packed, int N, int K, int kind, float *out,
+                                  moe_stream_t stream);
+
+/*
+ * One MoE layer's experts, all in device memory, experts stored back to back:
+ *   gate_up: E * moe_w4_packed_bytes(2F, H) bytes, expert e at
+ *            e * moe_w4_packed_bytes(2F, H), packed with kind MOE_W4_GATE_UP
+ *   down:    E * moe_w4_packed_bytes(H, F) bytes, kind MOE_W4_PLAIN
+ * The struct itself is a HOST struct passed by pointer; it is read during
+ * the call only.
+ */
+typedef struct {
+  int E, H, F;
+  const void *gate_up;
+  const void *down;
+} moe_w4_layer;
+
+/* ======================================================================== */
+/* Routing and permutation                                                   */
+/* ======================================================================== */
+
+/*
+ * Top-k routing of T tokens over E experts from fp32 logits [T][E].
+ * idx [T][k]: the k largest logits' expert ids, larger logit first, equal
+ * logits to the lower expert id first.  w [T][k]: softmax over all E,
+ * restricted to the selected experts and renormalised to sum to one (equal to
+ * the softmax of the selected logits).  Source: the router of "Drama 3 int4",
+ * "What's quantized" (bf16 router); top-k, renormalisation and tie order are
+ * this library's reading.  Limits: 1 <= k <= min(E, 32), E <= 1024.
+ * T == 0 is a no-op.  Errors: INVALID_ARG, UNSUPPORTED_SHAPE.
+ */
+MOE_API moe_status moe_route(const float *logits, int T, int E, int k, int32_t *idx, float *w,
+                             moe_stream_t stream);
+
+/*
+ * Group the T*k rows r = t*k + j by expert idx[r] (stable: within an expert,
+ * rows in increasing r).  Outputs counts [E], offsets [E+1] (exclusive scan,
+ * offsets[E] = T*k), sorted_rows [T*k] (row ids in grouped order), inv [T*k]
+ * (inv[r] = position of row r).  If x (bf16 [T][H]) and x_perm are non-null,
+ * also gathers x_perm[p] = x[sorted_rows[p] / k] (bf16 [T*k][H], H % 8 == 0).
+ * Source: "drama-rs", "Apple Silicon (MLX)": prefill groups rows by routed
+ * expert.  Counting is deterministic and uses no global atomics.
+ * Workspace: moe_permute_workspace_bytes(T, k, E).  idx values must lie in
+ * [0, E).  Errors: INVALID_ARG, UNSUPPORTED_SHAPE, WORKSPACE.
+ */
+MOE_API size_t moe_permute_workspace_bytes(int T, int k, int E);
+MOE_API moe_status moe_permute(const int32_t *idx, int T, int k, int E, const uint16_t *x,
+                               int H, int32_t *counts, int32_t *offsets, int32_t *sorted_rows,
+                               int32_t *inv, uint16_t *x_perm, void *ws, size_t ws_bytes,
+                               moe_stream_t stream);
+
+/* ======================================================================== */
+/* Expert FFN                                                                */
+/* ======================================================================== */
+
+/*
+ * Decode: the expert FFN of every row r = t*k + j, expert idx[r], on x[t]:
+ *   g, u = W_gate x, W_up x;  h = SiLU(g) * u;  y_rows[r] = W_down h
+ * for a small batch (1 <= T <= 16 tokens, T*k <= 256), streaming each selected
+ * expert's int4 weights from HBM once per call whatever the number of tokens
+ * routed to it.  x bf16 [T][H]; idx [T][k] (from moe_route); y_rows fp32
+ * [T*k][H].  Accumulation is fp32; h is rounded to bf16 before the down
+ * projection.  Source: "drama-rs", "Footprint and speed" (decode is weight
+ * streaming GEMVs) and "Experts: where they run" (decode is memory-bandwidth
+ * bound); the SwiGLU expert of the Qwen3.5-MoE backbone.
+ * Workspace: moe_decode_workspace_bytes(T, k, F); it must be zero-filled
+ * before its first use, and every successful call leaves it zero-filled again
+ * (so one workspace serves any number of stream-ordered calls).  Calls that
+ * share a workspace must not overlap in time.
+ * Requirements: H % 64 == 0, F % 64 == 0, idx values in [0, E), the k
+ * experts of a token distinct.  Errors: INVALID_ARG, UNSUPPORTED_SHAPE,
+ * WORKSPACE, CUDA.  A device-side wait that times out (it cannot under the
+ * requirements above) raises the device error word: see moe_device_error().
+ */
+MOE_API size_t moe_decode_workspace_bytes(int T, int k, int F);
+MOE_API moe_status moe_ffn_w4a16_decode(const moe_w4_layer *layer, const uint16_t *x,
+                                        const int32_t *idx, int T, int k, float *y_rows,
+                                        void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Prefill: grouped GEMM over experts.  x_perm bf16 [rows][H] holds the rows
+ * grouped by expert (from moe_permute), offsets [E+1] (device) delimits the
+ * groups.  Writes y_perm bf16 [rows][H] = W_down (SiLU(W_gate x) * W_up x)
+ * for every row with its group's expert, on the tensor cores (tcgen05, fp32
+ * accumulation in tensor memory, h rounded to bf16).
+ * Source: "drama-rs", "Layout" (prefill: grouped MoE) and "Apple Silicon
+ * (MLX)" (prefill groups rows by routed expert).
+ * Workspace: moe_prefill_workspace_bytes(rows, F).
+ * Requirements: H % 128 == 0, F % 128 == 0, offsets non-decreasing with
+ * offsets[0] == 0 and offsets[E] == rows.  rows == 0 is a no-op.
+ */
+MOE_API size_t moe_prefill_workspace_bytes(int rows, int F);
+MOE_API moe_status moe_ffn_grouped_prefill(const moe_w4_layer *layer, const uint16_t *x_perm,
+                                           const int32_t *offsets, int rows, uint16_t *y_perm,
+                                           void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Router-weighted combine: y[t] = sum over j = 0..k-1 (in that order) of
+ * w[t][j] * Y[p(t*k + j)], accumulated in fp32 and rounded to nearest-even
+ * bf16.  Y is y_rows (fp32, y_dtype 0) or y_perm (bf16, y_dtype 1), [T*k][H];
+ * p = inv (from moe_permute) or the identity when inv is NULL.  Every output
+ * row is owned by one thread block: no atomics, deterministic.
+ * Requirements: H % 8 == 0.  T == 0 is a no-op.
+ */
+MOE_API moe_status moe_unpermute_combine(const void *Y, int y_dtype, const int32_t *inv,
+                                         const float *w, int T, int k, int H, uint16_t *y,
+                                         moe_stream_t stream);
+
+/* ======================================================================== */
+/* Device error word                                                         */
+/* ======================================================================== */
+/* Host pointer out receives (after a stream synchronise done by this call)
+ * the device error word: 0 = none, otherwise a code naming the kernel and
+ * wait that timed out.  The word is cleared on read. */
+MOE_API moe_status moe_device_error(int *out, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H_ */

@@ -1,0 +1,180 @@
+"""Python binding of libmoe, the routed 4-bit MoE FFN for B200 (sm_100a).
+
+Argument marshalling only: every function below forwards device pointers and
+sizes to the C ABI declared in ``include/moe.h`` under the same name; all work
+runs in the library's CUDA kernels.  Tensors are torch CUDA tensors (torch
+supplies device memory and streams); bf16/f16 buffers may be torch.bfloat16 /
+torch.float16 or int16/uint16 views of the same bits.
+
+The library must be built (``python -m quantized_moe_route_b200.build`` or
+``__graft_entry__.build()``); importing the binding without it raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoe.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE = 0, 1, 2
+MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = 3, 4, 5
+MOE_W4_PLAIN, MOE_W4_GATE_UP = 0, 1
+
+_lib = None
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        L = lib()
+        msg = L.moe_status_string(status).decode()
+        if status == MOE_ERR_CUDA:
+            msg += " (" + L.moe_last_error_string().decode() + ")"
+        super().__init__(f"{where}: {msg}")
+
+
+class moe_w4_layer(ctypes.Structure):
+    _fields_ = [("E", ctypes.c_int), ("H", ctypes.c_int), ("F", ctypes.c_int),
+                ("gate_up", ctypes.c_void_p), ("down", ctypes.c_void_p)]
+
+
+_vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+SIGNATURES = {
+    "moe_status_string": (ctypes.c_char_p, [_i]),
+    "moe_last_error_string": (ctypes.c_char_p, []),
+    "moe_version": (ctypes.c_char_p, []),
+    "moe_w4_packed_bytes": (_sz, [_i, _i]),
+    "moe_quantize_w4": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp]),
+    "moe_pack_w4": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
+    "moe_unpack_w4": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "moe_dequant_w4": (_i, [_vp, _i, _i, _i, _vp, _vp]),
+    "moe_route": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
+    "moe_permute_workspace_bytes": (_sz, [_i, _i, _i]),
+    "moe_permute": (_i, [_vp, _i, _i, _i, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_decode_workspace_bytes": (_sz, [_i, _i, _i]),
+    "moe_ffn_w4a16_decode": (_i, [ctypes.POINTER(moe_w4_layer), _vp, _vp, _i, _i, _vp, _vp, _sz, _vp]),
+    "moe_prefill_workspace_bytes": (_sz, [_i, _i]),
+    "moe_ffn_grouped_prefill": (_i, [ctypes.POINTER(moe_w4_layer), _vp, _vp, _i, _vp, _vp, _sz, _vp]),
+    "moe_unpermute_combine": (_i, [_vp, _i, _vp, _vp, _i, _i, _i, _vp, _vp]),
+    "moe_device_error": (_i, [ctypes.POINTER(ctypes.c_int), _vp]),
+}
+
+
+def lib():
+    """The loaded libmoe (raises if the in-tree build is missing)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libmoe.so is not built ({LIB_PATH}); run quantized_moe_route_b200/build.py")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(status, where):
+    if status != MOE_OK:
+        raise MoeError(status, where)
+
+
+# ---------------------------------------------------------------- int4 weights
+def moe_w4_packed_bytes(N: int, K: int) -> int:
+    return lib().moe_w4_packed_bytes(N, K)
+
+
+def moe_quantize_w4(w, codes, scale, minv, stream=None):
+    N, K = w.shape
+    _check(lib().moe_quantize_w4(_p(w), N, K, _p(codes), _p(scale), _p(minv), _stream(stream)),
+           "moe_quantize_w4")
+
+
+def moe_pack_w4(codes, scale, minv, kind, packed, stream=None):
+    N, K = codes.shape
+    nbytes = packed.numel() * packed.element_size()
+    _check(lib().moe_pack_w4(_p(codes), _p(scale), _p(minv), N, K, kind, _p(packed), nbytes,
+                             _stream(stream)), "moe_pack_w4")
+
+
+def moe_unpack_w4(packed, N, K, kind, codes, scale, minv, stream=None):
+    _check(lib().moe_unpack_w4(_p(packed), N, K, kind, _p(codes), _p(scale), _p(minv),
+                               _stream(stream)), "moe_unpack_w4")
+
+
+def moe_dequant_w4(packed, N, K, kind, out, stream=None):
+    _check(lib().moe_dequant_w4(_p(packed), N, K, kind, _p(out), _stream(stream)), "moe_dequant_w4")
+
+
+def make_layer(E, H, F, gate_up, down) -> moe_w4_layer:
+    """Host descriptor of one layer's packed experts (device buffers)."""
+    return moe_w4_layer(E, H, F, gate_up.data_ptr(), down.data_ptr())
+
+
+# ---------------------------------------------------------------- routing / permutation
+def moe_route(logits, k, idx, w, stream=None):
+    T, E = logits.shape
+    _check(lib().moe_route(_p(logits), T, E, k, _p(idx), _p(w), _stream(stream)), "moe_route")
+
+
+def moe_permute_workspace_bytes(T, k, E) -> int:
+    return lib().moe_permute_workspace_bytes(T, k, E)
+
+
+def moe_permute(idx, E, counts, offsets, sorted_rows, inv, ws, x=None, x_perm=None, stream=None):
+    T, k = idx.shape
+    H = 0 if x is None else x.shape[1]
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib().moe_permute(_p(idx), T, k, E, _p(x), H, _p(counts), _p(offsets), _p(sorted_rows),
+                             _p(inv), _p(x_perm), _p(ws), nbytes, _stream(stream)), "moe_permute")
+
+
+# ---------------------------------------------------------------- expert FFN
+def moe_decode_workspace_bytes(T, k, F) -> int:
+    return lib().moe_decode_workspace_bytes(T, k, F)
+
+
+def moe_ffn_w4a16_decode(layer: moe_w4_layer, x, idx, y_rows, ws, stream=None):
+    T, k = idx.shape
+    _check(lib().moe_ffn_w4a16_decode(ctypes.byref(layer), _p(x), _p(idx), T, k, _p(y_rows), _p(ws),
+                                      ws.numel() * ws.element_size(), _stream(stream)),
+           "moe_ffn_w4a16_decode")
+
+
+def moe_prefill_workspace_bytes(rows, F) -> int:
+    return lib().moe_prefill_workspace_bytes(rows, F)
+
+
+def moe_ffn_grouped_prefill(layer: moe_w4_layer, x_perm, offsets, y_perm, ws, stream=None):
+    rows = x_perm.shape[0]
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib().moe_ffn_grouped_prefill(ctypes.byref(layer), _p(x_perm), _p(offsets), rows,
+                                         _p(y_perm), _p(ws), nbytes, _stream(stream)),
+           "moe_ffn_grouped_prefill")
+
+
+def moe_unpermute_combine(Y, w, y, inv=None, stream=None):
+    T, k = w.shape
+    H = y.shape[1]
+    y_dtype = 0 if Y.element_size() == 4 else 1
+    _check(lib().moe_unpermute_combine(_p(Y), y_dtype, _p(inv), _p(w), T, k, H, _p(y),
+                                       _stream(stream)), "moe_unpermute_combine")
+
+
+def moe_device_error(stream=None) -> int:
+    out = ctypes.c_int(0)
+    _check(lib().moe_device_error(ctypes.byref(out), _stream(stream)), "moe_device_error")
+    return out.value

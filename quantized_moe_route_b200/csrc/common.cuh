@@ -1,0 +1,177 @@
+// common.cuh -- shared host/device helpers of libmoe (sm_100a only).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "libmoe is written for sm_100a (B200) only"
+#endif
+
+namespace moe {
+
+// ---------------------------------------------------------------- host side
+void set_cuda_error(cudaError_t e);
+moe_status launch_status();  // checks cudaGetLastError after a launch
+
+inline cudaStream_t as_stream(moe_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Device error word (one per device, cleared by moe_device_error).
+enum : int {
+  DEVERR_NONE = 0,
+  DEVERR_DECODE_H_WAIT = 0x101,   // decode: down projection waited too long for h
+  DEVERR_PREFILL_WAIT = 0x201,    // prefill: a pipeline barrier wait gave up
+};
+int *device_error_word();  // device address of the word on the current device
+
+// Layout of one packed int4 block: 16 rows x 64 input channels.
+constexpr int kBlkRows = 16;
+constexpr int kGroup = 64;
+constexpr int kBlkCodeBytes = 512;
+constexpr int kBlkBytes = 576;
+
+__host__ __device__ inline size_t w4_packed_bytes(int N, int K) {
+  return (size_t)(N / kBlkRows) * (size_t)(K / kGroup) * kBlkBytes;
+}
+
+// Device strip index of canonical row n (a multiple of 16).  Gate/up:
+// canonical rows [0, F) gate, [F, 2F) up; device strips alternate gate, up.
+__host__ __device__ inline int w4_strip_of_row(int n, int N, int kind) {
+  if (kind == MOE_W4_GATE_UP) {
+    int F = N / 2;
+    return n < F ? 2 * (n / kBlkRows) : 2 * ((n - F) / kBlkRows) + 1;
+  }
+  return n / kBlkRows;
+}
+__host__ __device__ inline int w4_row_of_strip(int s, int N, int kind) {
+  if (kind == MOE_W4_GATE_UP) {
+    int F = N / 2;
+    return (s & 1) ? F + (s >> 1) * kBlkRows : (s >> 1) * kBlkRows;
+  }
+  return s * kBlkRows;
+}
+
+// Position of canonical (row r in 0..15, channel c in 0..63) of a block:
+// lane (0..31), word (0..3) and nibble shift inside the word.  The word of
+// lane l = 4*g + t for k16-step j holds, nibble by nibble (shift 0, 4, 8, ...,
+// 28): (g, 16j+2t), (g+8, 16j+2t), (g, 16j+2t+8), (g+8, 16j+2t+8),
+//       (g, 16j+2t+1), (g+8, 16j+2t+1), (g, 16j+2t+9), (g+8, 16j+2t+9).
+// Masking the word with 0x000F000F after a right shift of 0, 4, 8 or 12 gives
+// the bf16x2 pairs of the m16n8k16 A fragment registers a0a1, a2a3, a4a5, a6a7.
+__host__ __device__ inline void w4_block_pos(int r, int c, int *lane, int *word, int *shift) {
+  int g = r & 7, hi_row = r >> 3;
+  int j = c >> 4, cc = c & 15;
+  int hi_k = cc >> 3, t = (cc & 7) >> 1, odd = cc & 1;
+  *lane = 4 * g + t;
+  *word = j;
+  *shift = 16 * odd + 8 * hi_k + 4 * hi_row;
+}
+
+// ---------------------------------------------------------------- device side
+#ifdef __CUDACC__
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// mbarrier (shared memory, CTA scope)
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: returns false (and leaves the barrier alone) after `limit`
+// failed polls.  Each try_wait itself suspends for a hardware-chosen time.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
+                                                  uint32_t limit) {
+  for (uint32_t i = 0; i < limit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+// 1-D bulk copy global -> shared, completion counted on an mbarrier (no
+// multicast).  Addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
+                                         uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void bulk_g2s_evict_first(void *dst, const void *src, uint32_t bytes,
+                                                     uint64_t *bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], "
+      "%2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// Legacy warp-level MMA used by the decode kernel as its dot-product engine:
+// D[16x8] (fp32) = A[16x16] (bf16, row) * B[16x8] (bf16, col) + C.
+__device__ __forceinline__ void mma_bf16_16816(float d[4], const uint32_t a[4], uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_gpu_add(int *p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
+  return __uint_as_float(((uint32_t)b) << 16);
+}
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
+  __nv_bfloat16 h = __float2bfloat16_rn(f);
+  return *reinterpret_cast<uint16_t *>(&h);
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  return (uint32_t)f32_to_bf16_bits(lo) | ((uint32_t)f32_to_bf16_bits(hi) << 16);
+}
+__device__ __forceinline__ float f16_bits_to_f32(uint16_t b) {
+  return __half2float(__ushort_as_half(b));
+}
+
+#endif  // __CUDACC__
+
+}  // namespace moe

@@ -1,0 +1,180 @@
+// permute.cu -- group the T*k routed rows by expert ("drama-rs", section
+// "Apple Silicon (MLX)": prefill groups rows by routed expert).
+//
+// Three stream-ordered kernels, no global atomics:
+//   1. per-chunk expert histograms (shared-memory counters),
+//   2. one block: totals, exclusive scan -> offsets, per-chunk bases,
+//   3. per chunk: stable ranks with warp match + popc, scatter of
+//      sorted_rows / inv, and the optional gather of x rows into x_perm.
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kPermChunk = 256;  // rows per chunk (one block each)
+
+__global__ void perm_hist_kernel(const int32_t *__restrict__ idx, int R, int E,
+                                 int32_t *__restrict__ hist) {
+  extern __shared__ int32_t sh[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) sh[e] = 0;
+  __syncthreads();
+  const int r0 = blockIdx.x * kPermChunk;
+  for (int r = r0 + threadIdx.x; r < min(R, r0 + kPermChunk); r += blockDim.x)
+    if ((unsigned)idx[r] < (unsigned)E) atomicAdd(&sh[idx[r]], 1);  // ids outside [0, E) are skipped
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(size_t)blockIdx.x * E + e] = sh[e];
+}
+
+// One block of up to 1024 threads; thread e walks the chunks of expert e.
+__global__ void perm_scan_kernel(const int32_t *__restrict__ hist, int nchunks, int E,
+                                 int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
+                                 int32_t *__restrict__ base) {
+  extern __shared__ int32_t sh[];  // [E] totals then scanned
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int s = 0;
+    for (int c = 0; c < nchunks; ++c) s += hist[(size_t)c * E + e];
+    sh[e] = s;
+    counts[e] = s;
+  }
+  __syncthreads();
+  // block-wide exclusive scan of sh[0..E), 1024 entries per pass
+  __shared__ int32_t warp_sum[32];
+  __shared__ int32_t carry;
+  if (threadIdx.x == 0) carry = 0;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  for (int e0 = 0; e0 < E; e0 += blockDim.x) {
+    __syncthreads();
+    const int e = e0 + threadIdx.x;
+    const int v = e < E ? sh[e] : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    if (lane == 31) warp_sum[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+      int ws = lane < (int)(blockDim.x >> 5) ? warp_sum[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int n = __shfl_up_sync(0xffffffffu, ws, o);
+        if (lane >= o) ws += n;
+      }
+      warp_sum[lane] = ws;  // inclusive over warps
+    }
+    __syncthreads();
+    const int excl = carry + (wid ? warp_sum[wid - 1] : 0) + incl - v;
+    if (e < E) {
+      sh[e] = excl;
+      offsets[e] = excl;
+    }
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) carry = excl + v;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) offsets[E] = carry;
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = sh[e];
+    for (int c = 0; c < nchunks; ++c) {
+      base[(size_t)c * E + e] = run;
+      run += hist[(size_t)c * E + e];
+    }
+  }
+}
+
+// One warp assigns positions to the chunk's rows 32 at a time, in row order;
+// then the whole block copies the activation rows.
+__global__ void perm_scatter_kernel(const int32_t *__restrict__ idx, int R, int E, int k,
+                                    const int32_t *__restrict__ base,
+                                    int32_t *__restrict__ sorted_rows, int32_t *__restrict__ inv,
+                                    const uint16_t *__restrict__ x, int H,
+                                    uint16_t *__restrict__ x_perm) {
+  extern __shared__ int32_t run[];  // [E] running position per expert
+  __shared__ int32_t pos_of[kPermChunk];
+  const int r0 = blockIdx.x * kPermChunk;
+  const int nrows = min(R - r0, kPermChunk);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) run[e] = base[(size_t)blockIdx.x * E + e];
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    for (int i0 = 0; i0 < nrows; i0 += 32) {
+      const int i = i0 + lane;
+      const int ei = i < nrows ? idx[r0 + i] : -1;
+      const bool valid = (unsigned)ei < (unsigned)E;  // ids outside [0, E) are skipped
+      const int e = valid ? ei : -1 - lane;           // invalid lanes never match
+      const uint32_t active = __ballot_sync(0xffffffffu, valid);
+      const uint32_t peers = __match_any_sync(0xffffffffu, e) & active;
+      if (valid) {
+        const int rank = __popc(peers & ((1u << lane) - 1u));
+        const int p = run[e] + rank;
+        pos_of[i] = p;
+        sorted_rows[p] = r0 + i;
+        inv[r0 + i] = p;
+      }
+      __syncwarp();
+      if (valid && lane == __ffs(peers) - 1) run[e] += __popc(peers);
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  if (!x_perm) return;
+  const int vec = H / 8;  // 16-byte vectors per row
+  for (int i = 0; i < nrows; ++i) {
+    if ((unsigned)idx[r0 + i] >= (unsigned)E) continue;
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)((r0 + i) / k) * H);
+    uint4 *dst = reinterpret_cast<uint4 *>(x_perm + (size_t)pos_of[i] * H);
+    for (int v = threadIdx.x; v < vec; v += blockDim.x) dst[v] = src[v];
+  }
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+static int perm_chunks(int R) { return (R + kPermChunk - 1) / kPermChunk; }
+
+extern "C" MOE_API size_t moe_permute_workspace_bytes(int T, int k, int E) {
+  if (T <= 0 || k <= 0 || E <= 0) return 0;
+  return 2 * sizeof(int32_t) * (size_t)perm_chunks(T * k) * (size_t)E;
+}
+
+extern "C" MOE_API moe_status moe_permute(const int32_t *idx, int T, int k, int E,
+                                          const uint16_t *x, int H, int32_t *counts,
+                                          int32_t *offsets, int32_t *sorted_rows, int32_t *inv,
+                                          uint16_t *x_perm, void *ws, size_t ws_bytes,
+                                          moe_stream_t stream) {
+  if (T < 0 || k <= 0 || E <= 0 || k > E) return MOE_ERR_INVALID_ARG;
+  if (E > 8192) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  if (T == 0) {  // empty batch: all counts zero, offsets all zero
+    cudaError_t e1 = cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, s);
+    cudaError_t e2 = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), s);
+    if (e1 != cudaSuccess || e2 != cudaSuccess) {
+      set_cuda_error(e1 != cudaSuccess ? e1 : e2);
+      return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+  }
+  if (!idx || !sorted_rows || !inv) return MOE_ERR_INVALID_ARG;
+  const bool gather = (x_perm != nullptr);
+  if (gather && (!x || H <= 0)) return MOE_ERR_INVALID_ARG;
+  if (gather && (H % 8 || reinterpret_cast<uintptr_t>(x) % 16 ||
+                 reinterpret_cast<uintptr_t>(x_perm) % 16))
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)T * k > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED_SHAPE;
+  const int R = T * k, nch = perm_chunks(R);
+  if (!ws || ws_bytes < moe_permute_workspace_bytes(T, k, E)) return MOE_ERR_WORKSPACE;
+  int32_t *hist = static_cast<int32_t *>(ws);
+  int32_t *base = hist + (size_t)nch * E;
+  const size_t shE = sizeof(int32_t) * (size_t)E;
+  perm_hist_kernel<<<nch, 256, shE, s>>>(idx, R, E, hist);
+  moe_status st = launch_status();
+  if (st != MOE_OK) return st;
+  perm_scan_kernel<<<1, 1024, shE, s>>>(hist, nch, E, counts, offsets, base);
+  st = launch_status();
+  if (st != MOE_OK) return st;
+  perm_scatter_kernel<<<nch, 256, shE, s>>>(idx, R, E, k, base, sorted_rows, inv, x, H, x_perm);
+  return launch_status();
+}

@@ -53,7 +53,16 @@ def irwin_hall_scale(sigma: float) -> np.float32:
 
 
 def normal_f32(seed: int, a: int, b: int, n: int, sigma: float, start: int = 0) -> np.ndarray:
-    """n approximately N(0, sigma^2) fp32 values of stream (a, b)."""
+    """n approximately N(0, sigma^2) fp32 values of stream (a, b) (C twin)."""
+    out = np.empty(n, np.float32)
+    if n:
+        _cpu().synth_normal_f32_cpu(out.ctypes.data, n, 1, a, 0, b, seed,
+                                    float(irwin_hall_scale(sigma)), start)
+    return out
+
+
+def normal_f32_numpy(seed: int, a: int, b: int, n: int, sigma: float, start: int = 0) -> np.ndarray:
+    """Reference numpy form of normal_f32 (slow; pins the C and CUDA twins)."""
     i = np.arange(start, start + n, dtype=np.uint64)
     r = philox4x32_10((i & _MASK32).astype(np.uint32), (i >> np.uint64(32)).astype(np.uint32),
                       np.uint32(a), np.uint32(b), np.uint32(seed), np.uint32(KEY_HI))
@@ -103,3 +112,70 @@ def zipf_bias(seed: int, E: int, s: float = 1.1) -> np.ndarray:
     rng = np.random.Generator(np.random.Philox(key=seed))
     rank = rng.permutation(E) + 1
     return (-s * np.log(rank.astype(np.float64))).astype(np.float32)
+
+
+# ---------------------------------------------------------------- CUDA twin
+import ctypes as _ct
+import os as _os
+import subprocess as _sp
+
+_HERE = _os.path.dirname(_os.path.abspath(__file__))
+_CU = _os.path.join(_HERE, "synth_gen.cu")
+_SO = _os.path.join(_HERE, "libsynth.so")
+_cuda_lib = None
+_C = _os.path.join(_HERE, "synth_cpu.c")
+_CSO = _os.path.join(_HERE, "libsynth_cpu.so")
+_cpu_lib = None
+
+
+def build_cpu(force: bool = False) -> str:
+    if force or not _os.path.exists(_CSO) or _os.path.getmtime(_CSO) < _os.path.getmtime(_C):
+        tmp = _CSO + f".tmp{_os.getpid()}"
+        _sp.check_call(["gcc", "-O3", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-o", tmp, _C])
+        _os.replace(tmp, _CSO)
+    return _CSO
+
+
+def _cpu():
+    global _cpu_lib
+    if _cpu_lib is None:
+        L = _ct.CDLL(build_cpu())
+        L.synth_normal_f32_cpu.restype = None
+        L.synth_normal_f32_cpu.argtypes = [_ct.c_void_p, _ct.c_uint64, _ct.c_int, _ct.c_uint32, _ct.c_uint32,
+                                           _ct.c_uint32, _ct.c_uint32, _ct.c_float, _ct.c_uint64]
+        _cpu_lib = L
+    return _cpu_lib
+
+
+def build_cuda(force: bool = False) -> str:
+    """Compile the CUDA twin of the generator (sm_100a)."""
+    if force or not _os.path.exists(_SO) or _os.path.getmtime(_SO) < _os.path.getmtime(_CU):
+        tmp = _SO + f".tmp{_os.getpid()}"
+        _sp.check_call([_os.environ.get("NVCC", "nvcc"), "-gencode", "arch=compute_100a,code=sm_100a",
+                        "-O3", "-shared", "-Xcompiler", "-fPIC", "-o", tmp, _CU])
+        _os.replace(tmp, _SO)
+    return _SO
+
+
+def _cuda():
+    global _cuda_lib
+    if _cuda_lib is None:
+        L = _ct.CDLL(build_cuda())
+        L.synth_normal_f32.restype = _ct.c_int
+        L.synth_normal_f32.argtypes = [_ct.c_void_p, _ct.c_uint64, _ct.c_int, _ct.c_uint32, _ct.c_uint32,
+                                       _ct.c_uint32, _ct.c_uint32, _ct.c_float, _ct.c_uint64, _ct.c_void_p]
+        _cuda_lib = L
+    return _cuda_lib
+
+
+def cuda_expert_weights(out, seed: int, layer: int, expert0: int, proj: int, sigma: float = 0.02,
+                        stream=None):
+    """Fill torch CUDA fp32 tensor out [count][N][K] with the matrices of experts
+    expert0 .. expert0+count-1 (identical bits to expert_weights())."""
+    import torch
+    count, N, K = out.shape
+    s = torch.cuda.current_stream() if stream is None else stream
+    rc = _cuda().synth_normal_f32(out.data_ptr(), N * K, count, 4 * expert0 + proj, 4, layer, seed,
+                                  float(irwin_hall_scale(sigma)), 0, _ct.c_void_p(s.cuda_stream))
+    if rc:
+        raise RuntimeError(f"synth_normal_f32 failed with CUDA error {rc}")

@@ -1,0 +1,85 @@
+"""GPU parity of the decode path (route -> weight-streaming FFN -> combine)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import quantized_moe_route_b200 as moe
+from moe_testlib import Layer, decode_workspace, ffn_close, u16, to_u16
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_decode(layer, x, logits, k, ws=None):
+    T = x.shape[0]
+    xd = u16(x)
+    ld = torch.from_numpy(np.ascontiguousarray(logits)).cuda()
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    moe.moe_route(ld, k, idx, w)
+    y_rows = torch.full((T * k, layer.H), float("nan"), device="cuda")
+    ws = decode_workspace(T, k, layer.F) if ws is None else ws
+    moe.moe_ffn_w4a16_decode(layer.desc, xd, idx, y_rows, ws)
+    y = torch.empty((T, layer.H), dtype=torch.int16, device="cuda")
+    moe.moe_unpermute_combine(y_rows, w, y)
+    torch.cuda.synchronize()
+    assert moe.moe_device_error() == 0
+    return idx.cpu().numpy(), y_rows.cpu().numpy(), to_u16(y), ws
+
+
+def _check_layer(seed, E, H, F, T, k, logits=None, repeat=1):
+    x = synth.activations_bf16(seed, 0, T, H)
+    if logits is None:
+        logits = synth.router_logits(seed, 0, T, E)
+    oidx, _ = oracle.route(logits, k)
+    layer = Layer(seed, 0, E, H, F, oidx.ravel())
+    idx, y_rows, y, ws = _run_decode(layer, x, logits, k)
+    assert np.array_equal(idx, oidx)
+    _, _, oy_rows, oy = oracle.moe_forward_w4(x, logits, k, layer.canon)
+    ffn_close(y_rows, oy_rows, "y_rows")
+    ffn_close(synth.bf16_bits_to_f32(y), synth.bf16_bits_to_f32(oy), "y")
+    for _ in range(repeat - 1):  # the workspace is left ready for the next call
+        _, y_rows2, y2, ws = _run_decode(layer, x, logits, k, ws)
+        assert np.array_equal(y_rows2, y_rows) and np.array_equal(y2, y)
+
+
+def test_decode_tiny_layer():
+    """1 layer, 8 experts, top-2, hidden 128, width 64, 4 tokens."""
+    _check_layer(0, 8, 128, 64, 4, 2, repeat=3)
+
+
+def test_decode_single_token_full_shape():
+    """256 experts, top-8, hidden 2048, width 512, 1 token."""
+    _check_layer(1, 256, 2048, 512, 1, 8, repeat=2)
+
+
+@pytest.mark.parametrize("T", [3, 16])
+def test_decode_batches(T):
+    _check_layer(2 + T, 64, 1024, 256, T, 8)
+
+
+def test_decode_all_tokens_on_one_expert():
+    """16 tokens all routed to expert 3 first: one expert serves 16 rows (two n8 blocks)."""
+    T, E, k = 16, 32, 4
+    logits = synth.router_logits(7, 0, T, E)
+    logits[:, 3] += 50.0
+    _check_layer(7, E, 512, 128, T, k, logits=logits.astype(np.float32))
+
+
+def test_decode_hand_set_constant_codes_closed_form():
+    """All codes 2, scale 0.5, min -0.5: every weight 0.5; closed-form output."""
+    E, H, F, T, k = 8, 128, 64, 2, 2
+    s = np.full((2 * F, H // 64), np.float16(0.5).view(np.uint16), np.uint16)
+    m = np.full((2 * F, H // 64), np.float16(-0.5).view(np.uint16), np.uint16)
+    gu = (np.full((2 * F, H), 2, np.uint8), s, m)
+    d = (np.full((H, F), 2, np.uint8), s[:H, :1].copy(), m[:H, :1].copy())
+    wts = {e: (gu, d) for e in range(E)}
+    layer = Layer(0, 0, E, H, F, range(E), weights=wts)
+    x = synth.f32_to_bf16_bits(np.full((T, H), 1.0 / 64, np.float32))
+    logits = synth.router_logits(3, 0, T, E)
+    _, y_rows, y, _ = _run_decode(layer, x, logits, k)
+    g = 0.5 * H / 64  # = sum of weights * x
+    h = g / (1 + np.exp(-g)) * g
+    h_bf16 = float(synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(np.array([h], np.float32)))[0])
+    np.testing.assert_allclose(y_rows, 0.5 * F * h_bf16, rtol=1e-6)

@@ -39,6 +39,12 @@ def test_generator_moments_and_determinism():
     assert np.array_equal(c, a[1000:1100])
 
 
+def test_generator_c_twin_matches_numpy_definition():
+    ref = synth.normal_f32_numpy(9, 4 * 17 + 1, 3, 50000, 0.02, start=2 ** 32 - 100)
+    got = synth.normal_f32(9, 4 * 17 + 1, 3, 50000, 0.02, start=2 ** 32 - 100)
+    assert np.array_equal(ref.view(np.uint32), got.view(np.uint32))
+
+
 # ------------------------------------------------------------------ binary16
 def test_f16_decode_exhaustive_matches_numpy():
     bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
