@@ -190,6 +190,30 @@ MOE_API moe_status moe_ffn_w4a16_decode(const moe_w4_layer *layer, const uint16_
                                         void *ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * Allocation-free form of moe_ffn_w4a16_decode (the pages have no counterpart;
+ * this is a library convenience).  Same inputs, outputs and results, but no
+ * workspace argument: the scratch lives in one fixed array of 516 KiB
+ * (4 KiB of counters + 512 KiB of h) inside the library's device memory,
+ * which every GPU that loads the library keeps until the process exits.  It
+ * is for callers that cannot allocate device memory, such as plugins whose
+ * host application owns and budgets all device memory, or programs with a
+ * fixed memory plan that forbids allocation once serving has started.
+ *   - Limit: T * k * F * 4 <= 512 KiB (e.g. T*k = 256 rows at F = 512);
+ *     larger calls return MOE_ERR_WORKSPACE.  Other limits as for
+ *     moe_ffn_w4a16_decode.
+ *   - Allocates nothing: no cudaMalloc, no cudaFree.  Each call clears the
+ *     counters with a cudaMemsetAsync on `stream`, then launches the kernel.
+ *   - The first call on a device looks up the array's device address on that
+ *     (current) device; make that first call before any stream capture.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind: two calls whose executions overlap on the GPU (different
+ *     streams, no ordering between them) race and give wrong results.
+ */
+MOE_API moe_status moe_ffn_w4a16_decode_static(const moe_w4_layer *layer, const uint16_t *x,
+                                               const int32_t *idx, int T, int k, float *y_rows,
+                                               moe_stream_t stream);
+
+/*
  * Prefill: grouped GEMM over experts.  x_perm bf16 [rows][H] holds the rows
  * grouped by expert (from moe_permute), offsets [E+1] (device) delimits the
  * groups.  Writes y_perm bf16 [rows][H] = W_down (SiLU(W_gate x) * W_up x)

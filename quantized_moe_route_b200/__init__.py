@@ -54,6 +54,7 @@ SIGNATURES = {
     "moe_permute": (_i, [_vp, _i, _i, _i, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_decode_workspace_bytes": (_sz, [_i, _i, _i]),
     "moe_ffn_w4a16_decode": (_i, [ctypes.POINTER(moe_w4_layer), _vp, _vp, _i, _i, _vp, _vp, _sz, _vp]),
+    "moe_ffn_w4a16_decode_static": (_i, [ctypes.POINTER(moe_w4_layer), _vp, _vp, _i, _i, _vp, _vp]),
     "moe_prefill_workspace_bytes": (_sz, [_i, _i]),
     "moe_ffn_grouped_prefill": (_i, [ctypes.POINTER(moe_w4_layer), _vp, _vp, _i, _vp, _vp, _sz, _vp]),
     "moe_unpermute_combine": (_i, [_vp, _i, _vp, _vp, _i, _i, _i, _vp, _vp]),
@@ -152,6 +153,13 @@ def moe_ffn_w4a16_decode(layer: moe_w4_layer, x, idx, y_rows, ws, stream=None):
     _check(lib().moe_ffn_w4a16_decode(ctypes.byref(layer), _p(x), _p(idx), T, k, _p(y_rows), _p(ws),
                                       ws.numel() * ws.element_size(), _stream(stream)),
            "moe_ffn_w4a16_decode")
+
+
+def moe_ffn_w4a16_decode_static(layer: moe_w4_layer, x, idx, y_rows, stream=None):
+    """Decode without a workspace (scratch in a fixed library-owned array)."""
+    T, k = idx.shape
+    _check(lib().moe_ffn_w4a16_decode_static(ctypes.byref(layer), _p(x), _p(idx), T, k, _p(y_rows),
+                                             _stream(stream)), "moe_ffn_w4a16_decode_static")
 
 
 def moe_prefill_workspace_bytes(rows, F) -> int:

@@ -526,3 +526,121 @@ extern "C" MOE_API moe_status moe_ffn_w4a16_decode(const moe_w4_layer *layer, co
   }
   return MOE_OK;
 }
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of the decode call.
+//
+// Some callers cannot allocate device memory at all: plugins and embedded
+// hosts whose device memory is owned and budgeted by the host application,
+// and programs with a fixed memory plan that forbids any allocation once they
+// have started serving.  They cannot supply the scratch workspace that
+// moe_ffn_w4a16_decode needs, so this variant keeps its scratch (the per-slot
+// counters and the h buffer) in one fixed array in the library's own device
+// memory instead.  The array is a module global: every GPU that loads the
+// library holds it until the process exits.
+// ---------------------------------------------------------------------------
+namespace moe {
+
+constexpr size_t kStaticFlagBytes = 4096;
+constexpr size_t kStaticHBytes = 512 * 1024;  // T*k*F*4 bytes of h at most
+constexpr size_t kStaticScratchBytes = kStaticFlagBytes + kStaticHBytes;
+
+static __device__ __align__(256) uint8_t g_decode_scratch[kStaticScratchBytes];
+
+// Device address of g_decode_scratch on the current device, looked up once per
+// device (the lookup needs that device to be current).
+static uint8_t *static_scratch_address(moe_status *st) {
+  static uint8_t *addr[64] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= 64) {
+    set_cuda_error(e == cudaSuccess ? cudaErrorInvalidDevice : e);
+    *st = MOE_ERR_CUDA;
+    return nullptr;
+  }
+  if (!addr[dev]) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess || !p) {
+      set_cuda_error(e == cudaSuccess ? cudaErrorInvalidSymbol : e);
+      *st = MOE_ERR_CUDA;
+      return nullptr;
+    }
+    addr[dev] = static_cast<uint8_t *>(p);
+  }
+  *st = MOE_OK;
+  return addr[dev];
+}
+
+}  // namespace moe
+
+extern "C" MOE_API moe_status moe_ffn_w4a16_decode_static(const moe_w4_layer *layer,
+                                                          const uint16_t *x, const int32_t *idx,
+                                                          int T, int k, float *y_rows,
+                                                          moe_stream_t stream) {
+  if (!layer || T < 0 || k <= 0) return MOE_ERR_INVALID_ARG;
+  const int E = layer->E, H = layer->H, F = layer->F;
+  if (E <= 0 || H <= 0 || F <= 0 || k > E) return MOE_ERR_INVALID_ARG;
+  if (H % 64 || F % 64 || E > kDecMaxE || T > kDecMaxTok || T * k > kDecMaxRows)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  // the fixed scratch holds h for at most kStaticHBytes / 4 values
+  if ((size_t)T * k * F * sizeof(float) > kStaticHBytes) return MOE_ERR_WORKSPACE;
+  if (T == 0) return MOE_OK;
+  if (!layer->gate_up || !layer->down || !x || !idx || !y_rows) return MOE_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(layer->gate_up) % 16 ||
+      reinterpret_cast<uintptr_t>(layer->down) % 16 || reinterpret_cast<uintptr_t>(x) % 16)
+    return MOE_ERR_INVALID_ARG;
+
+  moe_status st;
+  uint8_t *scratch = static_scratch_address(&st);
+  if (!scratch) return st;
+  int *err = device_error_word();
+  if (!err) return MOE_ERR_CUDA;
+  // The array keeps whatever the previous call left in it; the counters must
+  // start at zero, so clear them on the caller's stream before the launch.
+  cudaError_t e = cudaMemsetAsync(scratch, 0, kStaticFlagBytes, as_stream(stream));
+  if (e != cudaSuccess) {
+    set_cuda_error(e);
+    return MOE_ERR_CUDA;
+  }
+
+  DecodeArgs a;
+  a.gu = static_cast<const uint8_t *>(layer->gate_up);
+  a.dn = static_cast<const uint8_t *>(layer->down);
+  a.gu_stride = w4_packed_bytes(2 * F, H);
+  a.dn_stride = w4_packed_bytes(H, F);
+  a.x = x;
+  a.idx = idx;
+  a.y_rows = y_rows;
+  a.flags = reinterpret_cast<int *>(scratch);
+  a.hbuf = reinterpret_cast<float *>(scratch + kStaticFlagBytes);
+  a.err = err;
+  a.T = T;
+  a.k = k;
+  a.E = E;
+  a.H = H;
+  a.F = F;
+  const uint32_t itemA = 2u * (H / 64) * kBlkBytes, itemB = 4u * (F / 64) * kBlkBytes;
+  a.stage_bytes = (max(itemA, itemB) + 127u) / 128u * 128u;
+
+  int dev = 0, sms = 0, smem_max = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  int nst = 8;
+  while (nst > 1 && decode_smem_layout(T, H, F, nst, a.stage_bytes).total > (uint32_t)smem_max - 1024)
+    --nst;
+  const DecodeSmem L = decode_smem_layout(T, H, F, nst, a.stage_bytes);
+  if (L.total > (uint32_t)smem_max - 1024) return MOE_ERR_UNSUPPORTED_SHAPE;
+  a.nstages = nst;
+  e = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem_max - 1024);
+  if (e != cudaSuccess) {
+    set_cuda_error(e);
+    return MOE_ERR_CUDA;
+  }
+  const int maxItems = T * k * (F / 16 + H / kDecOutRows);
+  const int grid = max(1, min(sms, maxItems));
+  decode_kernel<<<grid, kDecThreads, L.total, as_stream(stream)>>>(a);
+  return launch_status();
+}
