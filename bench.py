@@ -182,6 +182,8 @@ def layer_inputs(seed, l, T):
 
 
 def run_gpu(args, log):
+    global LAYERS
+    LAYERS = args.layers
     import torch
     import quantized_moe_route_b200 as moe
     world, rank, local = dist_setup()
@@ -191,9 +193,8 @@ def run_gpu(args, log):
     seed = 1000 + rank
     layers = build_layers(LAYERS, seed, log)
     k = TOPK
-    # per-layer device inputs, routing outputs and workspaces
-    xs, ls = [], []
-    uniq = []
+    # per-layer device inputs (activations and router logits of every layer)
+    xs, ls, uniq = [], [], []
     for l in range(LAYERS):
         x, lg = layer_inputs(seed, l, T)
         xs.append(torch.from_numpy(x.view(np.int16)).to(dev))
@@ -215,21 +216,39 @@ def run_gpu(args, log):
             ev[1].record(stream)
         moe.moe_unpermute_combine(y_rows, w, y, stream=stream)
 
-    def capture(steps, first, events=None):
+    def capture(fn, steps, first, events=None):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for i in range(steps):
-                step((first + i) % LAYERS, None if events is None else events[i])
+                if events is None:
+                    fn((first + i) % LAYERS)
+                else:
+                    fn((first + i) % LAYERS, events[i])
         return g
 
+    def run_steps(fn, K, first):
+        """Exactly K steps: full graphs of G steps plus one remainder graph."""
+        G = min(K, args.graph_steps)
+        graphs = []
+        if K // G:
+            graphs.append((capture(fn, G, first), K // G))
+        if K % G:
+            graphs.append((capture(fn, K % G, first + (K // G) * G), 1))
+        return graphs
+
+    def replay(graphs):
+        with torch.cuda.stream(stream):  # a graph replays on the current stream
+            for g, n in graphs:
+                for _ in range(n):
+                    g.replay()
+
     K, W = args.steps, args.warmup
-    # untimed warm-up (eager once, then a graph of W steps)
-    for l in range(min(W, LAYERS)):
+    for l in range(min(W, LAYERS)):  # eager first touches, untimed
         step(l)
     torch.cuda.synchronize()
-    g_warm = capture(W, 0)
-    g_main = capture(K, W)
-    g_warm.replay()
+    g_warm = run_steps(step, W, 0)
+    g_main = run_steps(step, K, W)
+    replay(g_warm)
     torch.cuda.synchronize()
 
     dist_barrier()
@@ -238,30 +257,31 @@ def run_gpu(args, log):
         dist_barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        g_main.replay()
+        replay(g_main)
         e1.record(stream)
         e1.synchronize()
         torch.cuda.synchronize()
         dist_barrier()
-    ms_local = e0.elapsed_time(e1)
-    ms = dist_max(ms_local)
+    ms = dist_max(e0.elapsed_time(e1))
     tokens = K * T * world
     value = tokens / (ms / 1e3)
 
-    # kernel-duration pass: the same K steps with events around each FFN launch
+    # kernel-duration pass: the same kind of steps with events around each FFN launch
+    P = min(K, args.graph_steps)
     evs = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
-           for _ in range(K)]
-    g_prof = capture(K, W, evs)
-    g_prof.replay()
+           for _ in range(P)]
+    g_prof = capture(step, P, W, evs)
+    with torch.cuda.stream(stream):
+        g_prof.replay()
     torch.cuda.synchronize()
-    durs = [a.elapsed_time(b) for a, b in evs]
-    dur_ms = sum(durs) / len(durs)
-    byts = [uniq[(W + i) % LAYERS] * EXPERT_BYTES + T * H * 2 + T * k * 4 + T * k * H * 4 for i in range(K)]
-    alg_bytes = sum(byts) / K
+    dur_ms = sum(a.elapsed_time(b) for a, b in evs) / P
+    alg_bytes = sum(uniq[(W + i) % LAYERS] * EXPERT_BYTES + T * H * 2 + T * k * 4 + T * k * H * 4
+                    for i in range(P)) / P
     peak, peak_kind = peaks()
     achieved = alg_bytes / (dur_ms / 1e3) / 1e9
 
-    # end-to-end through the C ABI with host buffers: H2D inputs, D2H output every step
+    # end to end through the C ABI with host buffers: H2D of the step's inputs
+    # from pinned memory and D2H of its result, every step
     hx = [torch.from_numpy(layer_inputs(seed, l, T)[0].view(np.int16)).pin_memory() for l in range(LAYERS)]
     hl = [torch.from_numpy(layer_inputs(seed, l, T)[1]).pin_memory() for l in range(LAYERS)]
     hy = torch.empty((T, H), dtype=torch.int16).pin_memory()
@@ -276,21 +296,17 @@ def run_gpu(args, log):
         moe.moe_unpermute_combine(y_rows, w, y, stream=stream)
         hy.copy_(y, non_blocking=True)
 
-    ge = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
         for l in range(3):
-            e2e_step(l)
+            e2e_step(l % LAYERS)
     stream.synchronize()
-    with torch.cuda.graph(ge, stream=stream):
-        with torch.cuda.stream(stream):
-            for i in range(K):
-                e2e_step((W + i) % LAYERS)
-    ge.replay()
+    g_e2e = run_steps(e2e_step, K, W)
+    replay(g_e2e)
     torch.cuda.synchronize()
     dist_barrier()
     a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a0.record(stream)
-    ge.replay()
+    replay(g_e2e)
     a1.record(stream)
     a1.synchronize()
     e2e_ms = dist_max(a0.elapsed_time(a1))
@@ -302,8 +318,9 @@ def run_gpu(args, log):
         "dtype": "int4 weights (f16 scale/min), bf16 activations, fp32 accumulate", "data": "synthetic",
         "config": {"workload": WORKLOAD, "experts": E, "top_k": k, "hidden": H, "expert_width": F,
                    "tokens_per_step": T, "resident_layers": LAYERS, "seed": 1000,
-                   "l2": "inputs larger than L2 (18.1 GB resident, 40-layer rotation)",
-                   "parallelism": f"replicas x{world}", "graph": "CUDA graph of K steps, PDL between kernels"},
+                   "l2": f"inputs larger than L2 ({LAYERS}-layer rotation, {LAYERS * E * EXPERT_BYTES / 1e9:.1f} GB)",
+                   "parallelism": f"replicas x{world}",
+                   "launch": f"CUDA graphs of {min(K, args.graph_steps)} steps, PDL into the FFN kernel"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": None, "kernel": "moe::decode_kernel",
                      "peak_kind": peak_kind, "alg_bytes_per_launch": alg_bytes,
@@ -315,9 +332,9 @@ def run_gpu(args, log):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(seed, T, budget_s=args.cpu_seconds, log=log)
+    del g_main, g_warm, g_prof, g_e2e
     if world > 1:
         import torch.distributed as dist
-        del g_main, g_warm, g_prof, ge
         dist.barrier()
         dist.destroy_process_group()
     return out if rank == 0 else None
@@ -401,10 +418,13 @@ def run_reference(args, log):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--steps", type=int, default=100000, help="timed steps")
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--tokens", type=int, default=1)
+    ap.add_argument("--layers", type=int, default=LAYERS,
+                    help="resident layers the steps rotate over (40 = 18.1 GB, larger than L2)")
+    ap.add_argument("--graph-steps", type=int, default=400, help="steps captured per CUDA graph")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quiet", action="store_true")

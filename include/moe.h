@@ -175,10 +175,12 @@ MOE_API moe_status moe_permute(const int32_t *idx, int T, int k, int E, const ui
  * projection.  Source: "drama-rs", "Footprint and speed" (decode is weight
  * streaming GEMVs) and "Experts: where they run" (decode is memory-bandwidth
  * bound); the SwiGLU expert of the Qwen3.5-MoE backbone.
- * Workspace: moe_decode_workspace_bytes(T, k, F); it must be zero-filled
- * before its first use, and every successful call leaves it zero-filled again
- * (so one workspace serves any number of stream-ordered calls).  Calls that
- * share a workspace must not overlap in time.
+ * Workspace: moe_decode_workspace_bytes(T, k, F) bytes (a call counter and
+ * the h handoff buffer), 16-byte aligned.  Zero-fill it once before its
+ * first use; every call leaves it ready for the next stream-ordered call, so
+ * one workspace serves any number of calls.  Calls that share a workspace
+ * must not overlap in time.  After a call that raised the device error word,
+ * zero-fill the workspace again.
  * Requirements: H % 64 == 0, F % 64 == 0, idx values in [0, E), the k
  * experts of a token distinct.  Errors: INVALID_ARG, UNSUPPORTED_SHAPE,
  * WORKSPACE, CUDA.  A device-side wait that times out (it cannot under the
@@ -193,16 +195,19 @@ MOE_API moe_status moe_ffn_w4a16_decode(const moe_w4_layer *layer, const uint16_
  * Allocation-free form of moe_ffn_w4a16_decode (the pages have no counterpart;
  * this is a library convenience).  Same inputs, outputs and results, but no
  * workspace argument: the scratch lives in one fixed array of 516 KiB
- * (4 KiB of counters + 512 KiB of h) inside the library's device memory,
+ * (4 KiB of counter words + 512 KiB of h handoff words) inside the library's
+ * device memory,
  * which every GPU that loads the library keeps until the process exits.  It
  * is for callers that cannot allocate device memory, such as plugins whose
  * host application owns and budgets all device memory, or programs with a
  * fixed memory plan that forbids allocation once serving has started.
- *   - Limit: T * k * F * 4 <= 512 KiB (e.g. T*k = 256 rows at F = 512);
+ *   - Limit: T * k * F * 8 <= 512 KiB (one 8-byte handoff word per h value;
+ *     e.g. T*k = 128 rows at F = 512);
  *     larger calls return MOE_ERR_WORKSPACE.  Other limits as for
  *     moe_ffn_w4a16_decode.
  *   - Allocates nothing: no cudaMalloc, no cudaFree.  Each call clears the
- *     counters with a cudaMemsetAsync on `stream`, then launches the kernel.
+ *     CTA counter word with a cudaMemsetAsync on `stream`, then launches the
+ *     kernel; the call-number word keeps counting across calls.
  *   - The first call on a device looks up the array's device address on that
  *     (current) device; make that first call before any stream capture.
  *   - Every call on a device shares the one array and leaves its contents

@@ -13,8 +13,10 @@ constexpr int kRouteMaxPerLane = 32;  // E <= 1024
 
 // Lane l owns experts l, l + 32, l + 64, ... (coalesced loads).  Each of the
 // k rounds takes the warp-wide maximum (value, then lowest id) of the
-// not-yet-taken experts.  Weights are exp(l_j - max) / sum over the selected
-// of exp(l_j' - max): the renormalised softmax restricted to the selection.
+// not-yet-taken experts; only the winning lane rescans its own entries.
+// Weights are exp(l_j - max) / sum over the selected of exp(l_j' - max): the
+// renormalised softmax restricted to the selection.
+template <int PER>
 __global__ void route_kernel(const float *__restrict__ logits, int T, int E, int k,
                              int32_t *__restrict__ idx, float *__restrict__ w) {
   const int warps = blockDim.x / 32;
@@ -22,45 +24,51 @@ __global__ void route_kernel(const float *__restrict__ logits, int T, int E, int
   if (t >= T) return;
   const int lane = threadIdx.x & 31;
   const float *l = logits + (size_t)t * E;
-  float v[kRouteMaxPerLane];
-  const int per = (E + 31) / 32;
+  float v[PER];
 #pragma unroll
-  for (int i = 0; i < kRouteMaxPerLane; ++i) {
-    int e = lane + 32 * i;
-    v[i] = (i < per && e < E) ? l[e] : -INFINITY;
+  for (int i = 0; i < PER; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = e < E ? l[e] : -INFINITY;
   }
   uint32_t taken = 0;  // bit i: expert lane + 32 i already selected
-  float top = 0.f, denom = 0.f, my_w = 0.f;
-  int my_idx = 0;
-  for (int j = 0; j < k; ++j) {
-    // local best among the lane's untaken entries (lowest id on ties: the
-    // entries are visited in increasing id, strict > keeps the first)
-    float bv = -INFINITY;
-    int bi = -1;
+  // local best of the untaken entries: entries visited in increasing id and
+  // strict > keeps the lowest id among equals; -1 = nothing left
+  auto local_best = [&](float &bv, int &bi) {
+    bv = -INFINITY;
+    bi = -1;
 #pragma unroll
-    for (int i = 0; i < kRouteMaxPerLane; ++i) {
-      int e = lane + 32 * i;
-      if (i < per && e < E && !((taken >> i) & 1u) && (bi < 0 || v[i] > bv)) {
+    for (int i = 0; i < PER; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !((taken >> i) & 1u) && (bi < 0 || v[i] > bv)) {
         bv = v[i];
         bi = e;
       }
     }
-    // warp arg-max: larger value, then lower id; lanes with nothing left carry
-    // id = INT_MAX so they never win
+  };
+  float bv;
+  int bi;
+  local_best(bv, bi);
+  float top = 0.f, denom = 0.f, my_w = 0.f;
+  int my_idx = 0;
+  for (int j = 0; j < k; ++j) {
+    // warp arg-max: larger value, then lower id; exhausted lanes carry INT_MAX
     float rv = bv;
     int ri = bi < 0 ? 0x7fffffff : bi;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      float ov = __shfl_xor_sync(0xffffffffu, rv, o);
-      int oi = __shfl_xor_sync(0xffffffffu, ri, o);
+      const float ov = __shfl_xor_sync(0xffffffffu, rv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, ri, o);
       if (oi != 0x7fffffff && (ri == 0x7fffffff || ov > rv || (ov == rv && oi < ri))) {
         rv = ov;
         ri = oi;
       }
     }
-    if ((ri & 31) == lane) taken |= 1u << (ri >> 5);
+    if ((ri & 31) == lane) {
+      taken |= 1u << (ri >> 5);
+      local_best(bv, bi);
+    }
     if (j == 0) top = rv;
-    float ex = expf(rv - top);
+    const float ex = expf(rv - top);
     denom += ex;
     if (lane == j) {
       my_idx = ri;
@@ -83,7 +91,15 @@ extern "C" MOE_API moe_status moe_route(const float *logits, int T, int E, int k
   if (E > 32 * kRouteMaxPerLane || k > 32) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (T == 0) return MOE_OK;
   if (!logits || !idx || !w) return MOE_ERR_INVALID_ARG;
-  const int threads = 256, warps = threads / 32;
-  route_kernel<<<(T + warps - 1) / warps, threads, 0, as_stream(stream)>>>(logits, T, E, k, idx, w);
+  const int threads = 128, warps = threads / 32;
+  const dim3 grid((T + warps - 1) / warps);
+  cudaStream_t s = as_stream(stream);
+  const int per = (E + 31) / 32;
+  if (per <= 1) route_kernel<1><<<grid, threads, 0, s>>>(logits, T, E, k, idx, w);
+  else if (per <= 2) route_kernel<2><<<grid, threads, 0, s>>>(logits, T, E, k, idx, w);
+  else if (per <= 4) route_kernel<4><<<grid, threads, 0, s>>>(logits, T, E, k, idx, w);
+  else if (per <= 8) route_kernel<8><<<grid, threads, 0, s>>>(logits, T, E, k, idx, w);
+  else if (per <= 16) route_kernel<16><<<grid, threads, 0, s>>>(logits, T, E, k, idx, w);
+  else route_kernel<32><<<grid, threads, 0, s>>>(logits, T, E, k, idx, w);
   return launch_status();
 }

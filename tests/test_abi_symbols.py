@@ -36,4 +36,4 @@ def test_host_only_queries():
     assert L.moe_w4_packed_bytes(1024, 2048) == 1179648
     assert L.moe_status_string(2) == b"MOE_ERR_UNSUPPORTED_SHAPE"
     assert L.moe_version().startswith(b"moe-w4-b200")
-    assert L.moe_decode_workspace_bytes(1, 8, 512) >= 8 * 512 * 4
+    assert L.moe_decode_workspace_bytes(1, 8, 512) >= 8 * 512 * 8  # one 8-byte h word per value

@@ -83,3 +83,18 @@ def test_decode_hand_set_constant_codes_closed_form():
     h = g / (1 + np.exp(-g)) * g
     h_bf16 = float(synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(np.array([h], np.float32)))[0])
     np.testing.assert_allclose(y_rows, 0.5 * F * h_bf16, rtol=1e-6)
+
+
+def test_decode_workspace_reuse_across_batch_sizes():
+    """One workspace serves calls of different batch sizes in a row: stale h
+    words of earlier calls never pass for the current call's."""
+    E, H, F, k = 64, 512, 128, 8
+    ws = decode_workspace(16, k, F)
+    for T, seed in [(16, 40), (1, 41), (16, 42), (3, 43)]:
+        x = synth.activations_bf16(seed, 0, T, H)
+        logits = synth.router_logits(seed, 0, T, E)
+        oidx, _ = oracle.route(logits, k)
+        layer = Layer(seed, 0, E, H, F, oidx.ravel())
+        idx, y_rows, y, ws = _run_decode(layer, x, logits, k, ws)
+        _, _, oy_rows, oy = oracle.moe_forward_w4(x, logits, k, layer.canon)
+        ffn_close(y_rows, oy_rows, f"y_rows T={T}")

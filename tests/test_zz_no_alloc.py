@@ -58,8 +58,8 @@ def test_static_scratch_decode_matches_workspace_decode(E, H, F, T, k):
 def test_static_scratch_rejects_sizes_over_its_limit():
     L = moe.lib()
     buf = torch.zeros(64, dtype=torch.uint8, device="cuda")
-    desc = moe.moe_w4_layer(256, 2048, 2048, buf.data_ptr(), buf.data_ptr())
-    # 16 tokens x 8 rows x F=2048 x 4 B = 1 MiB of h > 512 KiB
+    desc = moe.moe_w4_layer(256, 2048, 4096, buf.data_ptr(), buf.data_ptr())
+    # 16 tokens x 8 rows x F=4096 x 8 B = 4 MiB of h words > 512 KiB
     st = L.moe_ffn_w4a16_decode_static(ctypes.byref(desc), buf.data_ptr(), buf.data_ptr(), 16, 8,
                                        buf.data_ptr(), None)
     assert st == moe.MOE_ERR_WORKSPACE
