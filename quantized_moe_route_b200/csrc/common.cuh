@@ -114,6 +114,12 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
   return false;
 }
 
+// Order this thread's generic-proxy shared-memory accesses before later
+// async-proxy accesses (bulk/TMA copies, tensor-core operand reads).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // 1-D bulk copy global -> shared, completion counted on an mbarrier (no
 // multicast).  Addresses 16-byte aligned, size a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,

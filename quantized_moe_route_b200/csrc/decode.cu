@@ -31,8 +31,10 @@
 
 namespace moe {
 
-constexpr int kDecWarps = 8;
+constexpr int kDecWarps = 16;             // two teams of eight warps
 constexpr int kDecThreads = kDecWarps * 32;
+constexpr int kTeamWarps = 8;
+constexpr int kTeamThreads = kTeamWarps * 32;
 constexpr int kDecMaxTok = 16;   // tokens per expert per call (two n8 blocks)
 constexpr int kDecMaxRows = 256; // T * k
 constexpr int kDecMaxE = 1024;
@@ -50,16 +52,29 @@ struct DecodeArgs {
   unsigned int *ctrl;        // [0] last epoch, [1] CTAs done
   int *err;
   int T, k, E, H, F;
-  int nstages;
+  int nstages;               // even: team t owns the stages s = t (mod 2)
   uint32_t stage_bytes;
+  uint32_t h_off;            // offset of a B item's h tile inside its stage
 };
 
 struct DecodeSmem {
   // byte offsets into dynamic shared memory
-  uint32_t stages, x, xsum, red, h, hsum, bars, meta, total;
+  uint32_t stages, x, xsum, hsum, bars, meta, total;
 };
 
 __host__ __device__ inline int dec_ntok_cols(int T) { return T > 8 ? 16 : 8; }
+
+// Stage buffer: an A item's weights, or a B item's weights followed by its h
+// tile; after the compute the same buffer holds the cross-warp partial sums.
+__host__ __device__ inline uint32_t dec_stage_bytes(int T, int H, int F, uint32_t *h_off) {
+  const uint32_t itemA = 2u * (H / 64) * kBlkBytes, itemB = 4u * (F / 64) * kBlkBytes;
+  const uint32_t hoff = (itemB + 127u) / 128u * 128u;
+  const uint32_t red = kTeamWarps * 2u * 16u * (uint32_t)dec_ntok_cols(T) * 4u;
+  uint32_t b = itemA > hoff + (uint32_t)T * F * 2u ? itemA : hoff + (uint32_t)T * F * 2u;
+  b = b > red ? b : red;
+  *h_off = hoff;
+  return (b + 127u) / 128u * 128u;
+}
 
 __host__ __device__ inline DecodeSmem decode_smem_layout(int T, int H, int F, int nstages,
                                                          uint32_t stage_bytes) {
@@ -71,15 +86,12 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int T, int H, int F, in
     o += bytes;
     return at;
   };
-  const uint32_t nt = (uint32_t)dec_ntok_cols(T);
   L.stages = take((uint32_t)nstages * stage_bytes, 128);
   L.x = take((uint32_t)T * H * 2, 16);
   L.xsum = take((uint32_t)T * (H / 64) * 4, 16);
-  L.red = take(kDecWarps * 2 * 16 * nt * 4, 16);
-  L.h = take((uint32_t)T * F * 2, 16);
-  L.hsum = take((uint32_t)T * (F / 64) * 4, 16);
+  L.hsum = take(2u * T * (F / 64) * 4, 16);
   L.bars = take((uint32_t)nstages * 8, 8);
-  L.meta = take(2048 * 4, 16);
+  L.meta = take(3200 * 4, 16);  // routing tables + 256 x 8 row-set words
   L.total = o;
   return L;
 }
@@ -87,6 +99,21 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int T, int H, int F, in
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Barriers of one team (named barrier 1 + team, 256 threads).
+__device__ __forceinline__ void team_sync(int id) {
+  asm volatile("bar.sync %0, 256;" ::"r"(id) : "memory");
+}
+__device__ __forceinline__ bool team_or(int id, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, 256, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id)
+      : "memory");
+  return r != 0;
 }
 
 __device__ __forceinline__ int warp_inclusive_scan(int v) {
@@ -232,11 +259,11 @@ __device__ __forceinline__ void frag_to_red(float *red, const float acc[2][4], i
 
 // Sums of 64 consecutive bf16 values: rows [nrows][ld] -> out[n][g] for the
 // first ngroups groups; eight threads per sum, one 16-byte vector each.
+// `t` / `nthreads`: this thread's index among the participating threads.
 __device__ __forceinline__ void group_sums(const uint16_t *rows, int nrows, int ld, int ngroups,
-                                           float *out) {
+                                           float *out, int t, int nthreads) {
   const int tasks = nrows * ngroups * 8;
-  for (int v = threadIdx.x; v < ((tasks + kDecThreads - 1) / kDecThreads) * kDecThreads;
-       v += kDecThreads) {
+  for (int v = t; v < ((tasks + nthreads - 1) / nthreads) * nthreads; v += nthreads) {
     float s = 0.f;
     const int task = v >> 3, part = v & 7;
     if (v < tasks) {
@@ -253,30 +280,27 @@ __device__ __forceinline__ void group_sums(const uint16_t *rows, int nrows, int 
   }
 }
 
-__global__ void __launch_bounds__(kDecThreads) decode_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const DecodeSmem L = decode_smem_layout(a.T, a.H, a.F, a.nstages, a.stage_bytes);
   uint16_t *x_s = reinterpret_cast<uint16_t *>(smem + L.x);
   float *xsum_s = reinterpret_cast<float *>(smem + L.xsum);
-  float *red_s = reinterpret_cast<float *>(smem + L.red);
-  uint16_t *h_s = reinterpret_cast<uint16_t *>(smem + L.h);
-  float *hsum_s = reinterpret_cast<float *>(smem + L.hsum);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
   int *meta = reinterpret_cast<int *>(smem + L.meta);
   uint32_t *emask = reinterpret_cast<uint32_t *>(meta);  // [32] expert presence bits
   int *wbase = meta + 32;                                 // [32] slots before word w
   int *slot_expert = meta + 64;                           // [256]
-  int *run = slot_expert + kDecMaxRows;                   // [256] rows per slot
-  int *slot_off = run + kDecMaxRows;                      // [257]
+  int *slot_off = slot_expert + kDecMaxRows;              // [257]
   int *slot_rows = slot_off + kDecMaxRows + 1;            // [256] row ids grouped by slot
   int *ridx = slot_rows + kDecMaxRows;                    // [256] expert of row
-  int *row_slot = ridx + kDecMaxRows;                     // [256]
-  int *row_rank = row_slot + kDecMaxRows;                 // [256]
-  int *misc = row_rank + kDecMaxRows;                     // [0] U, [1] abort, [2] epoch
-  __shared__ int tok_list[kDecMaxTok];
+  int *misc = ridx + kDecMaxRows;                         // [0] U, [1] abort, [2] epoch
+  uint32_t *rmask = reinterpret_cast<uint32_t *>(misc + 8);  // [256 slots][8 words] rows of a slot
+  __shared__ int tok_lists[2][kDecMaxTok];
   __shared__ int ident[kDecMaxTok];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int team = warp / kTeamWarps, tw = warp % kTeamWarps, ttid = tid % kTeamThreads;
+  const int bar_id = 1 + team;
   const int T = a.T, k = a.k, E = a.E, H = a.H, F = a.F;
   const int R = T * k, Gh = H / 64, Gf = F / 64, nt = dec_ntok_cols(T);
   const uint32_t stripA = (uint32_t)Gh * kBlkBytes, stripB = (uint32_t)Gf * kBlkBytes;
@@ -288,8 +312,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(DecodeArgs a) {
   }
   if (tid < kDecMaxTok) ident[tid] = tid;
   if (tid < 32) emask[tid] = 0u;
-  static_assert(kDecThreads == kDecMaxRows, "one thread per routed row");
-  run[tid] = 0;
+  for (int i = tid; i < kDecMaxRows * 8; i += kDecThreads) rmask[i] = 0u;
   pdl_wait();  // inputs of this call may come from the previous kernel
   if (tid == 0) {
     unsigned int ep = a.ctrl[0] + 1u;  // this call's epoch; never 0 (zeroed words never match)
@@ -357,27 +380,28 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(DecodeArgs a) {
   }
   __syncthreads();
   pdl_launch_dependents();
-  // rows of each slot in increasing row id; activation group sums
+  // rows of each slot as a bit set; activation group sums
+  int my_slot = 0;
   if (tid < R) {
     const int e = ridx[tid];
-    const int slot = wbase[e >> 5] + __popc(emask[e >> 5] & ((1u << (e & 31)) - 1u));
-    int rank = 0;
-    for (int r = 0; r < tid; ++r) rank += (ridx[r] == e);
-    row_slot[tid] = slot;
-    row_rank[tid] = rank;
-    atomicAdd(&run[slot], 1);
+    my_slot = wbase[e >> 5] + __popc(emask[e >> 5] & ((1u << (e & 31)) - 1u));
+    atomicOr(&rmask[my_slot * 8 + (tid >> 5)], 1u << (tid & 31));
   }
-  group_sums(x_s, T, H, Gh, xsum_s);
+  group_sums(x_s, T, H, Gh, xsum_s, tid, kDecThreads);
   __syncthreads();
   const int U = misc[0];
   const unsigned int epoch = (unsigned int)misc[2];
-  if (warp == 0) {  // exclusive scan of the U slot sizes, 8 slots per lane
+  if (warp == 0) {  // slot sizes and their exclusive scan, 8 slots per lane
     int v[8], s = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int sl = 8 * lane + i;
-      v[i] = sl < U ? run[sl] : 0;
-      s += v[i];
+      int c = 0;
+      if (sl < U)
+#pragma unroll
+        for (int w = 0; w < 8; ++w) c += __popc(rmask[sl * 8 + w]);
+      v[i] = c;
+      s += c;
     }
     int ex = warp_inclusive_scan(s) - s;
 #pragma unroll
@@ -389,14 +413,22 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(DecodeArgs a) {
     if (lane == 31) slot_off[U] = ex;
   }
   __syncthreads();
-  if (tid < R) slot_rows[slot_off[row_slot[tid]] + row_rank[tid]] = tid;
+  if (tid < R) {  // rank of this row among its slot's rows, in row order
+    int rank = __popc(rmask[my_slot * 8 + (tid >> 5)] & ((1u << (tid & 31)) - 1u));
+    for (int w = 0; w < (tid >> 5); ++w) rank += __popc(rmask[my_slot * 8 + w]);
+    slot_rows[slot_off[my_slot] + rank] = tid;
+  }
   __syncthreads();
 
   const int nA = U * (F / 16), nItems = nA + U * (H / kDecOutRows);
   const int myCount = (int)blockIdx.x < nItems ? (nItems - 1 - (int)blockIdx.x) / G + 1 : 0;
   const uint64_t pol = policy_evict_first();
+  int *tok_list = tok_lists[team];
+  float *hsum_s = reinterpret_cast<float *>(smem + L.hsum) + (size_t)team * T * Gf;
 
-  for (int q = 0; q < myCount; ++q) {
+  // ---- team `team` runs the CTA's items q = team, team + 2, ...
+  bool aborted = false;
+  for (int q = team; q < myCount; q += 2) {
     const int item = blockIdx.x + q * G;
     const int stage = q % a.nstages;
     const uint32_t parity = (uint32_t)(q / a.nstages) & 1u;
@@ -404,78 +436,65 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(DecodeArgs a) {
     int slot, sub;
     item_of(item, nA, &isA, &slot, &sub);
     const int r0 = slot_off[slot], ntok = slot_off[slot + 1] - r0;
-    if (tid < kDecMaxTok) tok_list[tid] = tid < ntok ? slot_rows[r0 + tid] / k : 0;
+    uint8_t *st = smem + L.stages + (size_t)stage * a.stage_bytes;
+    if (ttid < kDecMaxTok) tok_list[ttid] = ttid < ntok ? slot_rows[r0 + ttid] / k : 0;
+    uint16_t *h_s = reinterpret_cast<uint16_t *>(st + a.h_off);
 
     if (!isA) {
       // B item: poll this slot's h words until all carry this call's epoch
-      // (bounded: only a broken contract waits for seconds), then bf16 tile
+      // (bounded: only a broken contract waits for seconds), into the bf16
+      // tile that sits behind the weights in this stage
       const int words = ntok * F;
       uint32_t spins = 0;
       bool ready = false;
       while (true) {
         bool mine = true;
-        for (int v = tid; v < words; v += kDecThreads) {
+        for (int v = ttid; v < words; v += kTeamThreads) {
           const int n = v / F, f = v % F;
           const unsigned long long w =
               ld_relaxed_u64(a.hbuf + (size_t)slot_rows[r0 + n] * F + f);
           if ((unsigned int)(w & 0xFFFFFFFFull) != epoch) mine = false;
           else h_s[(size_t)n * F + f] = (uint16_t)(w >> 32);
         }
-        ready = !__syncthreads_or(!mine);
+        ready = !team_or(bar_id, !mine);
         if (ready || ++spins > (1u << 20)) break;
         __nanosleep(100);
       }
       if (!ready) {
-        if (tid == 0) {
-          atomicExch(a.err, DEVERR_DECODE_H_WAIT);
-          misc[1] = 1;
-        }
+        if (ttid == 0) atomicExch(a.err, DEVERR_DECODE_H_WAIT);
+        aborted = true;
         break;
       }
-      group_sums(h_s, ntok, F, Gf, hsum_s);
+      group_sums(h_s, ntok, F, Gf, hsum_s, ttid, kTeamThreads);
     }
     // wait for this item's weights (every thread observes the barrier)
     const bool landed = mbar_wait_bounded(&bars[stage], parity, 1u << 26);
-    if (__syncthreads_or(!landed)) {  // only a copy stalled for seconds gets here
-      if (tid == 0) {
-        atomicExch(a.err, DEVERR_DECODE_H_WAIT);
-        misc[1] = 1;
-      }
+    if (team_or(bar_id, !landed)) {  // only a copy stalled for seconds gets here
+      if (ttid == 0) atomicExch(a.err, DEVERR_DECODE_H_WAIT);
+      aborted = true;
       break;
     }
-    const uint8_t *st = smem + L.stages + (size_t)stage * a.stage_bytes;
     const int nbmax = ntok > 8 ? 2 : 1;
+    float *red = reinterpret_cast<float *>(st);  // reused once the weights are consumed
     if (isA) {
       float acc[2][2][4] = {};
       const uint8_t *base[2] = {st, st + stripA};
       if (nbmax == 2)
-        warp_groups<2, 2>(base, warp, kDecWarps, Gh, x_s, H, tok_list, ntok, xsum_s, Gh, acc);
+        warp_groups<2, 2>(base, tw, kTeamWarps, Gh, x_s, H, tok_list, ntok, xsum_s, Gh, acc);
       else
-        warp_groups<1, 2>(base, warp, kDecWarps, Gh, x_s, H, tok_list, ntok, xsum_s, Gh, acc);
-      frag_to_red(red_s + (size_t)(warp * 2 + 0) * 16 * nt, acc[0], nbmax, nt);
-      frag_to_red(red_s + (size_t)(warp * 2 + 1) * 16 * nt, acc[1], nbmax, nt);
-    } else {
-      // warp -> strip (warp & 3), groups of parity (warp >> 2)
-      float acc[1][2][4] = {};
-      const uint8_t *base[1] = {st + (size_t)(warp & 3) * stripB};
-      if (nbmax == 2)
-        warp_groups<2, 1>(base, warp >> 2, 2, Gf, h_s, F, ident, ntok, hsum_s, Gf, acc);
-      else
-        warp_groups<1, 1>(base, warp >> 2, 2, Gf, h_s, F, ident, ntok, hsum_s, Gf, acc);
-      frag_to_red(red_s + (size_t)warp * 16 * nt, acc[0], nbmax, nt);
-    }
-    __syncthreads();
-    // the stage is free again: refill it with item q + nstages
-    if (tid == 0 && q + a.nstages < myCount) issue(blockIdx.x + (q + a.nstages) * G, nA, stage, pol);
-    if (isA) {
-      // reduce over warps: thread -> (row, token); h = SiLU(g) * u
-      const int row = tid >> 4, n = tid & 15;
+        warp_groups<1, 2>(base, tw, kTeamWarps, Gh, x_s, H, tok_list, ntok, xsum_s, Gh, acc);
+      team_sync(bar_id);  // all weights read
+      frag_to_red(red + (size_t)(tw * 2 + 0) * 16 * nt, acc[0], nbmax, nt);
+      frag_to_red(red + (size_t)(tw * 2 + 1) * 16 * nt, acc[1], nbmax, nt);
+      team_sync(bar_id);
+      // thread -> (row, token); h = SiLU(g) * u
+      const int row = ttid >> 4, n = ttid & 15;
       if (n < ntok) {
         float g = 0.f, u = 0.f;
 #pragma unroll
-        for (int w = 0; w < kDecWarps; ++w) {
-          g += red_s[(size_t)(w * 2 + 0) * 16 * nt + row * nt + n];
-          u += red_s[(size_t)(w * 2 + 1) * 16 * nt + row * nt + n];
+        for (int w = 0; w < kTeamWarps; ++w) {
+          g += red[(size_t)(w * 2 + 0) * 16 * nt + row * nt + n];
+          u += red[(size_t)(w * 2 + 1) * 16 * nt + row * nt + n];
         }
         const float h = g / (1.0f + expf(-g)) * u;
         const unsigned long long wv =
@@ -483,22 +502,37 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(DecodeArgs a) {
         a.hbuf[(size_t)slot_rows[r0 + n] * F + 16 * sub + row] = wv;
       }
     } else {
-      for (int v = tid; v < 4 * 16 * nt; v += kDecThreads) {
+      // warp -> strip (tw & 3), groups of parity (tw >> 2)
+      float acc[1][2][4] = {};
+      const uint8_t *base[1] = {st + (size_t)(tw & 3) * stripB};
+      if (nbmax == 2)
+        warp_groups<2, 1>(base, tw >> 2, 2, Gf, h_s, F, ident, ntok, hsum_s, Gf, acc);
+      else
+        warp_groups<1, 1>(base, tw >> 2, 2, Gf, h_s, F, ident, ntok, hsum_s, Gf, acc);
+      team_sync(bar_id);  // all weights read
+      frag_to_red(red + (size_t)tw * 16 * nt, acc[0], nbmax, nt);
+      team_sync(bar_id);
+      for (int v = ttid; v < 4 * 16 * nt; v += kTeamThreads) {
         const int strip = v / (16 * nt), rem = v % (16 * nt);
         const int row = rem / nt, n = rem % nt;
         if (n < ntok) {
-          const float y = red_s[(size_t)strip * 16 * nt + rem] + red_s[(size_t)(strip + 4) * 16 * nt + rem];
+          const float y = red[(size_t)strip * 16 * nt + rem] + red[(size_t)(strip + 4) * 16 * nt + rem];
           a.y_rows[(size_t)slot_rows[r0 + n] * H + kDecOutRows * sub + 16 * strip + row] = y;
         }
       }
     }
-    __syncthreads();
+    // generic-proxy writes to this stage are done; the next copy into it is
+    // an async-proxy write
+    fence_proxy_async_smem();
+    team_sync(bar_id);
+    if (ttid == 0 && q + a.nstages < myCount) issue(blockIdx.x + (q + a.nstages) * G, nA, stage, pol);
   }
 
-  // ---- aborted: let in-flight copies land before the CTA exits
-  if (misc[1] && tid == 0) {
-    for (int s = 0; s < a.nstages; ++s) mbar_wait_bounded(&bars[s], 0, 1u << 20);
+  // ---- aborted: let this team's in-flight copies land before leaving
+  if (aborted && ttid == 0) {
+    for (int s = team; s < a.nstages; s += 2) mbar_wait_bounded(&bars[s], 0, 1u << 20);
   }
+  __syncthreads();
   // ---- last CTA out records this call's epoch for the next call
   if (tid == 0) {
     const unsigned int done = atomicAdd(&a.ctrl[1], 1u);
@@ -514,35 +548,30 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(DecodeArgs a) {
 // CTAs); as many weight stages as fit.
 static moe_status decode_launch(DecodeArgs &a, bool pdl, cudaStream_t stream) {
   const int H = a.H, F = a.F, T = a.T, k = a.k;
-  const uint32_t itemA = 2u * (H / 64) * kBlkBytes, itemB = 4u * (F / 64) * kBlkBytes;
-  a.stage_bytes = (max(itemA, itemB) + 127u) / 128u * 128u;
+  a.stage_bytes = dec_stage_bytes(T, H, F, &a.h_off);
   int dev = 0, sms = 0, smem_max = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  const uint32_t cap1 = (uint32_t)smem_max - 1024, cap2 = cap1 / 2 - 1024;
-  int nst = 8;
-  uint32_t cap = cap2;
-  if (decode_smem_layout(T, H, F, 2, a.stage_bytes).total > cap2) cap = cap1;
-  while (nst > 1 && decode_smem_layout(T, H, F, nst, a.stage_bytes).total > cap) --nst;
+  const uint32_t cap = (uint32_t)smem_max - 1024;
+  int nst = 8;  // even: the two teams own alternate stages
+  while (nst > 2 && decode_smem_layout(T, H, F, nst, a.stage_bytes).total > cap) nst -= 2;
   const DecodeSmem L = decode_smem_layout(T, H, F, nst, a.stage_bytes);
-  if (L.total > cap1) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (L.total > cap) return MOE_ERR_UNSUPPORTED_SHAPE;
   a.nstages = nst;
   static bool attr_done[64] = {false};
   if (dev < 64 && !attr_done[dev]) {
     cudaError_t e = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)cap1);
+                                         (int)cap);
     if (e != cudaSuccess) {
       set_cuda_error(e);
       return MOE_ERR_CUDA;
     }
     attr_done[dev] = true;
   }
-  int per_sm = 0;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel, kDecThreads, L.total);
-  per_sm = max(1, min(per_sm, 2));
+  // one CTA per SM, all resident (B items wait on A items of other CTAs)
   const int maxItems = T * k * (F / 16 + H / kDecOutRows);
-  const int grid = max(1, min(sms * per_sm, maxItems));
+  const int grid = max(1, min(sms, (maxItems + 1) / 2));
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);

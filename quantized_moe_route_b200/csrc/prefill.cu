@@ -1,11 +1,467 @@
-// prefill.cu -- grouped expert FFN on the tensor cores (tcgen05).
+// prefill.cu -- grouped expert FFN on the 5th-generation tensor cores.
+//
+// Prefill groups the rows of a batch by routed expert ("drama-rs", sections
+// "Apple Silicon (MLX)" and "Layout": prefill runs a grouped MoE); every
+// expert's rows then form a dense contraction with that expert's weights.
+// Two launches of one kernel template:
+//   gate/up:  D_gate, D_up [128 features][BN rows] = W [128][H] . X[BN][H]^T,
+//             epilogue h = SiLU(D_gate) * D_up -> bf16 workspace [rows][F]
+//   down:     D [128 outputs][BN rows] = W_down [128][F] . h[BN][F]^T
+//             epilogue -> y_perm bf16 [rows][H]
+// The weights are the MMA's A operand (M = 128 rows of one matrix), the rows
+// of an expert its B operand (N = BN tokens), so a few-row expert wastes N,
+// not M.
+//
+// Per 64-channel k block (one quantisation group):
+//   producer warp:   bulk copies of the packed int4 blocks, TMA (128-byte
+//                    swizzle) of the activation tile
+//   dequant warps:   int4 -> bf16 (fp32 q*s+m, rounded to nearest even) into
+//                    the 128-byte-swizzled K-major smem layout the MMA reads
+//   MMA thread:      tcgen05.mma kind::f16 (bf16 x bf16 -> fp32 in tensor
+//                    memory), four k16 steps per block, commit -> stage free
+// then the dequant warps run the epilogue from tensor memory (tcgen05.ld).
+// Every wait is bounded; a timeout raises the device error word.
+#include <cuda.h>
+
 #include "common.cuh"
+
+namespace moe {
+
+constexpr int kPfThreads = 192;  // warp 0 producer, warp 1 MMA, warps 2..5 dequant + epilogue
+constexpr int kPfBM = 128;       // weight rows per matrix per tile
+constexpr int kPfBN = 128;       // rows (tokens) per tile
+constexpr int kPfBK = 64;        // k block = one quantisation group
+constexpr uint32_t kPfWaitLimit = 1u << 24;
+
+template <bool kGU>
+struct PfCfg {
+  static constexpr int kMats = kGU ? 2 : 1;
+  static constexpr uint32_t kRawBytes = kMats * 8 * kBlkBytes;              // 8 strips per matrix
+  static constexpr uint32_t kABytes = kMats * kPfBM * kPfBK * 2;            // bf16 tiles
+  static constexpr uint32_t kBBytes = kPfBN * kPfBK * 2;                    // activation tile
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes + ((kRawBytes + 1023) / 1024) * 1024;
+  static constexpr int kStages = kGU ? 3 : 5;
+  static constexpr uint32_t kTmemCols = kGU ? 2 * kPfBN : kPfBN;  // 256 or 128 (powers of two)
+  // stage layout: [A tiles][B tile][raw int4], all 1024-aligned
+  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 /*align slack*/ + 4096;
+};
+
+struct PrefillArgs {
+  const uint8_t *w;        // expert weights (gate_up or down), expert e at e * w_stride
+  size_t w_stride;
+  const int32_t *offsets;  // [E + 1]
+  uint16_t *out;           // gate/up: h [rows][F]; down: y_perm [rows][H]
+  int *err;
+  int E, K, rows;
+  int n_sub;               // weight tiles per row chunk: F/128 (gate/up) or H/128 (down)
+  int ld_out;              // F (gate/up) or H (down)
+  int F;                   // gate/up: features per matrix (strip index of the up half)
+};
+
+// ---------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int c0, int c1,
+                                            uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t v[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 bytes in 8-row (1024-byte) atoms.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);        // start address
+  d |= (uint64_t)1u << 16;                        // leading byte offset (unused for this layout)
+  d |= (uint64_t)(1024u >> 4) << 32;              // stride byte offset: next 8-row atom
+  d |= (uint64_t)1u << 46;                        // descriptor version (sm_100)
+  d |= (uint64_t)2u << 61;                        // 128-byte swizzle
+  return d;
+}
+// Instruction descriptor of kind::f16: bf16 A and B, fp32 D, both K-major,
+// M = 128, N = n.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kPfBM >> 4) << 24);
+}
+
+// Byte offset of element (row, k) (k even) of a 128-row x 64-k bf16 tile in
+// the 128-byte-swizzled K-major layout.
+__device__ __forceinline__ uint32_t sw128_offset(int row, int k) {
+  return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((((k >> 3) ^ (row & 7)) << 4) | ((k & 7) << 1)));
+}
+
+__device__ __forceinline__ float code_to_f32(uint32_t w, int shift) {
+  return __uint_as_float(((w >> shift) & 0xFu) | 0x4B000000u) - 8388608.0f;
+}
+
+// ---------------------------------------------------------------- tiles
+// Tile t of a CTA: row chunk t / n_sub (chunks of kPfBN rows, expert after
+// expert), weight tile t % n_sub.  chunk_start[e] = first chunk of expert e.
+struct TileInfo {
+  int e, row0, nvalid, sub;
+};
+__device__ __forceinline__ TileInfo tile_info(int t, int n_sub, const int *chunk_start, int E,
+                                              const int32_t *offsets) {
+  const int chunk = t / n_sub;
+  int lo = 0, hi = E - 1;  // last expert with chunk_start[e] <= chunk
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (chunk_start[mid] <= chunk) lo = mid;
+    else hi = mid - 1;
+  }
+  TileInfo ti;
+  ti.e = lo;
+  ti.row0 = offsets[lo] + (chunk - chunk_start[lo]) * kPfBN;
+  ti.nvalid = min(kPfBN, offsets[lo + 1] - ti.row0);
+  ti.sub = t % n_sub;
+  return ti;
+}
+
+template <bool kGU>
+__global__ void __launch_bounds__(kPfThreads, 1)
+    prefill_kernel(PrefillArgs a, const __grid_constant__ CUtensorMap act_map) {
+  using C = PfCfg<kGU>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *tail = smem + C::kStages * C::kStageBytes;  // barriers, tables
+  uint64_t *full_raw = reinterpret_cast<uint64_t *>(tail);
+  uint64_t *full_b = full_raw + C::kStages;
+  uint64_t *full_a = full_b + C::kStages;
+  uint64_t *empty = full_a + C::kStages;
+  uint64_t *tmem_full = empty + C::kStages;
+  uint64_t *tmem_empty = tmem_full + 1;
+  uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(tmem_empty + 1);
+  volatile int *abort_s = reinterpret_cast<volatile int *>(tmem_base_s + 1);
+  int *ntiles_s = const_cast<int *>(abort_s) + 1;
+  int *chunk_start = ntiles_s + 1;  // [E + 1]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int KB = a.K / kPfBK;
+
+  if (tid == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full_raw[s], 1);
+      mbar_init(&full_b[s], 1);
+      mbar_init(&full_a[s], 128);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(tmem_full, 1);
+    mbar_init(tmem_empty, 128);
+    *abort_s = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_base_s, C::kTmemCols);
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // chunk table: chunk_start[e] = sum over e' < e of ceil(rows(e') / BN)
+  if (warp == 0) {
+    int carry = 0;
+    for (int e0 = 0; e0 < a.E; e0 += 32) {
+      const int e = e0 + lane;
+      const int n = e < a.E ? a.offsets[e + 1] - a.offsets[e] : 0;
+      const int c = (max(n, 0) + kPfBN - 1) / kPfBN;
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (e < a.E) chunk_start[e] = carry + incl - c;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      chunk_start[a.E] = carry;
+      *ntiles_s = carry * a.n_sub;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_base_s;
+  const int ntiles = *ntiles_s;
+  const int G = gridDim.x;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      for (int t = blockIdx.x; t < ntiles && !*abort_s; t += G) {
+        const TileInfo ti = tile_info(t, a.n_sub, chunk_start, a.E, a.offsets);
+        const uint8_t *wexp = a.w + (size_t)ti.e * a.w_stride;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % C::kStages;
+          const uint32_t ph = (it / C::kStages) & 1u;
+          if (!mbar_wait_bounded(&empty[s], ph ^ 1u, kPfWaitLimit)) {
+            atomicExch(a.err, DEVERR_PREFILL_WAIT);
+            *abort_s = 1;
+            break;
+          }
+          uint8_t *st = smem + s * C::kStageBytes;
+          uint8_t *raw = st + C::kABytes + C::kBBytes;
+          mbar_arrive_expect_tx(&full_raw[s], C::kRawBytes);
+          for (int m = 0; m < C::kMats; ++m)
+            for (int i = 0; i < 8; ++i) {
+              // strip of tile row block i: gate/up interleave strips (2j gate, 2j+1 up)
+              const int srow = ti.sub * 8 + i;  // 16-row strip index within one matrix
+              const int strip = kGU ? 2 * srow + m : srow;
+              bulk_g2s(raw + (m * 8 + i) * kBlkBytes,
+                       wexp + ((size_t)strip * KB + kb) * kBlkBytes, kBlkBytes, &full_raw[s]);
+            }
+          mbar_arrive_expect_tx(&full_b[s], C::kBBytes);
+          uint8_t *btile = st + C::kABytes;
+          for (int r = 0; r < kPfBN; r += 64)
+            tma_load_2d(btile + r * 128, &act_map, kb * kPfBK, ti.row0 + r, &full_b[s]);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t it = 0, tcount = 0;
+      constexpr uint32_t idesc = idesc_bf16_f32(kPfBN);
+      for (int t = blockIdx.x; t < ntiles && !*abort_s; t += G, ++tcount) {
+        if (!mbar_wait_bounded(tmem_empty, (tcount & 1u) ^ 1u, kPfWaitLimit)) {
+          atomicExch(a.err, DEVERR_PREFILL_WAIT);
+          *abort_s = 1;
+          break;
+        }
+        tc_fence_after();
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % C::kStages;
+          const uint32_t ph = (it / C::kStages) & 1u;
+          if (!mbar_wait_bounded(&full_b[s], ph, kPfWaitLimit) ||
+              !mbar_wait_bounded(&full_a[s], ph, kPfWaitLimit)) {
+            atomicExch(a.err, DEVERR_PREFILL_WAIT);
+            *abort_s = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = smem_u32(smem + s * C::kStageBytes);
+          const uint32_t bt = st + C::kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kPfBK / 16; ++kk) {
+            const uint64_t bdesc = smem_desc_sw128(bt + kk * 32);
+#pragma unroll
+            for (int m = 0; m < C::kMats; ++m) {
+              const uint64_t adesc = smem_desc_sw128(st + m * (kPfBM * 128) + kk * 32);
+              tc_mma_bf16(tmem_base + m * kPfBN, adesc, bdesc, idesc, (kb | kk) ? 1u : 0u);
+            }
+          }
+          tc_commit(&empty[s]);  // the stage is free once these MMAs have read it
+        }
+        if (!ok) break;
+        tc_commit(tmem_full);  // accumulators complete
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ dequant + epilogue
+    const int dw = warp - 2;            // 0..3
+    const int quarter = warp & 3;       // TMEM lanes this warp may read
+    const int gi = lane >> 2, t4 = lane & 3;
+    uint32_t it = 0, tcount = 0;
+    for (int t = blockIdx.x; t < ntiles; t += G, ++tcount) {
+      const TileInfo ti = tile_info(t, a.n_sub, chunk_start, a.E, a.offsets);
+      bool ok = true;
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        const int s = it % C::kStages;
+        const uint32_t ph = (it / C::kStages) & 1u;
+        const bool landed = mbar_wait_bounded(&full_raw[s], ph, kPfWaitLimit);
+        if (!landed || *abort_s) {
+          if (!landed) {
+            atomicExch(a.err, DEVERR_PREFILL_WAIT);
+            *abort_s = 1;
+          }
+          ok = false;
+          break;
+        }
+        uint8_t *st = smem + s * C::kStageBytes;
+        const uint8_t *raw = st + C::kABytes + C::kBBytes;
+        // blocks b = dw, dw + 4, ...: matrix b / 8, 16-row block b % 8
+        for (int b = dw; b < C::kMats * 8; b += 4) {
+          const uint8_t *blk = raw + b * kBlkBytes;
+          const int m = b >> 3, rb = (b & 7) * 16;
+          uint8_t *atile = st + m * (kPfBM * 128);
+          const uint4 cw = *reinterpret_cast<const uint4 *>(blk + 16 * lane);
+          const uint32_t sm0 = *reinterpret_cast<const uint32_t *>(blk + kBlkCodeBytes + 4 * gi);
+          const uint32_t sm1 = *reinterpret_cast<const uint32_t *>(blk + kBlkCodeBytes + 4 * (gi + 8));
+          const float s0 = f16_bits_to_f32((uint16_t)(sm0 & 0xFFFFu)), m0 = f16_bits_to_f32((uint16_t)(sm0 >> 16));
+          const float s1 = f16_bits_to_f32((uint16_t)(sm1 & 0xFFFFu)), m1 = f16_bits_to_f32((uint16_t)(sm1 >> 16));
+          const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t w = words[j];
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr)
+#pragma unroll
+              for (int hk = 0; hk < 2; ++hk) {
+                const int sh = 8 * hk + 4 * hr;
+                const float sc = hr ? s1 : s0, mn = hr ? m1 : m0;
+                const float lo = __fmaf_rn(code_to_f32(w, sh), sc, mn);
+                const float hi = __fmaf_rn(code_to_f32(w, sh + 16), sc, mn);
+                const int row = rb + gi + 8 * hr, k = 16 * j + 2 * t4 + 8 * hk;
+                *reinterpret_cast<uint32_t *>(atile + sw128_offset(row, k)) = pack_bf16x2(lo, hi);
+              }
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&full_a[s]);
+      }
+      if (!ok) break;
+      // ---- epilogue: accumulators of this tile
+      if (!mbar_wait_bounded(tmem_full, tcount & 1u, kPfWaitLimit)) {
+        atomicExch(a.err, DEVERR_PREFILL_WAIT);
+        *abort_s = 1;
+        break;
+      }
+      tc_fence_after();
+      const int feat = ti.sub * kPfBM + quarter * 32 + lane;  // this thread's weight row
+      const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16);
+      for (int c0 = 0; c0 < kPfBN; c0 += 16) {
+        if (c0 >= ti.nvalid) break;  // uniform across the warp
+        uint32_t v0[16], v1[16];
+        tmem_ld16(trow + c0, v0);
+        if (kGU) tmem_ld16(trow + kPfBN + c0, v1);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          if (c0 + c < ti.nvalid) {
+            float y;
+            if (kGU) {
+              const float g = __uint_as_float(v0[c]), u = __uint_as_float(v1[c]);
+              y = g / (1.0f + expf(-g)) * u;
+            } else {
+              y = __uint_as_float(v0[c]);
+            }
+            a.out[(size_t)(ti.row0 + c0 + c) * a.ld_out + feat] = f32_to_bf16_bits(y);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tmem_empty);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// bf16 [rows][cols] row-major, boxes of 64 columns x 64 rows, 128-byte swizzle.
+static bool make_act_map(CUtensorMap *map, const void *base, int rows, int cols) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool kGU>
+static moe_status prefill_launch(const PrefillArgs &a, const CUtensorMap &map, cudaStream_t stream) {
+  using C = PfCfg<kGU>;
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  static bool attr_done[64] = {false};
+  if (dev < 64 && !attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<kGU>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmemBytes);
+    if (e != cudaSuccess) {
+      set_cuda_error(e);
+      return MOE_ERR_CUDA;
+    }
+    attr_done[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(sms);
+  cfg.blockDim = dim3(kPfThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_kernel<kGU>, a, map);
+  if (e != cudaSuccess) {
+    set_cuda_error(e);
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+}  // namespace moe
 
 using namespace moe;
 
 extern "C" MOE_API size_t moe_prefill_workspace_bytes(int rows, int F) {
   if (rows <= 0 || F <= 0) return 0;
-  return (size_t)rows * F * 2 + 4096;
+  return (size_t)rows * F * 2;
 }
 
 extern "C" MOE_API moe_status moe_ffn_grouped_prefill(const moe_w4_layer *layer,
@@ -13,7 +469,46 @@ extern "C" MOE_API moe_status moe_ffn_grouped_prefill(const moe_w4_layer *layer,
                                                       const int32_t *offsets, int rows,
                                                       uint16_t *y_perm, void *ws, size_t ws_bytes,
                                                       moe_stream_t stream) {
-  (void)layer; (void)x_perm; (void)offsets; (void)rows; (void)y_perm; (void)ws; (void)ws_bytes;
-  (void)stream;
-  return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!layer || rows < 0) return MOE_ERR_INVALID_ARG;
+  const int E = layer->E, H = layer->H, F = layer->F;
+  if (E <= 0 || H <= 0 || F <= 0) return MOE_ERR_INVALID_ARG;
+  if (H % kPfBM || F % kPfBM || E > 960) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (rows == 0) return MOE_OK;
+  if (!layer->gate_up || !layer->down || !x_perm || !offsets || !y_perm) return MOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < moe_prefill_workspace_bytes(rows, F)) return MOE_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(x_perm) % 16 || reinterpret_cast<uintptr_t>(ws) % 16 ||
+      reinterpret_cast<uintptr_t>(y_perm) % 16 || reinterpret_cast<uintptr_t>(layer->gate_up) % 16 ||
+      reinterpret_cast<uintptr_t>(layer->down) % 16)
+    return MOE_ERR_INVALID_ARG;
+  int *err = device_error_word();
+  if (!err) return MOE_ERR_CUDA;
+  uint16_t *h = static_cast<uint16_t *>(ws);
+  CUtensorMap xmap, hmap;
+  if (!make_act_map(&xmap, x_perm, rows, H) || !make_act_map(&hmap, h, rows, F)) {
+    set_cuda_error(cudaErrorInvalidValue);
+    return MOE_ERR_CUDA;
+  }
+  cudaStream_t s = as_stream(stream);
+  PrefillArgs gu;
+  gu.w = static_cast<const uint8_t *>(layer->gate_up);
+  gu.w_stride = w4_packed_bytes(2 * F, H);
+  gu.offsets = offsets;
+  gu.out = h;
+  gu.err = err;
+  gu.E = E;
+  gu.K = H;
+  gu.rows = rows;
+  gu.n_sub = F / kPfBM;
+  gu.ld_out = F;
+  gu.F = F;
+  moe_status st = prefill_launch<true>(gu, xmap, s);
+  if (st != MOE_OK) return st;
+  PrefillArgs dn = gu;
+  dn.w = static_cast<const uint8_t *>(layer->down);
+  dn.w_stride = w4_packed_bytes(H, F);
+  dn.out = y_perm;
+  dn.K = F;
+  dn.n_sub = H / kPfBM;
+  dn.ld_out = H;
+  return prefill_launch<false>(dn, hmap, s);
 }
