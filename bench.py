@@ -340,6 +340,174 @@ def run_gpu(args, log):
     return out if rank == 0 else None
 
 
+PREFILL_WORKLOAD = ("grouped prefill: 2048 tokens x top-8 = 16,384 routed rows over 256 experts "
+                    "(router logits N(0,1) + Zipf(1.1) expert bias), hidden 2048, expert width 512; "
+                    "route, permute, tcgen05 grouped FFN, combine; 4 resident layers rotated")
+
+
+def run_gpu_prefill(args, log):
+    import torch
+    import synth
+    import quantized_moe_route_b200 as moe
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    T, k, nl = args.tokens, TOPK, args.layers
+    seed = 3000 + rank
+    layers = build_layers(nl, seed, log)
+    bias = synth.zipf_bias(seed, E)
+    xs, ls = [], []
+    for l in range(nl):
+        xs.append(torch.from_numpy(synth.activations_bf16(seed, l, T, H).view(np.int16)).to(dev))
+        ls.append(torch.from_numpy((synth.router_logits(seed, l, T, E) + bias[None, :]).astype(np.float32)).to(dev))
+    R = T * k
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    sorted_rows = torch.empty(R, dtype=torch.int32, device=dev)
+    inv = torch.empty(R, dtype=torch.int32, device=dev)
+    pws = torch.empty(moe.moe_permute_workspace_bytes(T, k, E), dtype=torch.uint8, device=dev)
+    x_perm = torch.empty((R, H), dtype=torch.int16, device=dev)
+    y_perm = torch.empty((R, H), dtype=torch.int16, device=dev)
+    fws = torch.empty(moe.moe_prefill_workspace_bytes(R, F), dtype=torch.uint8, device=dev)
+    y = torch.empty((T, H), dtype=torch.int16, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(l, ev=None, xin=None, lin=None):
+        moe.moe_route(ls[l] if lin is None else lin, k, idx, w, stream=stream)
+        moe.moe_permute(idx, E, counts, offsets, sorted_rows, inv, pws, x=xs[l] if xin is None else xin,
+                        x_perm=x_perm, stream=stream)
+        if ev is not None:
+            ev[0].record(stream)
+        moe.moe_ffn_grouped_prefill(layers[l][2], x_perm, offsets, y_perm, fws, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        moe.moe_unpermute_combine(y_perm, w, y, inv=inv, stream=stream)
+
+    K, W = args.steps, args.warmup
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            step(i % nl)
+    torch.cuda.synchronize()
+    dist_barrier()
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        dist_barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(K):
+                step((W + i) % nl)
+            e1.record(stream)
+        e1.synchronize()
+        torch.cuda.synchronize()
+        dist_barrier()
+    ms = dist_max(e0.elapsed_time(e1))
+    tokens = K * T * world
+    value = tokens / (ms / 1e3)
+
+    # kernel-duration pass: events around the two grouped-GEMM launches
+    P = min(K, 50)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(P)]
+    with torch.cuda.stream(stream):
+        for i in range(P):
+            step((W + i) % nl, evs[i])
+    torch.cuda.synchronize()
+    dur_ms = sum(a.elapsed_time(b) for a, b in evs) / P
+    flops = R * 6.0 * H * F
+    achieved = flops / (dur_ms / 1e3) / 1e12
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak, peak_kind = float(json.load(f)["bf16_tflops_sustained"]), "measured (sustained bf16)"
+    except Exception:
+        peak, peak_kind = 1400.0, "fallback (sustained bf16)"
+
+    # end to end: H2D of x and logits from pinned memory, D2H of y, every step
+    import synth as _s
+    hx = [torch.from_numpy(_s.activations_bf16(seed, l, T, H).view(np.int16)).pin_memory() for l in range(nl)]
+    hl = [torch.from_numpy((_s.router_logits(seed, l, T, E) + bias[None, :]).astype(np.float32)).pin_memory()
+          for l in range(nl)]
+    hy = torch.empty((T, H), dtype=torch.int16).pin_memory()
+    dx = torch.empty((T, H), dtype=torch.int16, device=dev)
+    dl = torch.empty((T, E), dtype=torch.float32, device=dev)
+    with torch.cuda.stream(stream):
+        for i in range(2):
+            dx.copy_(hx[i % nl], non_blocking=True)
+            dl.copy_(hl[i % nl], non_blocking=True)
+            step(i % nl, xin=dx, lin=dl)
+            hy.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a0.record(stream)
+        for i in range(K):
+            dx.copy_(hx[(W + i) % nl], non_blocking=True)
+            dl.copy_(hl[(W + i) % nl], non_blocking=True)
+            step((W + i) % nl, xin=dx, lin=dl)
+            hy.copy_(y, non_blocking=True)
+        a1.record(stream)
+    a1.synchronize()
+    e2e_ms = dist_max(a0.elapsed_time(a1))
+
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int4 weights (f16 scale/min), bf16 activations, fp32 accumulate", "data": "synthetic",
+        "config": {"workload": PREFILL_WORKLOAD, "experts": E, "top_k": k, "hidden": H, "expert_width": F,
+                   "tokens_per_step": T, "routed_rows": R, "resident_layers": nl,
+                   "l2": "inputs larger than L2 (453 MB of experts per layer, 67 MB permuted rows)",
+                   "parallelism": f"replicas x{world}", "launch": "stream-ordered, PDL into the FFN kernels"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "moe::prefill_kernel (gate/up + down launches)", "peak_kind": peak_kind,
+                     "alg_flop_per_launch_pair": flops, "avg_pair_us": dur_ms * 1e3},
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2 + T * E * 4,
+                "d2h_bytes_per_step": T * H * 2},
+        "gpu_launches": 7 * K,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline_prefill(seed, bias, budget_s=args.cpu_seconds, log=log)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return out if rank == 0 else None
+
+
+def cpu_baseline_prefill(seed, bias, budget_s, log):
+    """The oracle on sampled tokens of the prefill workload (rows per second
+    scaled to tokens/s); weights of the sampled tokens' experts only."""
+    import oracle
+    import synth
+    T = 2048
+    x = synth.activations_bf16(seed, 0, T, H)
+    lg = (synth.router_logits(seed, 0, T, E) + bias[None, :]).astype(np.float32)
+    idx, _ = oracle.route(lg, TOPK)
+    toks = list(range(0, T, 97))[:8]
+    need = sorted(set(idx[toks].ravel().tolist()))
+    import torch
+    experts = {}
+    for e in need:
+        wg = torch.empty((1, 2 * F, H), device="cuda")
+        wd = torch.empty((1, H, F), device="cuda")
+        synth.cuda_expert_weights(wg, seed, 0, e, synth.PROJ_GATE_UP)
+        synth.cuda_expert_weights(wd, seed, 0, e, synth.PROJ_DOWN)
+        experts[e] = (oracle.quantize_w4(wg[0].cpu().numpy()), oracle.quantize_w4(wd[0].cpu().numpy()))
+    t0 = time.time()
+    n = 0
+    while True:
+        t = toks[n % len(toks)]
+        oracle.moe_forward_w4(x[t:t + 1], lg[t:t + 1], TOPK, experts)
+        n += 1
+        if time.time() - t0 >= budget_s:
+            break
+    dt = time.time() - t0
+    return {"value": n / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} tokens of the 2048-token prefill batch (8 distinct, all 8 experts each), {dt:.1f}s"}
+
+
 # ---------------------------------------------------------------------------- CPU oracle
 def oracle_pool(seed, T, n, log, use_gpu_generator):
     """n sampled token-layers: canonical weights of their routed experts, built
@@ -421,7 +589,8 @@ def main():
     ap.add_argument("--steps", type=int, default=100000, help="timed steps")
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--tokens", type=int, default=1)
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill"])
+    ap.add_argument("--tokens", type=int, default=None, help="tokens per step (decode 1, prefill 2048)")
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="resident layers the steps rotate over (40 = 18.1 GB, larger than L2)")
     ap.add_argument("--graph-steps", type=int, default=400, help="steps captured per CUDA graph")
@@ -431,6 +600,10 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.tokens is None:
+        args.tokens = 2048 if args.workload == "prefill" else 1
+    if args.workload == "prefill" and args.layers == LAYERS:
+        args.layers = 4
 
     def log(msg):
         if not args.quiet:
@@ -438,6 +611,8 @@ def main():
 
     if args.impl == "reference":
         out = run_reference(args, log)
+    elif args.workload == "prefill":
+        out = run_gpu_prefill(args, log)
     else:
         out = run_gpu(args, log)
     if out is not None:

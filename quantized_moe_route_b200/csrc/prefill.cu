@@ -27,23 +27,34 @@
 
 namespace moe {
 
-constexpr int kPfThreads = 192;  // warp 0 producer, warp 1 MMA, warps 2..5 dequant + epilogue
+constexpr int kPfDqWarps = 16;   // warps 3..18: dequant, then epilogue
+constexpr int kPfDqThreads = kPfDqWarps * 32;
+constexpr int kPfThreads = (3 + kPfDqWarps) * 32;  // warp 0 int4 producer, 1 MMA, 2 activation producer
 constexpr int kPfBM = 128;       // weight rows per matrix per tile
-constexpr int kPfBN = 128;       // rows (tokens) per tile
+constexpr int kPfBN = 256;       // rows (tokens) per tile (the MMA's N is trimmed to the valid rows)
 constexpr int kPfBK = 64;        // k block = one quantisation group
 constexpr uint32_t kPfWaitLimit = 1u << 24;
 
+// Three rings: packed int4 blocks (deep: hides HBM latency, released by the
+// dequant warps), bf16 weight tiles (dequant -> MMA), activation tiles (TMA ->
+// MMA).
 template <bool kGU>
 struct PfCfg {
   static constexpr int kMats = kGU ? 2 : 1;
   static constexpr uint32_t kRawBytes = kMats * 8 * kBlkBytes;              // 8 strips per matrix
+  static constexpr uint32_t kRawStride = (kRawBytes + 127) / 128 * 128;
   static constexpr uint32_t kABytes = kMats * kPfBM * kPfBK * 2;            // bf16 tiles
   static constexpr uint32_t kBBytes = kPfBN * kPfBK * 2;                    // activation tile
-  static constexpr uint32_t kStageBytes = kABytes + kBBytes + ((kRawBytes + 1023) / 1024) * 1024;
-  static constexpr int kStages = kGU ? 3 : 5;
-  static constexpr uint32_t kTmemCols = kGU ? 2 * kPfBN : kPfBN;  // 256 or 128 (powers of two)
-  // stage layout: [A tiles][B tile][raw int4], all 1024-aligned
-  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 /*align slack*/ + 4096;
+  static constexpr int kRawStages = kGU ? 6 : 10;
+  static constexpr int kAStages = 2;
+  static constexpr int kBStages = 3;
+  static constexpr uint32_t kTmemCols = kGU ? 2 * kPfBN : kPfBN;  // 512 or 256 (powers of two)
+  // layout: [A ring][B ring][raw ring], 1024-aligned tiles
+  static constexpr uint32_t kAOff = 0;
+  static constexpr uint32_t kBOff = kAOff + kAStages * kABytes;
+  static constexpr uint32_t kRawOff = kBOff + kBStages * kBBytes;
+  static constexpr uint32_t kTailOff = kRawOff + kRawStages * kRawStride;
+  static constexpr uint32_t kSmemBytes = kTailOff + 1024 /*align slack*/ + 4096;
 };
 
 struct PrefillArgs {
@@ -125,16 +136,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int n) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kPfBM >> 4) << 24);
 }
 
-// Byte offset of element (row, k) (k even) of a 128-row x 64-k bf16 tile in
-// the 128-byte-swizzled K-major layout.
-__device__ __forceinline__ uint32_t sw128_offset(int row, int k) {
-  return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((((k >> 3) ^ (row & 7)) << 4) | ((k & 7) << 1)));
-}
-
-__device__ __forceinline__ float code_to_f32(uint32_t w, int shift) {
-  return __uint_as_float(((w >> shift) & 0xFu) | 0x4B000000u) - 8388608.0f;
-}
-
 // ---------------------------------------------------------------- tiles
 // Tile t of a CTA: row chunk t / n_sub (chunks of kPfBN rows, expert after
 // expert), weight tile t % n_sub.  chunk_start[e] = first chunk of expert e.
@@ -164,12 +165,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   using C = PfCfg<kGU>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *tail = smem + C::kStages * C::kStageBytes;  // barriers, tables
-  uint64_t *full_raw = reinterpret_cast<uint64_t *>(tail);
-  uint64_t *full_b = full_raw + C::kStages;
-  uint64_t *full_a = full_b + C::kStages;
-  uint64_t *empty = full_a + C::kStages;
-  uint64_t *tmem_full = empty + C::kStages;
+  uint8_t *tail = smem + C::kTailOff;  // barriers, tables
+  uint64_t *raw_full = reinterpret_cast<uint64_t *>(tail);
+  uint64_t *raw_empty = raw_full + C::kRawStages;
+  uint64_t *a_full = raw_empty + C::kRawStages;
+  uint64_t *a_empty = a_full + C::kAStages;
+  uint64_t *b_full = a_empty + C::kAStages;
+  uint64_t *b_empty = b_full + C::kBStages;
+  uint64_t *tmem_full = b_empty + C::kBStages;
   uint64_t *tmem_empty = tmem_full + 1;
   uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(tmem_empty + 1);
   volatile int *abort_s = reinterpret_cast<volatile int *>(tmem_base_s + 1);
@@ -180,14 +183,20 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const int KB = a.K / kPfBK;
 
   if (tid == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full_raw[s], 1);
-      mbar_init(&full_b[s], 1);
-      mbar_init(&full_a[s], 128);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < C::kRawStages; ++s) {
+      mbar_init(&raw_full[s], 1);
+      mbar_init(&raw_empty[s], kPfDqWarps);
+    }
+    for (int s = 0; s < C::kAStages; ++s) {
+      mbar_init(&a_full[s], kPfDqWarps);
+      mbar_init(&a_empty[s], 1);
+    }
+    for (int s = 0; s < C::kBStages; ++s) {
+      mbar_init(&b_full[s], 1);
+      mbar_init(&b_empty[s], 1);
     }
     mbar_init(tmem_full, 1);
-    mbar_init(tmem_empty, 128);
+    mbar_init(tmem_empty, kPfDqThreads);
     *abort_s = 0;
     fence_mbar_init();
   }
@@ -220,37 +229,56 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const uint32_t tmem_base = *tmem_base_s;
   const int ntiles = *ntiles_s;
   const int G = gridDim.x;
+  auto fail = [&]() {
+    atomicExch(a.err, DEVERR_PREFILL_WAIT);
+    *abort_s = 1;
+  };
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ int4 producer
     if (lane == 0) {
       uint32_t it = 0;
       for (int t = blockIdx.x; t < ntiles && !*abort_s; t += G) {
         const TileInfo ti = tile_info(t, a.n_sub, chunk_start, a.E, a.offsets);
         const uint8_t *wexp = a.w + (size_t)ti.e * a.w_stride;
         for (int kb = 0; kb < KB; ++kb, ++it) {
-          const int s = it % C::kStages;
-          const uint32_t ph = (it / C::kStages) & 1u;
-          if (!mbar_wait_bounded(&empty[s], ph ^ 1u, kPfWaitLimit)) {
-            atomicExch(a.err, DEVERR_PREFILL_WAIT);
-            *abort_s = 1;
+          const int s = it % C::kRawStages;
+          const uint32_t ph = (it / C::kRawStages) & 1u;
+          if (!mbar_wait_bounded(&raw_empty[s], ph ^ 1u, kPfWaitLimit)) {
+            fail();
             break;
           }
-          uint8_t *st = smem + s * C::kStageBytes;
-          uint8_t *raw = st + C::kABytes + C::kBBytes;
-          mbar_arrive_expect_tx(&full_raw[s], C::kRawBytes);
+          uint8_t *raw = smem + C::kRawOff + s * C::kRawStride;
+          mbar_arrive_expect_tx(&raw_full[s], C::kRawBytes);
           for (int m = 0; m < C::kMats; ++m)
             for (int i = 0; i < 8; ++i) {
-              // strip of tile row block i: gate/up interleave strips (2j gate, 2j+1 up)
-              const int srow = ti.sub * 8 + i;  // 16-row strip index within one matrix
+              // gate/up: strip 2 r is gate, 2 r + 1 up, of 16-feature block r
+              const int srow = ti.sub * 8 + i;
               const int strip = kGU ? 2 * srow + m : srow;
-              bulk_g2s(raw + (m * 8 + i) * kBlkBytes,
-                       wexp + ((size_t)strip * KB + kb) * kBlkBytes, kBlkBytes, &full_raw[s]);
+              bulk_g2s(raw + (m * 8 + i) * kBlkBytes, wexp + ((size_t)strip * KB + kb) * kBlkBytes,
+                       kBlkBytes, &raw_full[s]);
             }
-          mbar_arrive_expect_tx(&full_b[s], C::kBBytes);
-          uint8_t *btile = st + C::kABytes;
-          for (int r = 0; r < kPfBN; r += 64)
-            tma_load_2d(btile + r * 128, &act_map, kb * kPfBK, ti.row0 + r, &full_b[s]);
+        }
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ activation producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      for (int t = blockIdx.x; t < ntiles && !*abort_s; t += G) {
+        const TileInfo ti = tile_info(t, a.n_sub, chunk_start, a.E, a.offsets);
+        const int nbox = (ti.nvalid + 63) / 64;  // whole 64-row boxes covering the valid rows
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % C::kBStages;
+          const uint32_t ph = (it / C::kBStages) & 1u;
+          if (!mbar_wait_bounded(&b_empty[s], ph ^ 1u, kPfWaitLimit)) {
+            fail();
+            break;
+          }
+          uint8_t *btile = smem + C::kBOff + s * C::kBBytes;
+          mbar_arrive_expect_tx(&b_full[s], (uint32_t)nbox * 64u * 128u);
+          for (int r = 0; r < nbox * 64; r += 64)
+            tma_load_2d(btile + r * 128, &act_map, kb * kPfBK, ti.row0 + r, &b_full[s]);
         }
       }
     }
@@ -258,38 +286,38 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       uint32_t it = 0, tcount = 0;
-      constexpr uint32_t idesc = idesc_bf16_f32(kPfBN);
       for (int t = blockIdx.x; t < ntiles && !*abort_s; t += G, ++tcount) {
+        const TileInfo ti = tile_info(t, a.n_sub, chunk_start, a.E, a.offsets);
+        const uint32_t idesc = idesc_bf16_f32((ti.nvalid + 15) & ~15);  // N: valid rows, rounded to 16
         if (!mbar_wait_bounded(tmem_empty, (tcount & 1u) ^ 1u, kPfWaitLimit)) {
-          atomicExch(a.err, DEVERR_PREFILL_WAIT);
-          *abort_s = 1;
+          fail();
           break;
         }
         tc_fence_after();
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb, ++it) {
-          const int s = it % C::kStages;
-          const uint32_t ph = (it / C::kStages) & 1u;
-          if (!mbar_wait_bounded(&full_b[s], ph, kPfWaitLimit) ||
-              !mbar_wait_bounded(&full_a[s], ph, kPfWaitLimit)) {
-            atomicExch(a.err, DEVERR_PREFILL_WAIT);
-            *abort_s = 1;
+          const int sa = it % C::kAStages, sb = it % C::kBStages;
+          const uint32_t pa = (it / C::kAStages) & 1u, pb = (it / C::kBStages) & 1u;
+          if (!mbar_wait_bounded(&b_full[sb], pb, kPfWaitLimit) ||
+              !mbar_wait_bounded(&a_full[sa], pa, kPfWaitLimit)) {
+            fail();
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t st = smem_u32(smem + s * C::kStageBytes);
-          const uint32_t bt = st + C::kABytes;
+          const uint32_t at = smem_u32(smem + C::kAOff + sa * C::kABytes);
+          const uint32_t bt = smem_u32(smem + C::kBOff + sb * C::kBBytes);
 #pragma unroll
           for (int kk = 0; kk < kPfBK / 16; ++kk) {
             const uint64_t bdesc = smem_desc_sw128(bt + kk * 32);
 #pragma unroll
             for (int m = 0; m < C::kMats; ++m) {
-              const uint64_t adesc = smem_desc_sw128(st + m * (kPfBM * 128) + kk * 32);
+              const uint64_t adesc = smem_desc_sw128(at + m * (kPfBM * 128) + kk * 32);
               tc_mma_bf16(tmem_base + m * kPfBN, adesc, bdesc, idesc, (kb | kk) ? 1u : 0u);
             }
           }
-          tc_commit(&empty[s]);  // the stage is free once these MMAs have read it
+          tc_commit(&a_empty[sa]);  // both operand stages are free once these MMAs have read them
+          tc_commit(&b_empty[sb]);
         }
         if (!ok) break;
         tc_commit(tmem_full);  // accumulators complete
@@ -297,68 +325,87 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ dequant + epilogue
-    const int dw = warp - 2;            // 0..3
+    const int dw = warp - 3;            // 0..15
     const int quarter = warp & 3;       // TMEM lanes this warp may read
+    const int cgrp = dw >> 2;           // epilogue: column group of this warp
     const int gi = lane >> 2, t4 = lane & 3;
+    // Swizzled byte offsets inside a 128-byte row of the pair (16 j + 2 t4 + 8 hk,
+    // +1): 16-byte chunk (2 j + hk) xor gi, byte 4 t4.  Rows g and g + 8 of a
+    // block have the same swizzle phase gi.  (Words 2 and 3 differ from words 0
+    // and 1 only in chunk bit 2: xor 64.)
+    uint32_t koff[2][2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int hk = 0; hk < 2; ++hk) koff[j][hk] = (uint32_t)((((2 * j + hk) ^ gi) << 4) | (t4 << 2));
     uint32_t it = 0, tcount = 0;
     for (int t = blockIdx.x; t < ntiles; t += G, ++tcount) {
       const TileInfo ti = tile_info(t, a.n_sub, chunk_start, a.E, a.offsets);
       bool ok = true;
       for (int kb = 0; kb < KB; ++kb, ++it) {
-        const int s = it % C::kStages;
-        const uint32_t ph = (it / C::kStages) & 1u;
-        const bool landed = mbar_wait_bounded(&full_raw[s], ph, kPfWaitLimit);
+        const int sr = it % C::kRawStages, sa = it % C::kAStages;
+        const uint32_t pr = (it / C::kRawStages) & 1u, pa = (it / C::kAStages) & 1u;
+        const bool landed = mbar_wait_bounded(&raw_full[sr], pr, kPfWaitLimit) &&
+                            mbar_wait_bounded(&a_empty[sa], pa ^ 1u, kPfWaitLimit);
         if (!landed || *abort_s) {
-          if (!landed) {
-            atomicExch(a.err, DEVERR_PREFILL_WAIT);
-            *abort_s = 1;
-          }
+          if (!landed) fail();
           ok = false;
           break;
         }
-        uint8_t *st = smem + s * C::kStageBytes;
-        const uint8_t *raw = st + C::kABytes + C::kBBytes;
-        // blocks b = dw, dw + 4, ...: matrix b / 8, 16-row block b % 8
-        for (int b = dw; b < C::kMats * 8; b += 4) {
+        const uint8_t *raw = smem + C::kRawOff + sr * C::kRawStride;
+        uint8_t *atiles = smem + C::kAOff + sa * C::kABytes;
+        // units (block b, word half wh): matrix b / 8, 16-row block b % 8,
+        // words 2 wh and 2 wh + 1 of every lane
+        for (int u = dw; u < C::kMats * 16; u += kPfDqWarps) {
+          const int b = u >> 1, wh = u & 1;
           const uint8_t *blk = raw + b * kBlkBytes;
           const int m = b >> 3, rb = (b & 7) * 16;
-          uint8_t *atile = st + m * (kPfBM * 128);
-          const uint4 cw = *reinterpret_cast<const uint4 *>(blk + 16 * lane);
+          uint8_t *atile = atiles + m * (kPfBM * 128);
+          const uint2 cw = *reinterpret_cast<const uint2 *>(blk + 16 * lane + 8 * wh);
           const uint32_t sm0 = *reinterpret_cast<const uint32_t *>(blk + kBlkCodeBytes + 4 * gi);
           const uint32_t sm1 = *reinterpret_cast<const uint32_t *>(blk + kBlkCodeBytes + 4 * (gi + 8));
-          const float s0 = f16_bits_to_f32((uint16_t)(sm0 & 0xFFFFu)), m0 = f16_bits_to_f32((uint16_t)(sm0 >> 16));
-          const float s1 = f16_bits_to_f32((uint16_t)(sm1 & 0xFFFFu)), m1 = f16_bits_to_f32((uint16_t)(sm1 >> 16));
-          const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+          // fp32 q * s + m computed as (128 + q) * s + (m - 128 s): the code
+          // becomes the bf16 value 128 + q by OR-ing 0x4300, and a bf16 is the
+          // top half of an fp32; m - 128 s is formed once per row and group
+          float sc[2], of[2];
+          sc[0] = f16_bits_to_f32((uint16_t)(sm0 & 0xFFFFu));
+          sc[1] = f16_bits_to_f32((uint16_t)(sm1 & 0xFFFFu));
+          of[0] = __fmaf_rn(-128.f, sc[0], f16_bits_to_f32((uint16_t)(sm0 >> 16)));
+          of[1] = __fmaf_rn(-128.f, sc[1], f16_bits_to_f32((uint16_t)(sm1 >> 16)));
+          uint8_t *rowp[2] = {atile + ((rb + gi) >> 3) * 1024 + gi * 128,
+                              atile + ((rb + gi + 8) >> 3) * 1024 + gi * 128};
+          const uint32_t wx = (uint32_t)wh << 6;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t w = words[j];
+          for (int jj = 0; jj < 2; ++jj) {
+            const uint32_t w = jj ? cw.y : cw.x;
 #pragma unroll
-            for (int hr = 0; hr < 2; ++hr)
-#pragma unroll
-              for (int hk = 0; hk < 2; ++hk) {
-                const int sh = 8 * hk + 4 * hr;
-                const float sc = hr ? s1 : s0, mn = hr ? m1 : m0;
-                const float lo = __fmaf_rn(code_to_f32(w, sh), sc, mn);
-                const float hi = __fmaf_rn(code_to_f32(w, sh + 16), sc, mn);
-                const int row = rb + gi + 8 * hr, k = 16 * j + 2 * t4 + 8 * hk;
-                *reinterpret_cast<uint32_t *>(atile + sw128_offset(row, k)) = pack_bf16x2(lo, hi);
-              }
+            for (int i = 0; i < 4; ++i) {  // shift 4 i: hr = i & 1, hk = i >> 1
+              const int hr = i & 1, hk = i >> 1;
+              const uint32_t v = ((w >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
+              const float lo = __fmaf_rn(__uint_as_float(v << 16), sc[hr], of[hr]);
+              const float hi = __fmaf_rn(__uint_as_float(v & 0xFFFF0000u), sc[hr], of[hr]);
+              *reinterpret_cast<__nv_bfloat162 *>(rowp[hr] + (koff[jj][hk] ^ wx)) = __floats2bfloat162_rn(lo, hi);
+            }
           }
         }
         fence_proxy_async_smem();
-        mbar_arrive(&full_a[s]);
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&a_full[sa]);
+          mbar_arrive(&raw_empty[sr]);
+        }
       }
       if (!ok) break;
-      // ---- epilogue: accumulators of this tile
+      // ---- epilogue: accumulators of this tile; the four warps of a lane
+      // quarter split the columns
       if (!mbar_wait_bounded(tmem_full, tcount & 1u, kPfWaitLimit)) {
-        atomicExch(a.err, DEVERR_PREFILL_WAIT);
-        *abort_s = 1;
+        fail();
         break;
       }
       tc_fence_after();
       const int feat = ti.sub * kPfBM + quarter * 32 + lane;  // this thread's weight row
       const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16);
-      for (int c0 = 0; c0 < kPfBN; c0 += 16) {
+      for (int c0 = cgrp * 16; c0 < kPfBN; c0 += 64) {
         if (c0 >= ti.nvalid) break;  // uniform across the warp
         uint32_t v0[16], v1[16];
         tmem_ld16(trow + c0, v0);
@@ -369,7 +416,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             float y;
             if (kGU) {
               const float g = __uint_as_float(v0[c]), u = __uint_as_float(v1[c]);
-              y = g / (1.0f + expf(-g)) * u;
+              y = g / (1.0f + __expf(-g)) * u;
             } else {
               y = __uint_as_float(v0[c]);
             }
