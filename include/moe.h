@@ -192,6 +192,29 @@ MOE_API moe_status moe_ffn_w4a16_decode(const moe_w4_layer *layer, const uint16_
                                         void *ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * One whole MoE layer for a small batch in a single launch: routing (as
+ * moe_route, bit-identical), the weight-streaming expert FFN (as
+ * moe_ffn_w4a16_decode) and the router-weighted combine (as
+ * moe_unpermute_combine: j ascending, fp32, nearest-even bf16).
+ *   x bf16 [T][H], logits fp32 [T][E] -> y bf16 [T][H];
+ *   idx [T][k] / w [T][k]: optional outputs of the routing (both or neither).
+ * Workspace: moe_decode_layer_workspace_bytes(T, k, H, F) bytes, 16-byte
+ * aligned, zero-filled before first use, reusable by stream-ordered calls
+ * (as for moe_ffn_w4a16_decode).  Limits: 1 <= T <= 16, T*k <= 256,
+ * k <= 32, E <= 1024, H % 64 == 0, F % 64 == 0.  Each 64-output chunk of a
+ * token is summed by the last of its k down-projection work items, in j
+ * order, so the result does not depend on scheduling.
+ * Source: the same passages as moe_route, moe_ffn_w4a16_decode and
+ * moe_unpermute_combine ("Footprint and speed": a decode step is streamed
+ * weight GEMVs, here one launch per layer).
+ */
+MOE_API size_t moe_decode_layer_workspace_bytes(int T, int k, int H, int F);
+MOE_API moe_status moe_decode_layer_w4a16(const moe_w4_layer *layer, const uint16_t *x,
+                                          const float *logits, int T, int k, uint16_t *y,
+                                          int32_t *idx, float *w, void *ws, size_t ws_bytes,
+                                          moe_stream_t stream);
+
+/*
  * Allocation-free form of moe_ffn_w4a16_decode (the pages have no counterpart;
  * this is a library convenience).  Same inputs, outputs and results, but no
  * workspace argument: the scratch lives in one fixed array of 516 KiB

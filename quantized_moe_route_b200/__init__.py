@@ -55,6 +55,9 @@ SIGNATURES = {
     "moe_decode_workspace_bytes": (_sz, [_i, _i, _i]),
     "moe_ffn_w4a16_decode": (_i, [ctypes.POINTER(moe_w4_layer), _vp, _vp, _i, _i, _vp, _vp, _sz, _vp]),
     "moe_ffn_w4a16_decode_static": (_i, [ctypes.POINTER(moe_w4_layer), _vp, _vp, _i, _i, _vp, _vp]),
+    "moe_decode_layer_workspace_bytes": (_sz, [_i, _i, _i, _i]),
+    "moe_decode_layer_w4a16": (_i, [ctypes.POINTER(moe_w4_layer), _vp, _vp, _i, _i, _vp, _vp, _vp, _vp, _sz,
+                                    _vp]),
     "moe_prefill_workspace_bytes": (_sz, [_i, _i]),
     "moe_ffn_grouped_prefill": (_i, [ctypes.POINTER(moe_w4_layer), _vp, _vp, _i, _vp, _vp, _sz, _vp]),
     "moe_unpermute_combine": (_i, [_vp, _i, _vp, _vp, _i, _i, _i, _vp, _vp]),
@@ -160,6 +163,18 @@ def moe_ffn_w4a16_decode_static(layer: moe_w4_layer, x, idx, y_rows, stream=None
     T, k = idx.shape
     _check(lib().moe_ffn_w4a16_decode_static(ctypes.byref(layer), _p(x), _p(idx), T, k, _p(y_rows),
                                              _stream(stream)), "moe_ffn_w4a16_decode_static")
+
+
+def moe_decode_layer_workspace_bytes(T, k, H, F) -> int:
+    return lib().moe_decode_layer_workspace_bytes(T, k, H, F)
+
+
+def moe_decode_layer_w4a16(layer: moe_w4_layer, x, logits, k, y, ws, idx=None, w=None, stream=None):
+    """Route + expert FFN + combine of one layer in one launch."""
+    T = x.shape[0]
+    _check(lib().moe_decode_layer_w4a16(ctypes.byref(layer), _p(x), _p(logits), T, k, _p(y), _p(idx), _p(w),
+                                        _p(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "moe_decode_layer_w4a16")
 
 
 def moe_prefill_workspace_bytes(rows, F) -> int:

@@ -28,6 +28,7 @@
 // Activations enter as bf16 (exact), h is rounded to bf16 for the down
 // projection; all sums are fp32.
 #include "common.cuh"
+#include "route.cuh"
 
 namespace moe {
 
@@ -42,6 +43,11 @@ constexpr int kDecOutRows = 64;  // outputs per B item (4 strips)
 constexpr size_t kDecCtrlBytes = 4096;  // workspace head: epoch, done counter
 
 struct DecodeArgs {
+  const float *logits;       // fused form: router logits [T][E]
+  uint16_t *y;               // fused form: combined bf16 output [T][H]
+  int32_t *idx_out;          // fused form, optional: routing of every token
+  float *w_out;
+  unsigned long long *ybuf;  // fused form: [T*k][H] words {fp32 row output, epoch}
   const uint8_t *gu;
   const uint8_t *dn;
   size_t gu_stride, dn_stride;  // bytes per expert
@@ -91,7 +97,7 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int T, int H, int F, in
   L.xsum = take((uint32_t)T * (H / 64) * 4, 16);
   L.hsum = take(2u * T * (F / 64) * 4, 16);
   L.bars = take((uint32_t)nstages * 8, 8);
-  L.meta = take(3200 * 4, 16);  // routing tables + 256 x 8 row-set words
+  L.meta = take(3600 * 4, 16);  // routing tables + 256 x 8 row-set words
   L.total = o;
   return L;
 }
@@ -280,6 +286,12 @@ __device__ __forceinline__ void group_sums(const uint16_t *rows, int nrows, int 
   }
 }
 
+// kFused = false: routing comes in (idx), the k rows of every token go out as
+// fp32 y_rows.  kFused = true: the kernel routes the tokens itself from their
+// logits (PER logits per lane) and writes the router-weighted combine y; each
+// 64-output chunk of a token is combined by the down item of that token's
+// highest expert slot, which waits only on lower-numbered items.
+template <bool kFused, int PER>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const DecodeSmem L = decode_smem_layout(a.T, a.H, a.F, a.nstages, a.stage_bytes);
@@ -295,6 +307,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
   int *ridx = slot_rows + kDecMaxRows;                    // [256] expert of row
   int *misc = ridx + kDecMaxRows;                         // [0] U, [1] abort, [2] epoch
   uint32_t *rmask = reinterpret_cast<uint32_t *>(misc + 8);  // [256 slots][8 words] rows of a slot
+  float *rw = reinterpret_cast<float *>(rmask + kDecMaxRows * 8);  // [256] routing weights (fused)
+  int *maxslot = reinterpret_cast<int *>(rw + kDecMaxRows);        // [16] highest slot of a token
   __shared__ int tok_lists[2][kDecMaxTok];
   __shared__ int ident[kDecMaxTok];
 
@@ -346,7 +360,22 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
 
   // ---- routing table.  Unique experts in increasing id ("slots"); the
   // first weight copies go out as soon as the slots are known.
-  if (tid < R) {
+  if (kFused) {  // warp t routes token t
+    if (warp < T) {
+      int j_idx;
+      float j_w;
+      route_token_warp<PER>(a.logits + (size_t)warp * E, E, k, &j_idx, &j_w);
+      if (lane < k) {
+        ridx[warp * k + lane] = j_idx;
+        rw[warp * k + lane] = j_w;
+        atomicOr(&emask[j_idx >> 5], 1u << (j_idx & 31));
+        if (blockIdx.x == 0 && a.idx_out) {
+          a.idx_out[warp * k + lane] = j_idx;
+          a.w_out[warp * k + lane] = j_w;
+        }
+      }
+    }
+  } else if (tid < R) {
     int e = a.idx[tid];
     e = (e < 0 || e >= E) ? 0 : e;  // out-of-range ids are outside the contract; stay memory safe
     ridx[tid] = e;
@@ -417,6 +446,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
     int rank = __popc(rmask[my_slot * 8 + (tid >> 5)] & ((1u << (tid & 31)) - 1u));
     for (int w = 0; w < (tid >> 5); ++w) rank += __popc(rmask[my_slot * 8 + w]);
     slot_rows[slot_off[my_slot] + rank] = tid;
+  }
+  if (kFused && tid < T) {  // the slot whose down items combine token tid
+    int mx = 0;
+    for (int j = 0; j < k; ++j) {
+      const int e = ridx[tid * k + j];
+      mx = max(mx, wbase[e >> 5] + __popc(emask[e >> 5] & ((1u << (e & 31)) - 1u)));
+    }
+    maxslot[tid] = mx;
   }
   __syncthreads();
 
@@ -517,14 +554,53 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
         const int row = rem / nt, n = rem % nt;
         if (n < ntok) {
           const float y = red[(size_t)strip * 16 * nt + rem] + red[(size_t)(strip + 4) * 16 * nt + rem];
-          a.y_rows[(size_t)slot_rows[r0 + n] * H + kDecOutRows * sub + 16 * strip + row] = y;
+          const size_t o = (size_t)slot_rows[r0 + n] * H + kDecOutRows * sub + 16 * strip + row;
+          if (kFused)
+            a.ybuf[o] = ((unsigned long long)__float_as_uint(y) << 32) | (unsigned long long)epoch;
+          else
+            a.y_rows[o] = y;
+        }
+      }
+      if (kFused) {
+        // combine the tokens of this slot whose highest slot is this one:
+        // y[t][c] = sum over j (in order) of w[t][j] * row (t, j), polling the
+        // rows of lower slots until they carry this call's epoch
+        team_sync(bar_id);  // this item's own words are written
+        bool ok = true;
+        for (int v = ttid; v < ntok * kDecOutRows; v += kTeamThreads) {
+          const int n = v / kDecOutRows, c = v % kDecOutRows;
+          const int t = slot_rows[r0 + n] / k;
+          if (maxslot[t] != slot) continue;
+          float acc = 0.f;
+          for (int j = 0; j < k && ok; ++j) {
+            const unsigned long long *wp = a.ybuf + (size_t)(t * k + j) * H + kDecOutRows * sub + c;
+            unsigned long long wv = ld_relaxed_u64(wp);
+            uint32_t spins = 0;
+            while ((unsigned int)(wv & 0xFFFFFFFFull) != epoch) {
+              if (++spins > (1u << 22)) {
+                ok = false;
+                break;
+              }
+              __nanosleep(64);
+              wv = ld_relaxed_u64(wp);
+            }
+            acc = __fadd_rn(acc, __fmul_rn(rw[t * k + j], __uint_as_float((uint32_t)(wv >> 32))));
+          }
+          a.y[(size_t)t * H + kDecOutRows * sub + c] = f32_to_bf16_bits(acc);
+        }
+        if (!ok) {
+          atomicExch(a.err, DEVERR_DECODE_H_WAIT);
+          aborted = true;
         }
       }
     }
     // generic-proxy writes to this stage are done; the next copy into it is
     // an async-proxy write
     fence_proxy_async_smem();
-    team_sync(bar_id);
+    if (team_or(bar_id, aborted)) {
+      aborted = true;
+      break;
+    }
     if (ttid == 0 && q + a.nstages < myCount) issue(blockIdx.x + (q + a.nstages) * G, nA, stage, pol);
   }
 
@@ -546,6 +622,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
 
 // One or two CTAs per SM (all resident: B items wait on A items of other
 // CTAs); as many weight stages as fit.
+template <bool kFused, int PER>
 static moe_status decode_launch(DecodeArgs &a, bool pdl, cudaStream_t stream) {
   const int H = a.H, F = a.F, T = a.T, k = a.k;
   a.stage_bytes = dec_stage_bytes(T, H, F, &a.h_off);
@@ -561,7 +638,7 @@ static moe_status decode_launch(DecodeArgs &a, bool pdl, cudaStream_t stream) {
   a.nstages = nst;
   static bool attr_done[64] = {false};
   if (dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<kFused, PER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)cap);
     if (e != cudaSuccess) {
       set_cuda_error(e);
@@ -583,7 +660,7 @@ static moe_status decode_launch(DecodeArgs &a, bool pdl, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel, a);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<kFused, PER>, a);
   if (e != cudaSuccess) {
     set_cuda_error(e);
     return MOE_ERR_CUDA;
@@ -608,6 +685,11 @@ static moe_status decode_check(const moe_w4_layer *layer, const uint16_t *x, con
 
 static void decode_fill(DecodeArgs &a, const moe_w4_layer *layer, const uint16_t *x,
                         const int32_t *idx, int T, int k, float *y_rows, uint8_t *scratch) {
+  a.logits = nullptr;
+  a.y = nullptr;
+  a.idx_out = nullptr;
+  a.w_out = nullptr;
+  a.ybuf = nullptr;
   a.gu = static_cast<const uint8_t *>(layer->gate_up);
   a.dn = static_cast<const uint8_t *>(layer->down);
   a.gu_stride = w4_packed_bytes(2 * layer->F, layer->H);
@@ -645,7 +727,44 @@ extern "C" MOE_API moe_status moe_ffn_w4a16_decode(const moe_w4_layer *layer, co
   decode_fill(a, layer, x, idx, T, k, y_rows, static_cast<uint8_t *>(ws));
   a.err = device_error_word();
   if (!a.err) return MOE_ERR_CUDA;
-  return decode_launch(a, true, as_stream(stream));
+  return decode_launch<false, 8>(a, true, as_stream(stream));
+}
+
+extern "C" MOE_API size_t moe_decode_layer_workspace_bytes(int T, int k, int H, int F) {
+  if (T <= 0 || k <= 0 || H <= 0 || F <= 0) return 0;
+  return kDecCtrlBytes + sizeof(unsigned long long) * (size_t)T * k * ((size_t)F + (size_t)H);
+}
+
+extern "C" MOE_API moe_status moe_decode_layer_w4a16(const moe_w4_layer *layer, const uint16_t *x,
+                                                     const float *logits, int T, int k,
+                                                     uint16_t *y, int32_t *idx, float *w,
+                                                     void *ws, size_t ws_bytes,
+                                                     moe_stream_t stream) {
+  if (!layer || T < 0 || k <= 0) return MOE_ERR_INVALID_ARG;
+  const int E = layer->E, H = layer->H, F = layer->F;
+  if (E <= 0 || H <= 0 || F <= 0 || k > E) return MOE_ERR_INVALID_ARG;
+  if (H % 64 || F % 64 || E > kDecMaxE || T > kDecMaxTok || T * k > kDecMaxRows || k > 32)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return MOE_OK;
+  if (!layer->gate_up || !layer->down || !x || !logits || !y) return MOE_ERR_INVALID_ARG;
+  if ((idx == nullptr) != (w == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(layer->gate_up) % 16 ||
+      reinterpret_cast<uintptr_t>(layer->down) % 16 || reinterpret_cast<uintptr_t>(x) % 16 ||
+      reinterpret_cast<uintptr_t>(ws) % 16)
+    return MOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < moe_decode_layer_workspace_bytes(T, k, H, F)) return MOE_ERR_WORKSPACE;
+  DecodeArgs a;
+  decode_fill(a, layer, x, nullptr, T, k, nullptr, static_cast<uint8_t *>(ws));
+  a.logits = logits;
+  a.y = y;
+  a.idx_out = idx;
+  a.w_out = w;
+  a.ybuf = reinterpret_cast<unsigned long long *>(static_cast<uint8_t *>(ws) + kDecCtrlBytes +
+                                                  sizeof(unsigned long long) * (size_t)T * k * F);
+  a.err = device_error_word();
+  if (!a.err) return MOE_ERR_CUDA;
+  if (E <= 256) return decode_launch<true, 8>(a, true, as_stream(stream));
+  return decode_launch<true, 32>(a, true, as_stream(stream));
 }
 
 // ---------------------------------------------------------------------------
@@ -719,5 +838,5 @@ extern "C" MOE_API moe_status moe_ffn_w4a16_decode_static(const moe_w4_layer *la
     set_cuda_error(e);
     return MOE_ERR_CUDA;
   }
-  return decode_launch(a, false, as_stream(stream));
+  return decode_launch<false, 8>(a, false, as_stream(stream));
 }

@@ -37,3 +37,5 @@ def test_host_only_queries():
     assert L.moe_status_string(2) == b"MOE_ERR_UNSUPPORTED_SHAPE"
     assert L.moe_version().startswith(b"moe-w4-b200")
     assert L.moe_decode_workspace_bytes(1, 8, 512) >= 8 * 512 * 8  # one 8-byte h word per value
+    # fused layer: h words and one 8-byte output word per (row, channel)
+    assert L.moe_decode_layer_workspace_bytes(1, 8, 2048, 512) >= 8 * 8 * (512 + 2048)

@@ -98,3 +98,50 @@ def test_decode_workspace_reuse_across_batch_sizes():
         idx, y_rows, y, ws = _run_decode(layer, x, logits, k, ws)
         _, _, oy_rows, oy = oracle.moe_forward_w4(x, logits, k, layer.canon)
         ffn_close(y_rows, oy_rows, f"y_rows T={T}")
+
+
+def _fused(layer, x, logits, k, ws=None):
+    T = x.shape[0]
+    ws = torch.zeros(moe.moe_decode_layer_workspace_bytes(T, k, layer.H, layer.F), dtype=torch.uint8,
+                     device="cuda") if ws is None else ws
+    y = torch.empty((T, layer.H), dtype=torch.int16, device="cuda")
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    moe.moe_decode_layer_w4a16(layer.desc, u16(x), torch.from_numpy(np.ascontiguousarray(logits)).cuda(), k, y, ws,
+                               idx=idx, w=w)
+    torch.cuda.synchronize()
+    assert moe.moe_device_error() == 0
+    return to_u16(y), idx.cpu().numpy(), w.cpu().numpy(), ws
+
+
+@pytest.mark.parametrize("seed,E,H,F,T,k", [(50, 8, 128, 64, 4, 2), (51, 256, 2048, 512, 1, 8),
+                                            (52, 64, 1024, 256, 16, 8), (53, 300, 512, 128, 5, 3)])
+def test_fused_layer_matches_oracle_and_unfused_path(seed, E, H, F, T, k):
+    """One launch (route + FFN + combine) equals route -> decode -> combine
+    bit for bit, and the oracle within the FFN tolerance."""
+    x = synth.activations_bf16(seed, 0, T, H)
+    logits = synth.router_logits(seed, 0, T, E)
+    oidx, ow = oracle.route(logits, k)
+    layer = Layer(seed, 0, E, H, F, oidx.ravel())
+    y, idx, w, _ = _fused(layer, x, logits, k)
+    assert np.array_equal(idx, oidx)
+    np.testing.assert_allclose(w, ow, rtol=1e-6, atol=1e-7)
+    y_unfused = _run_decode(layer, x, logits, k)[2]
+    assert np.array_equal(y, y_unfused)
+    _, _, _, oy = oracle.moe_forward_w4(x, logits, k, layer.canon)
+    ffn_close(synth.bf16_bits_to_f32(y), synth.bf16_bits_to_f32(oy), "fused y")
+
+
+def test_fused_layer_one_expert_for_all_tokens_and_reuse():
+    T, E, k = 16, 32, 4
+    logits = synth.router_logits(54, 0, T, E)
+    logits[:, 7] += 50.0
+    logits = logits.astype(np.float32)
+    x = synth.activations_bf16(54, 0, T, 512)
+    oidx, _ = oracle.route(logits, k)
+    layer = Layer(54, 0, E, 512, 128, oidx.ravel())
+    y1, _, _, ws = _fused(layer, x, logits, k)
+    y2, _, _, ws = _fused(layer, x, logits, k, ws)  # the workspace carries over
+    assert np.array_equal(y1, y2)
+    _, _, _, oy = oracle.moe_forward_w4(x, logits, k, layer.canon)
+    ffn_close(synth.bf16_bits_to_f32(y1), synth.bf16_bits_to_f32(oy), "fused y")
