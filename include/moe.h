@@ -128,6 +128,81 @@ typedef struct {
 } moe_w4_layer;
 
 /* ======================================================================== */
+/* NVFP4 expert weights and activations (the variant)                        */
+/* ======================================================================== */
+/*
+ * Source: "Drama 3 - NVFP4 routed experts", section "Quantization": E2M1
+ * codes, one E4M3 scale per 16 input channels, one FP32 global scale per
+ * matrix with gate and up sharing theirs, round to nearest; activations are
+ * quantised dynamically per token (FP32 global, E4M3 block scales).  The
+ * formulas are this library's reading:
+ *   G   = amax / 2688 (= 448 * 6), or 1 when amax == 0
+ *   S_b = E4M3(amax_b / (6 G)), nearest-even, saturating at 448
+ *   q_i = E2M1(v_i / (S_b G)), nearest-even, saturating at +-6; 0 if S_b == 0
+ * each division and product one correctly rounded fp32 operation; the value
+ * of q_i is E2M1(q_i) * S_b * G.
+ * Canonical form of one [N][K] matrix: codes u8 [N][K] (E2M1 bit patterns
+ * 0..15, bit 3 the sign), sf u8 [N][K/16] (E4M3 bit patterns), and G.
+ * Device ("packed") form, moe_nvfp4_packed_bytes(N, K) = N * K * 9 / 16
+ * bytes: 16-row strips (gate/up: gate strip i next to up strip i, as for
+ * int4), each strip 16 rows of K/2 code bytes (logical byte b holds channel
+ * 2b in its low nibble; inside each 128-byte run of row r the 16-byte pieces
+ * are XOR-permuted by r & 7, the tensor cores' 128-byte shared-memory
+ * swizzle) followed by the scales as [K/64][16 rows][4] bytes.
+ * Requirements: N % 16 == 0 (gate/up: N % 32 == 0), K % 256 == 0.
+ */
+MOE_API size_t moe_nvfp4_packed_bytes(int N, int K);
+
+/* Device scalar *G = the global scale of n fp32 values v (formula above).
+ * G is also the scratch of the reduction; n == 0 gives 1.  Errors:
+ * INVALID_ARG. */
+MOE_API moe_status moe_nvfp4_global(const float *v, size_t n, float *G, moe_stream_t stream);
+
+/* Quantise fp32 v [N][K] with the device global *G to the canonical form:
+ * codes u8 [N][K], sf u8 [N][K/16].  v and codes 16-byte aligned.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE (K % 16). */
+MOE_API moe_status moe_quantize_nvfp4(const float *v, int N, int K, const float *G,
+                                      uint8_t *codes, uint8_t *sf, moe_stream_t stream);
+
+/* Canonical -> packed, and its exact inverse.  Errors as for moe_pack_w4
+ * (UNSUPPORTED_SHAPE for K % 256). */
+MOE_API moe_status moe_pack_nvfp4(const uint8_t *codes, const uint8_t *sf, int N, int K,
+                                  int kind, void *packed, size_t packed_bytes,
+                                  moe_stream_t stream);
+MOE_API moe_status moe_unpack_nvfp4(const void *packed, int N, int K, int kind,
+                                    uint8_t *codes, uint8_t *sf, moe_stream_t stream);
+
+/*
+ * Per-row (per-token) activation quantisation, one global per row:
+ * output row p quantises input row src = src_rows ? src_rows[p] / src_div : p
+ * of x ([*][K], bf16 when x_dtype == 0, fp32 when x_dtype == 1).  Outputs:
+ * codes u8 [rows][K/2] (two per byte, channel 2b in the low nibble of byte b),
+ * sf u8 [rows][K/16], G fp32 [rows].  With src_rows = sorted_rows and
+ * src_div = k (from moe_permute) this quantises and groups the rows by
+ * expert in one pass.  x 16-byte aligned, codes 8-byte aligned.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE (K % 16).
+ */
+MOE_API moe_status moe_quantize_nvfp4_rows(const void *x, int x_dtype, int rows, int K,
+                                           const int32_t *src_rows, int src_div,
+                                           uint8_t *codes, uint8_t *sf, float *G,
+                                           moe_stream_t stream);
+
+/*
+ * One MoE layer's NVFP4 experts, experts back to back as for moe_w4_layer
+ * (gate_up: E * moe_nvfp4_packed_bytes(2F, H), kind MOE_W4_GATE_UP; down:
+ * E * moe_nvfp4_packed_bytes(H, F), kind MOE_W4_PLAIN), with device arrays of
+ * the experts' globals g_gu [E] (shared by gate and up) and g_d [E].  A HOST
+ * struct read during the call only.
+ */
+typedef struct {
+  int E, H, F;
+  const void *gate_up;
+  const void *down;
+  const float *g_gu;
+  const float *g_d;
+} moe_nvfp4_layer;
+
+/* ======================================================================== */
 /* Routing and permutation                                                   */
 /* ======================================================================== */
 
@@ -210,6 +285,26 @@ MOE_API moe_status moe_ffn_w4a16_decode(const moe_w4_layer *layer, const uint16_
  */
 MOE_API size_t moe_decode_layer_workspace_bytes(int T, int k, int H, int F);
 MOE_API moe_status moe_decode_layer_w4a16(const moe_w4_layer *layer, const uint16_t *x,
+                                          const float *logits, int T, int k, uint16_t *y,
+                                          int32_t *idx, float *w, void *ws, size_t ws_bytes,
+                                          moe_stream_t stream);
+
+/*
+ * The NVFP4 form of moe_decode_layer_w4a16: one launch routes the T tokens,
+ * quantises each token's x to NVFP4 (per-token global, as
+ * moe_quantize_nvfp4_rows), runs every selected expert's FFN on the NVFP4
+ * weights of `layer` (fp32 sums of E2M1 * E4M3 products per 16-channel block,
+ * times the two globals; gate and up outputs scaled before SwiGLU), quantises
+ * each row's fp32 h to NVFP4 (per-row global) before the down projection, and
+ * writes the router-weighted combine y bf16 [T][H].
+ * Source: "Drama 3 - NVFP4 routed experts", section "Quantization" (NVFP4
+ * weights, dynamic per-token activation scales), and the passages of
+ * moe_decode_layer_w4a16.
+ * Workspace: moe_decode_layer_workspace_bytes(T, k, H, F), as for the int4
+ * form.  Limits as for moe_decode_layer_w4a16, with H % 256 == 0 and
+ * F % 256 == 0.
+ */
+MOE_API moe_status moe_decode_layer_nvfp4(const moe_nvfp4_layer *layer, const uint16_t *x,
                                           const float *logits, int T, int k, uint16_t *y,
                                           int32_t *idx, float *w, void *ws, size_t ws_bytes,
                                           moe_stream_t stream);

@@ -39,6 +39,12 @@ class moe_w4_layer(ctypes.Structure):
                 ("gate_up", ctypes.c_void_p), ("down", ctypes.c_void_p)]
 
 
+class moe_nvfp4_layer(ctypes.Structure):
+    _fields_ = [("E", ctypes.c_int), ("H", ctypes.c_int), ("F", ctypes.c_int),
+                ("gate_up", ctypes.c_void_p), ("down", ctypes.c_void_p),
+                ("g_gu", ctypes.c_void_p), ("g_d", ctypes.c_void_p)]
+
+
 _vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 SIGNATURES = {
     "moe_status_string": (ctypes.c_char_p, [_i]),
@@ -49,6 +55,12 @@ SIGNATURES = {
     "moe_pack_w4": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
     "moe_unpack_w4": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp]),
     "moe_dequant_w4": (_i, [_vp, _i, _i, _i, _vp, _vp]),
+    "moe_nvfp4_packed_bytes": (_sz, [_i, _i]),
+    "moe_nvfp4_global": (_i, [_vp, _sz, _vp, _vp]),
+    "moe_quantize_nvfp4": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp]),
+    "moe_pack_nvfp4": (_i, [_vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
+    "moe_unpack_nvfp4": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
+    "moe_quantize_nvfp4_rows": (_i, [_vp, _i, _i, _i, _vp, _i, _vp, _vp, _vp, _vp]),
     "moe_route": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
     "moe_permute_workspace_bytes": (_sz, [_i, _i, _i]),
     "moe_permute": (_i, [_vp, _i, _i, _i, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -58,6 +70,8 @@ SIGNATURES = {
     "moe_decode_layer_workspace_bytes": (_sz, [_i, _i, _i, _i]),
     "moe_decode_layer_w4a16": (_i, [ctypes.POINTER(moe_w4_layer), _vp, _vp, _i, _i, _vp, _vp, _vp, _vp, _sz,
                                     _vp]),
+    "moe_decode_layer_nvfp4": (_i, [ctypes.POINTER(moe_nvfp4_layer), _vp, _vp, _i, _i, _vp, _vp, _vp, _vp,
+                                    _sz, _vp]),
     "moe_prefill_workspace_bytes": (_sz, [_i, _i]),
     "moe_ffn_grouped_prefill": (_i, [ctypes.POINTER(moe_w4_layer), _vp, _vp, _i, _vp, _vp, _sz, _vp]),
     "moe_unpermute_combine": (_i, [_vp, _i, _vp, _vp, _i, _i, _i, _vp, _vp]),
@@ -114,6 +128,42 @@ def moe_pack_w4(codes, scale, minv, kind, packed, stream=None):
                              _stream(stream)), "moe_pack_w4")
 
 
+def moe_nvfp4_packed_bytes(N: int, K: int) -> int:
+    return lib().moe_nvfp4_packed_bytes(N, K)
+
+
+def moe_nvfp4_global(v, G, stream=None):
+    _check(lib().moe_nvfp4_global(_p(v), v.numel(), _p(G), _stream(stream)), "moe_nvfp4_global")
+
+
+def moe_quantize_nvfp4(v, G, codes, sf, stream=None):
+    N, K = v.shape
+    _check(lib().moe_quantize_nvfp4(_p(v), N, K, _p(G), _p(codes), _p(sf), _stream(stream)),
+           "moe_quantize_nvfp4")
+
+
+def moe_pack_nvfp4(codes, sf, kind, packed, stream=None):
+    N, K = codes.shape
+    nbytes = packed.numel() * packed.element_size()
+    _check(lib().moe_pack_nvfp4(_p(codes), _p(sf), N, K, kind, _p(packed), nbytes, _stream(stream)),
+           "moe_pack_nvfp4")
+
+
+def moe_unpack_nvfp4(packed, N, K, kind, codes, sf, stream=None):
+    _check(lib().moe_unpack_nvfp4(_p(packed), N, K, kind, _p(codes), _p(sf), _stream(stream)),
+           "moe_unpack_nvfp4")
+
+
+def moe_quantize_nvfp4_rows(x, codes, sf, G, src_rows=None, src_div=1, rows=None, stream=None):
+    """x: bf16 (or int16 bits) or fp32 [*][K]; rows defaults to x.shape[0]."""
+    import torch
+    K = x.shape[1]
+    rows = x.shape[0] if rows is None else rows
+    dt = 1 if x.dtype == torch.float32 else 0
+    _check(lib().moe_quantize_nvfp4_rows(_p(x), dt, rows, K, _p(src_rows), src_div, _p(codes), _p(sf),
+                                         _p(G), _stream(stream)), "moe_quantize_nvfp4_rows")
+
+
 def moe_unpack_w4(packed, N, K, kind, codes, scale, minv, stream=None):
     _check(lib().moe_unpack_w4(_p(packed), N, K, kind, _p(codes), _p(scale), _p(minv),
                                _stream(stream)), "moe_unpack_w4")
@@ -126,6 +176,11 @@ def moe_dequant_w4(packed, N, K, kind, out, stream=None):
 def make_layer(E, H, F, gate_up, down) -> moe_w4_layer:
     """Host descriptor of one layer's packed experts (device buffers)."""
     return moe_w4_layer(E, H, F, gate_up.data_ptr(), down.data_ptr())
+
+
+def make_nvfp4_layer(E, H, F, gate_up, down, g_gu, g_d) -> moe_nvfp4_layer:
+    """Host descriptor of one layer's packed NVFP4 experts and their globals (device buffers)."""
+    return moe_nvfp4_layer(E, H, F, gate_up.data_ptr(), down.data_ptr(), g_gu.data_ptr(), g_d.data_ptr())
 
 
 # ---------------------------------------------------------------- routing / permutation
@@ -175,6 +230,14 @@ def moe_decode_layer_w4a16(layer: moe_w4_layer, x, logits, k, y, ws, idx=None, w
     _check(lib().moe_decode_layer_w4a16(ctypes.byref(layer), _p(x), _p(logits), T, k, _p(y), _p(idx), _p(w),
                                         _p(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "moe_decode_layer_w4a16")
+
+
+def moe_decode_layer_nvfp4(layer: moe_nvfp4_layer, x, logits, k, y, ws, idx=None, w=None, stream=None):
+    """NVFP4 experts: route + in-kernel activation quantisation + FFN + combine, one launch."""
+    T = x.shape[0]
+    _check(lib().moe_decode_layer_nvfp4(ctypes.byref(layer), _p(x), _p(logits), T, k, _p(y), _p(idx), _p(w),
+                                        _p(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "moe_decode_layer_nvfp4")
 
 
 def moe_prefill_workspace_bytes(rows, F) -> int:

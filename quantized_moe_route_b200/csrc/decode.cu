@@ -27,7 +27,19 @@
 //   sum_k (q s + m) x_k = s D + (m - 128 s) X,   X = sum_k x_k.
 // Activations enter as bf16 (exact), h is rounded to bf16 for the down
 // projection; all sums are fp32.
+//
+// NVFP4 weights ("Drama 3 - NVFP4 routed experts", section "Quantization")
+// use the same items and strip sizes (4.5 bits per weight).  Each token's x
+// and each row's h are quantised to NVFP4 inside the kernel (per-row global,
+// E4M3 scale per 16 channels, E2M1 codes) and held in shared memory as the
+// exact f16 values E2M1 * S_b.  A code word gives two f16 fragment halves by
+// moving the 3 magnitude bits to bits 9..11 and the sign to bit 15, which is
+// the E2M1 value times 2^-14 for every code (0.5 lands on the f16 subnormal
+// 2^-15); the tensor core sums one 16-channel block per m16n8k16 step, the
+// weight block scale is applied to that step's result in fp32, and 2^14 and
+// the two globals are applied once per output.
 #include "common.cuh"
+#include "nvfp4.cuh"
 #include "route.cuh"
 
 namespace moe {
@@ -41,6 +53,7 @@ constexpr int kDecMaxRows = 256; // T * k
 constexpr int kDecMaxE = 1024;
 constexpr int kDecOutRows = 64;  // outputs per B item (4 strips)
 constexpr size_t kDecCtrlBytes = 4096;  // workspace head: epoch, done counter
+constexpr int kFmtW4 = 0, kFmtNvfp4 = 1;
 
 struct DecodeArgs {
   const float *logits;       // fused form: router logits [T][E]
@@ -51,10 +64,11 @@ struct DecodeArgs {
   const uint8_t *gu;
   const uint8_t *dn;
   size_t gu_stride, dn_stride;  // bytes per expert
+  const float *g_gu, *g_d;      // NVFP4: per-expert global scales
   const uint16_t *x;
   const int32_t *idx;
   float *y_rows;
-  unsigned long long *hbuf;  // [T*k][F] words {bf16 h << 32 | epoch}
+  unsigned long long *hbuf;  // [T*k][F] words {h << 32 | epoch}: bf16 h (int4), fp32 h (NVFP4)
   unsigned int *ctrl;        // [0] last epoch, [1] CTAs done
   int *err;
   int T, k, E, H, F;
@@ -82,7 +96,7 @@ __host__ __device__ inline uint32_t dec_stage_bytes(int T, int H, int F, uint32_
   return (b + 127u) / 128u * 128u;
 }
 
-__host__ __device__ inline DecodeSmem decode_smem_layout(int T, int H, int F, int nstages,
+__host__ __device__ inline DecodeSmem decode_smem_layout(int fmt, int T, int H, int F, int nstages,
                                                          uint32_t stage_bytes) {
   DecodeSmem L;
   uint32_t o = 0;
@@ -94,8 +108,10 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int T, int H, int F, in
   };
   L.stages = take((uint32_t)nstages * stage_bytes, 128);
   L.x = take((uint32_t)T * H * 2, 16);
-  L.xsum = take((uint32_t)T * (H / 64) * 4, 16);
-  L.hsum = take(2u * T * (F / 64) * 4, 16);
+  // int4: 64-channel group sums of x and of each team's h;
+  // NVFP4: the row globals of x and of each team's h
+  L.xsum = take(fmt == kFmtW4 ? (uint32_t)T * (H / 64) * 4 : (uint32_t)T * 4, 16);
+  L.hsum = take(fmt == kFmtW4 ? 2u * T * (F / 64) * 4 : 2u * T * 4, 16);
   L.bars = take((uint32_t)nstages * 8, 8);
   L.meta = take(3600 * 4, 16);  // routing tables + 256 x 8 row-set words
   L.total = o;
@@ -286,15 +302,158 @@ __device__ __forceinline__ void group_sums(const uint16_t *rows, int nrows, int 
   }
 }
 
+// ---------------------------------------------------------------- NVFP4
+__device__ __forceinline__ void mma_f16_16816(float d[4], const uint32_t a[4], uint32_t b0,
+                                              uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Two f16 fragment halves from the E2M1 codes at bits [sh, sh+4) and
+// [sh+16, sh+20) of w: magnitude bits to 9..11, sign to 15, i.e. the code's
+// value times 2^-14 (sh <= 12).
+__device__ __forceinline__ uint32_t e2m1x2_f16(uint32_t w, int sh) {
+  return ((w << (9 - sh)) & 0x0E000E00u) | ((w << (12 - sh)) & 0x80008000u);
+}
+
+__device__ __forceinline__ void e4m3x4_to_f32(uint32_t w, float f[4]) {
+  const __half2 lo(__nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xFFFFu), __NV_E4M3));
+  const __half2 hi(__nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w >> 16), __NV_E4M3));
+  const float2 a = __half22float2(lo), b = __half22float2(hi);
+  f[0] = a.x, f[1] = a.y, f[2] = b.x, f[3] = b.y;
+}
+
+// Shared-memory order of the 16 channels of a block: position p of the
+// tensor-core k index holds channel kNvPerm[p], matching the nibbles a lane
+// takes from its code word (lane t, word (t >> 1) of the block, byte t & 1
+// and byte (t & 1) + 2, low nibbles for k 2t, 2t+1, high nibbles for 2t+8,
+// 2t+9).
+// (p = k3 k2 k1 k0 in bits -> channel k2 k0 k1 k3: 0 4 2 6 8 12 10 14 1 5 3 7 9 13 11 15)
+__host__ __device__ constexpr int nv_perm(int p) {
+  return (((p >> 2) & 1) << 3) | ((p & 1) << 2) | (((p >> 1) & 1) << 1) | ((p >> 3) & 1);
+}
+
+// One warp quantises one row of nb 16-value blocks to NVFP4 and stores the
+// values E2M1(q) * S_b (exact in f16) in tensor-core k order at out[16 nb];
+// returns the row's global.  load(b, v) fills v with block b of the row.
+// The same fp32 operations as the format's quantiser decide every code.
+template <class Load>
+__device__ __forceinline__ float nvfp4_row_f16(Load load, int nb, uint16_t *out) {
+  const int lane = threadIdx.x & 31;
+  float amax = 0.f;
+  for (int b = lane; b < nb; b += 32) {
+    float v[16];
+    load(b, v);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float G = amax == 0.f ? 1.0f : __fdiv_rn(amax, 2688.0f);
+  for (int b = lane; b < nb; b += 32) {
+    float v[16];
+    load(b, v);
+    float bmax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
+    const __nv_fp8_storage_t s8 = __nv_cvt_float_to_fp8(__fdiv_rn(bmax, __fmul_rn(6.0f, G)),
+                                                        __NV_SATFINITE, __NV_E4M3);
+    const float sb = __half2float(__half(__nv_cvt_fp8_to_halfraw(s8, __NV_E4M3)));
+    const float scale = __fmul_rn(sb, G);
+    float q[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const __nv_fp4_storage_t c = __nv_cvt_float_to_fp4(__fdiv_rn(v[i], scale), __NV_E2M1,
+                                                         cudaRoundNearest);
+      const float e = __half2float(__half(__nv_cvt_fp4_to_halfraw(c, __NV_E2M1)));
+      q[i] = sb == 0.f ? 0.f : __fmul_rn(e, sb);
+    }
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      w[i] = (uint32_t)__half_as_ushort(__float2half_rn(q[nv_perm(2 * i)])) |
+             ((uint32_t)__half_as_ushort(__float2half_rn(q[nv_perm(2 * i + 1)])) << 16);
+    uint4 *dst = reinterpret_cast<uint4 *>(out + 16 * b);
+    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  }
+  return G;
+}
+
+// One warp, one 64-channel chunk g of NMAT NVFP4 strips (K channels each)
+// against up to 16 activation rows act[n][ld] (f16 in tensor-core k order):
+// acc += S_b * (sum over the block of code * 2^-14 * activation), block by
+// block.  The A fragments are built once for both token blocks.
+template <int NB, int NMAT>
+__device__ __forceinline__ void fp4_chunk_mma(const uint8_t *const (&strip)[NMAT], int K, int g,
+                                              const uint16_t *act, int ld, const int *tok_of,
+                                              int ntok, float acc[NMAT][2][4]) {
+  const int lane = threadIdx.x & 31, gi = lane >> 2, t4 = lane & 3;
+  const int sh = 8 * (t4 & 1);
+  const int rowoff = gi * (K / 2) + 128 * (g >> 2) + 4 * (t4 >> 1);
+  uint32_t af[NMAT][4][4];
+  float slo[NMAT][4], shi[NMAT][4];
+#pragma unroll
+  for (int m = 0; m < NMAT; ++m) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int off = rowoff + ((((2 * g + (j >> 1)) & 7) ^ (gi & 7)) << 4) + 8 * (j & 1);
+      const uint32_t wlo = *reinterpret_cast<const uint32_t *>(strip[m] + off);
+      const uint32_t whi = *reinterpret_cast<const uint32_t *>(strip[m] + off + 8 * (K / 2));
+      af[m][j][0] = e2m1x2_f16(wlo, sh);
+      af[m][j][1] = e2m1x2_f16(whi, sh);
+      af[m][j][2] = e2m1x2_f16(wlo, sh + 4);
+      af[m][j][3] = e2m1x2_f16(whi, sh + 4);
+    }
+    const uint8_t *sc = strip[m] + 8 * K + 64 * g;
+    e4m3x4_to_f32(*reinterpret_cast<const uint32_t *>(sc + 4 * gi), slo[m]);
+    e4m3x4_to_f32(*reinterpret_cast<const uint32_t *>(sc + 4 * (gi + 8)), shi[m]);
+  }
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb) {
+    const int n = nb * 8 + gi;
+    const bool live = n < ntok;
+    const uint16_t *arow = act + (size_t)(live ? tok_of[n] : 0) * ld + 64 * g + 2 * t4;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t b0 = live ? *reinterpret_cast<const uint32_t *>(arow + 16 * j) : 0u;
+      const uint32_t b1 = live ? *reinterpret_cast<const uint32_t *>(arow + 16 * j + 8) : 0u;
+#pragma unroll
+      for (int m = 0; m < NMAT; ++m) {
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_f16_16816(d, af[m][j], b0, b1);
+        acc[m][nb][0] = __fmaf_rn(slo[m][j], d[0], acc[m][nb][0]);
+        acc[m][nb][1] = __fmaf_rn(slo[m][j], d[1], acc[m][nb][1]);
+        acc[m][nb][2] = __fmaf_rn(shi[m][j], d[2], acc[m][nb][2]);
+        acc[m][nb][3] = __fmaf_rn(shi[m][j], d[3], acc[m][nb][3]);
+      }
+    }
+  }
+}
+
+template <int NB, int NMAT>
+__device__ __forceinline__ void fp4_warp_chunks(const uint8_t *const (&strip)[NMAT], int K,
+                                                int first, int step, const uint16_t *act, int ld,
+                                                const int *tok_of, int ntok,
+                                                float acc[NMAT][2][4]) {
+  for (int g = first; g < K / 64; g += step)
+    fp4_chunk_mma<NB, NMAT>(strip, K, g, act, ld, tok_of, ntok, acc);
+}
+
 // kFused = false: routing comes in (idx), the k rows of every token go out as
 // fp32 y_rows.  kFused = true: the kernel routes the tokens itself from their
 // logits (PER logits per lane) and writes the router-weighted combine y; each
 // 64-output chunk of a token is combined by the down item of that token's
 // highest expert slot, which waits only on lower-numbered items.
-template <bool kFused, int PER>
+template <int kFmt, bool kFused, int PER>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
+  static_assert(kFmt == kFmtW4 || kFused, "the NVFP4 decode exists in the fused form only");
+  constexpr bool kFp4 = kFmt == kFmtNvfp4;
   extern __shared__ __align__(128) uint8_t smem[];
-  const DecodeSmem L = decode_smem_layout(a.T, a.H, a.F, a.nstages, a.stage_bytes);
+  const DecodeSmem L = decode_smem_layout(kFmt, a.T, a.H, a.F, a.nstages, a.stage_bytes);
   uint16_t *x_s = reinterpret_cast<uint16_t *>(smem + L.x);
   float *xsum_s = reinterpret_cast<float *>(smem + L.xsum);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
@@ -402,7 +561,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
       const uint64_t pol = policy_evict_first();
       for (int q = 0; q < min(myCount, a.nstages); ++q) issue(blockIdx.x + q * G, nA, q, pol);
     }
-  } else {
+  } else if (!kFp4) {
     const int vec = T * H / 8;  // activations into shared memory
     for (int v = tid - 32; v < vec; v += kDecThreads - 32)
       reinterpret_cast<uint4 *>(x_s)[v] = reinterpret_cast<const uint4 *>(a.x)[v];
@@ -416,7 +575,27 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
     my_slot = wbase[e >> 5] + __popc(emask[e >> 5] & ((1u << (e & 31)) - 1u));
     atomicOr(&rmask[my_slot * 8 + (tid >> 5)], 1u << (tid & 31));
   }
-  group_sums(x_s, T, H, Gh, xsum_s, tid, kDecThreads);
+  if (!kFp4) {
+    group_sums(x_s, T, H, Gh, xsum_s, tid, kDecThreads);
+  } else if (warp < T) {  // warp t quantises token t: x_s = E2M1 * S_b (f16), xsum_s[t] = G
+    const uint16_t *xr = a.x + (size_t)warp * H;
+    const float G = nvfp4_row_f16(
+        [&](int b, float (&v)[16]) {
+          const uint4 *q = reinterpret_cast<const uint4 *>(xr + 16 * b);
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const uint4 u4 = q[i];
+            const uint32_t u[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              v[8 * i + 2 * jj] = __uint_as_float(u[jj] << 16);
+              v[8 * i + 2 * jj + 1] = __uint_as_float(u[jj] & 0xFFFF0000u);
+            }
+          }
+        },
+        H / 16, x_s + (size_t)warp * H);
+    if (lane == 0) xsum_s[warp] = G;
+  }
   __syncthreads();
   const int U = misc[0];
   const unsigned int epoch = (unsigned int)misc[2];
@@ -461,7 +640,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
   const int myCount = (int)blockIdx.x < nItems ? (nItems - 1 - (int)blockIdx.x) / G + 1 : 0;
   const uint64_t pol = policy_evict_first();
   int *tok_list = tok_lists[team];
-  float *hsum_s = reinterpret_cast<float *>(smem + L.hsum) + (size_t)team * T * Gf;
+  float *hsum_s = reinterpret_cast<float *>(smem + L.hsum) + (size_t)team * T * (kFp4 ? 1 : Gf);
 
   // ---- team `team` runs the CTA's items q = team, team + 2, ...
   bool aborted = false;
@@ -491,7 +670,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
           const unsigned long long w =
               ld_relaxed_u64(a.hbuf + (size_t)slot_rows[r0 + n] * F + f);
           if ((unsigned int)(w & 0xFFFFFFFFull) != epoch) mine = false;
-          else h_s[(size_t)n * F + f] = (uint16_t)(w >> 32);
+          else if (!kFp4) h_s[(size_t)n * F + f] = (uint16_t)(w >> 32);
         }
         ready = !team_or(bar_id, !mine);
         if (ready || ++spins > (1u << 20)) break;
@@ -502,7 +681,22 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
         aborted = true;
         break;
       }
-      group_sums(h_s, ntok, F, Gf, hsum_s, ttid, kTeamThreads);
+      if (!kFp4) {
+        group_sums(h_s, ntok, F, Gf, hsum_s, ttid, kTeamThreads);
+      } else {  // warp per row: h (fp32) -> NVFP4 -> E2M1 * S_b in h_s, G in hsum_s
+        for (int n = tw; n < ntok; n += kTeamWarps) {
+          const unsigned long long *hr = a.hbuf + (size_t)slot_rows[r0 + n] * F;
+          const float G = nvfp4_row_f16(
+              [&](int b, float (&v)[16]) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                  v[i] = __uint_as_float((uint32_t)(ld_relaxed_u64(hr + 16 * b + i) >> 32));
+              },
+              F / 16, h_s + (size_t)n * F);
+          if (lane == 0) hsum_s[n] = G;
+        }
+        team_sync(bar_id);
+      }
     }
     // wait for this item's weights (every thread observes the barrier)
     const bool landed = mbar_wait_bounded(&bars[stage], parity, 1u << 26);
@@ -516,10 +710,16 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
     if (isA) {
       float acc[2][2][4] = {};
       const uint8_t *base[2] = {st, st + stripA};
-      if (nbmax == 2)
+      if (kFp4) {
+        if (nbmax == 2)
+          fp4_warp_chunks<2, 2>(base, H, tw, kTeamWarps, x_s, H, tok_list, ntok, acc);
+        else
+          fp4_warp_chunks<1, 2>(base, H, tw, kTeamWarps, x_s, H, tok_list, ntok, acc);
+      } else if (nbmax == 2) {
         warp_groups<2, 2>(base, tw, kTeamWarps, Gh, x_s, H, tok_list, ntok, xsum_s, Gh, acc);
-      else
+      } else {
         warp_groups<1, 2>(base, tw, kTeamWarps, Gh, x_s, H, tok_list, ntok, xsum_s, Gh, acc);
+      }
       team_sync(bar_id);  // all weights read
       frag_to_red(red + (size_t)(tw * 2 + 0) * 16 * nt, acc[0], nbmax, nt);
       frag_to_red(red + (size_t)(tw * 2 + 1) * 16 * nt, acc[1], nbmax, nt);
@@ -533,19 +733,32 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
           g += red[(size_t)(w * 2 + 0) * 16 * nt + row * nt + n];
           u += red[(size_t)(w * 2 + 1) * 16 * nt + row * nt + n];
         }
-        const float h = g / (1.0f + expf(-g)) * u;
-        const unsigned long long wv =
-            ((unsigned long long)f32_to_bf16_bits(h) << 32) | (unsigned long long)epoch;
+        uint32_t hbits;
+        if (kFp4) {  // the sums carry 2^-14; then the x and weight globals
+          const float gs = __fmul_rn(xsum_s[tok_list[n]], a.g_gu[slot_expert[slot]]);
+          g = __fmul_rn(__fmul_rn(g, 16384.0f), gs);
+          u = __fmul_rn(__fmul_rn(u, 16384.0f), gs);
+          hbits = __float_as_uint(g / (1.0f + expf(-g)) * u);
+        } else {
+          hbits = f32_to_bf16_bits(g / (1.0f + expf(-g)) * u);
+        }
+        const unsigned long long wv = ((unsigned long long)hbits << 32) | (unsigned long long)epoch;
         a.hbuf[(size_t)slot_rows[r0 + n] * F + 16 * sub + row] = wv;
       }
     } else {
       // warp -> strip (tw & 3), groups of parity (tw >> 2)
       float acc[1][2][4] = {};
       const uint8_t *base[1] = {st + (size_t)(tw & 3) * stripB};
-      if (nbmax == 2)
+      if (kFp4) {
+        if (nbmax == 2)
+          fp4_warp_chunks<2, 1>(base, F, tw >> 2, 2, h_s, F, ident, ntok, acc);
+        else
+          fp4_warp_chunks<1, 1>(base, F, tw >> 2, 2, h_s, F, ident, ntok, acc);
+      } else if (nbmax == 2) {
         warp_groups<2, 1>(base, tw >> 2, 2, Gf, h_s, F, ident, ntok, hsum_s, Gf, acc);
-      else
+      } else {
         warp_groups<1, 1>(base, tw >> 2, 2, Gf, h_s, F, ident, ntok, hsum_s, Gf, acc);
+      }
       team_sync(bar_id);  // all weights read
       frag_to_red(red + (size_t)tw * 16 * nt, acc[0], nbmax, nt);
       team_sync(bar_id);
@@ -553,7 +766,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
         const int strip = v / (16 * nt), rem = v % (16 * nt);
         const int row = rem / nt, n = rem % nt;
         if (n < ntok) {
-          const float y = red[(size_t)strip * 16 * nt + rem] + red[(size_t)(strip + 4) * 16 * nt + rem];
+          float y = red[(size_t)strip * 16 * nt + rem] + red[(size_t)(strip + 4) * 16 * nt + rem];
+          if (kFp4)
+            y = __fmul_rn(__fmul_rn(y, 16384.0f), __fmul_rn(hsum_s[n], a.g_d[slot_expert[slot]]));
           const size_t o = (size_t)slot_rows[r0 + n] * H + kDecOutRows * sub + 16 * strip + row;
           if (kFused)
             a.ybuf[o] = ((unsigned long long)__float_as_uint(y) << 32) | (unsigned long long)epoch;
@@ -622,7 +837,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
 
 // One or two CTAs per SM (all resident: B items wait on A items of other
 // CTAs); as many weight stages as fit.
-template <bool kFused, int PER>
+template <int kFmt, bool kFused, int PER>
 static moe_status decode_launch(DecodeArgs &a, bool pdl, cudaStream_t stream) {
   const int H = a.H, F = a.F, T = a.T, k = a.k;
   a.stage_bytes = dec_stage_bytes(T, H, F, &a.h_off);
@@ -632,13 +847,13 @@ static moe_status decode_launch(DecodeArgs &a, bool pdl, cudaStream_t stream) {
   cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   const uint32_t cap = (uint32_t)smem_max - 1024;
   int nst = 8;  // even: the two teams own alternate stages
-  while (nst > 2 && decode_smem_layout(T, H, F, nst, a.stage_bytes).total > cap) nst -= 2;
-  const DecodeSmem L = decode_smem_layout(T, H, F, nst, a.stage_bytes);
+  while (nst > 2 && decode_smem_layout(kFmt, T, H, F, nst, a.stage_bytes).total > cap) nst -= 2;
+  const DecodeSmem L = decode_smem_layout(kFmt, T, H, F, nst, a.stage_bytes);
   if (L.total > cap) return MOE_ERR_UNSUPPORTED_SHAPE;
   a.nstages = nst;
   static bool attr_done[64] = {false};
   if (dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<kFused, PER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<kFmt, kFused, PER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)cap);
     if (e != cudaSuccess) {
       set_cuda_error(e);
@@ -660,7 +875,7 @@ static moe_status decode_launch(DecodeArgs &a, bool pdl, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<kFused, PER>, a);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<kFmt, kFused, PER>, a);
   if (e != cudaSuccess) {
     set_cuda_error(e);
     return MOE_ERR_CUDA;
@@ -697,6 +912,8 @@ static void decode_fill(DecodeArgs &a, const moe_w4_layer *layer, const uint16_t
   a.x = x;
   a.idx = idx;
   a.y_rows = y_rows;
+  a.g_gu = nullptr;
+  a.g_d = nullptr;
   a.T = T;
   a.k = k;
   a.E = layer->E;
@@ -727,7 +944,7 @@ extern "C" MOE_API moe_status moe_ffn_w4a16_decode(const moe_w4_layer *layer, co
   decode_fill(a, layer, x, idx, T, k, y_rows, static_cast<uint8_t *>(ws));
   a.err = device_error_word();
   if (!a.err) return MOE_ERR_CUDA;
-  return decode_launch<false, 8>(a, true, as_stream(stream));
+  return decode_launch<kFmtW4, false, 8>(a, true, as_stream(stream));
 }
 
 extern "C" MOE_API size_t moe_decode_layer_workspace_bytes(int T, int k, int H, int F) {
@@ -763,8 +980,46 @@ extern "C" MOE_API moe_status moe_decode_layer_w4a16(const moe_w4_layer *layer, 
                                                   sizeof(unsigned long long) * (size_t)T * k * F);
   a.err = device_error_word();
   if (!a.err) return MOE_ERR_CUDA;
-  if (E <= 256) return decode_launch<true, 8>(a, true, as_stream(stream));
-  return decode_launch<true, 32>(a, true, as_stream(stream));
+  if (E <= 256) return decode_launch<kFmtW4, true, 8>(a, true, as_stream(stream));
+  return decode_launch<kFmtW4, true, 32>(a, true, as_stream(stream));
+}
+
+extern "C" MOE_API moe_status moe_decode_layer_nvfp4(const moe_nvfp4_layer *layer,
+                                                     const uint16_t *x, const float *logits, int T,
+                                                     int k, uint16_t *y, int32_t *idx, float *w,
+                                                     void *ws, size_t ws_bytes,
+                                                     moe_stream_t stream) {
+  if (!layer || T < 0 || k <= 0) return MOE_ERR_INVALID_ARG;
+  const int E = layer->E, H = layer->H, F = layer->F;
+  if (E <= 0 || H <= 0 || F <= 0 || k > E) return MOE_ERR_INVALID_ARG;
+  if (H % 256 || F % 256 || E > kDecMaxE || T > kDecMaxTok || T * k > kDecMaxRows || k > 32)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return MOE_OK;
+  if (!layer->gate_up || !layer->down || !layer->g_gu || !layer->g_d || !x || !logits || !y)
+    return MOE_ERR_INVALID_ARG;
+  if ((idx == nullptr) != (w == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(layer->gate_up) % 16 ||
+      reinterpret_cast<uintptr_t>(layer->down) % 16 || reinterpret_cast<uintptr_t>(x) % 16 ||
+      reinterpret_cast<uintptr_t>(ws) % 16)
+    return MOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < moe_decode_layer_workspace_bytes(T, k, H, F)) return MOE_ERR_WORKSPACE;
+  moe_w4_layer l4 = {E, H, F, layer->gate_up, layer->down};
+  DecodeArgs a;
+  decode_fill(a, &l4, x, nullptr, T, k, nullptr, static_cast<uint8_t *>(ws));
+  a.gu_stride = (size_t)(2 * F / kBlkRows) * nvfp4_strip_bytes(H);
+  a.dn_stride = (size_t)(H / kBlkRows) * nvfp4_strip_bytes(F);
+  a.g_gu = layer->g_gu;
+  a.g_d = layer->g_d;
+  a.logits = logits;
+  a.y = y;
+  a.idx_out = idx;
+  a.w_out = w;
+  a.ybuf = reinterpret_cast<unsigned long long *>(static_cast<uint8_t *>(ws) + kDecCtrlBytes +
+                                                  sizeof(unsigned long long) * (size_t)T * k * F);
+  a.err = device_error_word();
+  if (!a.err) return MOE_ERR_CUDA;
+  if (E <= 256) return decode_launch<kFmtNvfp4, true, 8>(a, true, as_stream(stream));
+  return decode_launch<kFmtNvfp4, true, 32>(a, true, as_stream(stream));
 }
 
 // ---------------------------------------------------------------------------
@@ -838,5 +1093,5 @@ extern "C" MOE_API moe_status moe_ffn_w4a16_decode_static(const moe_w4_layer *la
     set_cuda_error(e);
     return MOE_ERR_CUDA;
   }
-  return decode_launch<false, 8>(a, false, as_stream(stream));
+  return decode_launch<kFmtW4, false, 8>(a, false, as_stream(stream));
 }

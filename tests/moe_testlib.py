@@ -64,6 +64,45 @@ class Layer:
         self.desc = moe.make_layer(E, H, F, self.gu, self.dn)
 
 
+class NvLayer:
+    """One NVFP4 MoE layer: canonical oracle weights (codes, sf, G) for the
+    experts that matter, packed device buffers and globals for all E."""
+
+    def __init__(self, seed, layer, E, H, F, experts):
+        self.E, self.H, self.F = E, H, F
+        self.canon = {}
+        gu_b = moe.moe_nvfp4_packed_bytes(2 * F, H)
+        d_b = moe.moe_nvfp4_packed_bytes(H, F)
+        self.gu = torch.zeros(E * gu_b, dtype=torch.uint8, device="cuda")
+        self.dn = torch.zeros(E * d_b, dtype=torch.uint8, device="cuda")
+        g_gu = np.ones(E, np.float32)
+        g_d = np.ones(E, np.float32)
+        for e in sorted(set(int(v) for v in experts)):
+            mats = []
+            for proj, (N, K) in ((synth.PROJ_GATE_UP, (2 * F, H)), (synth.PROJ_DOWN, (H, F))):
+                w = synth.expert_weights(seed, layer, e, proj, N, K)
+                G = oracle.nvfp4_global(w)
+                mats.append((*oracle.nvfp4_quantize(w, G), G))
+            self.canon[e] = tuple(mats)
+            g_gu[e], g_d[e] = mats[0][2], mats[1][2]
+            for (codes, sf, _), buf, nb, kind in ((mats[0], self.gu, gu_b, moe.MOE_W4_GATE_UP),
+                                                  (mats[1], self.dn, d_b, moe.MOE_W4_PLAIN)):
+                moe.moe_pack_nvfp4(torch.from_numpy(codes).cuda(), torch.from_numpy(sf).cuda(), kind,
+                                   buf[e * nb:(e + 1) * nb])
+        self.g_gu = torch.from_numpy(g_gu).cuda()
+        self.g_d = torch.from_numpy(g_d).cuda()
+        self.desc = moe.make_nvfp4_layer(E, H, F, self.gu, self.dn, self.g_gu, self.g_d)
+
+    def oracle_forward(self, x, logits, k):
+        """Oracle: route, per-row NVFP4 expert FFN, combine -> (idx, w, Y rows, y bf16 bits)."""
+        idx, w = oracle.route(logits, k)
+        T = x.shape[0]
+        Y = np.stack([oracle.expert_ffn_nvfp4(x[t], *self.canon[int(idx[t, j])])
+                      for t in range(T) for j in range(k)]).reshape(T, k, self.H)
+        y = np.stack([oracle.combine(Y[t], w[t:t + 1])[0] for t in range(T)])
+        return idx, w, Y, y
+
+
 def decode_workspace(T, k, F):
     n = moe.moe_decode_workspace_bytes(T, k, F)
     return torch.zeros(n, dtype=torch.uint8, device="cuda")
