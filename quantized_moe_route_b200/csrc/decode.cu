@@ -312,11 +312,13 @@ __device__ __forceinline__ void mma_f16_16816(float d[4], const uint32_t a[4], u
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Two f16 fragment halves from the E2M1 codes at bits [sh, sh+4) and
-// [sh+16, sh+20) of w: magnitude bits to 9..11, sign to 15, i.e. the code's
-// value times 2^-14 (sh <= 12).
-__device__ __forceinline__ uint32_t e2m1x2_f16(uint32_t w, int sh) {
-  return ((w << (9 - sh)) & 0x0E000E00u) | ((w << (12 - sh)) & 0x80008000u);
+// Two f16 fragment halves from the E2M1 codes at bits [SH, SH+4) and
+// [SH+16, SH+20) of w (SH = 0 or 4): magnitude bits to 9..11, sign to 15,
+// i.e. the code's value times 2^-14.
+template <int SH>
+__device__ __forceinline__ uint32_t e2m1x2_f16(uint32_t w) {
+  static_assert(SH == 0 || SH == 4, "nibble offset");
+  return ((w << (9 - SH)) & 0x0E000E00u) | ((w << (12 - SH)) & 0x80008000u);
 }
 
 __device__ __forceinline__ void e4m3x4_to_f32(uint32_t w, float f[4]) {
@@ -401,12 +403,13 @@ __device__ __forceinline__ void fp4_chunk_mma(const uint8_t *const (&strip)[NMAT
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int off = rowoff + ((((2 * g + (j >> 1)) & 7) ^ (gi & 7)) << 4) + 8 * (j & 1);
-      const uint32_t wlo = *reinterpret_cast<const uint32_t *>(strip[m] + off);
-      const uint32_t whi = *reinterpret_cast<const uint32_t *>(strip[m] + off + 8 * (K / 2));
-      af[m][j][0] = e2m1x2_f16(wlo, sh);
-      af[m][j][1] = e2m1x2_f16(whi, sh);
-      af[m][j][2] = e2m1x2_f16(wlo, sh + 4);
-      af[m][j][3] = e2m1x2_f16(whi, sh + 4);
+      // this lane's bytes (t & 1) and (t & 1) + 2 of the word, moved to bytes 0 and 2
+      const uint32_t wlo = *reinterpret_cast<const uint32_t *>(strip[m] + off) >> sh;
+      const uint32_t whi = *reinterpret_cast<const uint32_t *>(strip[m] + off + 8 * (K / 2)) >> sh;
+      af[m][j][0] = e2m1x2_f16<0>(wlo);
+      af[m][j][1] = e2m1x2_f16<0>(whi);
+      af[m][j][2] = e2m1x2_f16<4>(wlo);
+      af[m][j][3] = e2m1x2_f16<4>(whi);
     }
     const uint8_t *sc = strip[m] + 8 * K + 64 * g;
     e4m3x4_to_f32(*reinterpret_cast<const uint32_t *>(sc + 4 * gi), slo[m]);
