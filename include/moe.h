@@ -355,6 +355,33 @@ MOE_API moe_status moe_ffn_grouped_prefill(const moe_w4_layer *layer, const uint
                                            void *ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * Prefill with NVFP4 experts: grouped GEMM over experts on the block-scaled
+ * tensor cores (tcgen05 kind::mxf4nvf4: E2M1 x E2M1 with E4M3 scales per 16
+ * channels, fp32 accumulation in tensor memory; nothing is dequantised).
+ * Inputs: the rows grouped by expert and already quantised per row
+ * (moe_quantize_nvfp4_rows with src_rows = sorted_rows, src_div = k):
+ * x_codes [rows][H/2], x_sf [rows][H/16], x_G [rows]; offsets [E+1] (from
+ * moe_permute).  Writes y_perm bf16 [rows][H]:
+ *   g, u = (W_gate x, W_up x) * x_G * g_gu[e];  h = SiLU(g) * u   (fp32)
+ *   h -> NVFP4 per row (as moe_quantize_nvfp4_rows);  y = (W_down h) * h_G * g_d[e]
+ * Source: "Drama 3 - NVFP4 routed experts", section "Quantization" (NVFP4
+ * weights and dynamic per-token activation scales), "drama-rs", "Layout"
+ * (grouped MoE prefill).
+ * Workspace: moe_prefill_nvfp4_workspace_bytes(rows, F) bytes, 256-byte
+ * aligned: h fp32 [rows][F], then its codes [rows][F/2], scales [rows][F/16]
+ * and globals [rows], each section starting on a 256-byte boundary.
+ * Requirements: H % 256 == 0, F % 256 == 0, E <= 960, offsets as for
+ * moe_ffn_grouped_prefill; x_codes, x_sf, y_perm 16-byte aligned.  rows == 0
+ * is a no-op.
+ */
+MOE_API size_t moe_prefill_nvfp4_workspace_bytes(int rows, int F);
+MOE_API moe_status moe_ffn_grouped_prefill_nvfp4(const moe_nvfp4_layer *layer,
+                                                 const uint8_t *x_codes, const uint8_t *x_sf,
+                                                 const float *x_G, const int32_t *offsets,
+                                                 int rows, uint16_t *y_perm, void *ws,
+                                                 size_t ws_bytes, moe_stream_t stream);
+
+/*
  * Router-weighted combine: y[t] = sum over j = 0..k-1 (in that order) of
  * w[t][j] * Y[p(t*k + j)], accumulated in fp32 and rounded to nearest-even
  * bf16.  Y is y_rows (fp32, y_dtype 0) or y_perm (bf16, y_dtype 1), [T*k][H];

@@ -74,6 +74,9 @@ SIGNATURES = {
                                     _sz, _vp]),
     "moe_prefill_workspace_bytes": (_sz, [_i, _i]),
     "moe_ffn_grouped_prefill": (_i, [ctypes.POINTER(moe_w4_layer), _vp, _vp, _i, _vp, _vp, _sz, _vp]),
+    "moe_prefill_nvfp4_workspace_bytes": (_sz, [_i, _i]),
+    "moe_ffn_grouped_prefill_nvfp4": (_i, [ctypes.POINTER(moe_nvfp4_layer), _vp, _vp, _vp, _vp, _i, _vp, _vp, _sz,
+                                           _vp]),
     "moe_unpermute_combine": (_i, [_vp, _i, _vp, _vp, _i, _i, _i, _vp, _vp]),
     "moe_device_error": (_i, [ctypes.POINTER(ctypes.c_int), _vp]),
 }
@@ -238,6 +241,17 @@ def moe_decode_layer_nvfp4(layer: moe_nvfp4_layer, x, logits, k, y, ws, idx=None
     _check(lib().moe_decode_layer_nvfp4(ctypes.byref(layer), _p(x), _p(logits), T, k, _p(y), _p(idx), _p(w),
                                         _p(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "moe_decode_layer_nvfp4")
+
+
+def moe_prefill_nvfp4_workspace_bytes(rows, F) -> int:
+    return lib().moe_prefill_nvfp4_workspace_bytes(rows, F)
+
+
+def moe_ffn_grouped_prefill_nvfp4(layer: moe_nvfp4_layer, x_codes, x_sf, x_G, offsets, y_perm, ws, stream=None):
+    rows = x_codes.shape[0]
+    _check(lib().moe_ffn_grouped_prefill_nvfp4(ctypes.byref(layer), _p(x_codes), _p(x_sf), _p(x_G), _p(offsets),
+                                               rows, _p(y_perm), _p(ws), ws.numel() * ws.element_size(),
+                                               _stream(stream)), "moe_ffn_grouped_prefill_nvfp4")
 
 
 def moe_prefill_workspace_bytes(rows, F) -> int:
