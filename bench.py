@@ -38,6 +38,11 @@ EXPERT_BYTES = 1769472  # packed int4 gate/up + down of one expert (36 B per 64 
 METRIC = "routed-expert tokens/s + HBM GB/s (decode), TFLOP/s (prefill) vs roofline"
 WORKLOAD = ("single-layer decode: 256 experts, top-8, hidden 2048, expert width 512, 1 token per step; "
             "steps rotate over 40 resident int4 layers (18.1 GB) with fresh router logits per layer")
+NV_WORKLOAD = ("NVFP4 single-layer decode: 256 experts, top-8, hidden 2048, expert width 512, 1 token per step; "
+               "E2M1 weights with E4M3 scales per 16 channels and fp32 per-matrix globals, x and h quantised "
+               "per token/row in the kernel; steps rotate over 40 resident NVFP4 layers (18.1 GB)")
+DTYPE_W4 = "int4 weights (f16 scale/min), bf16 activations, fp32 accumulate"
+DTYPE_NV = "nvfp4 weights and activations (e2m1 + e4m3/16 + fp32 global), fp32 accumulate"
 
 
 # ---------------------------------------------------------------------------- helpers
@@ -137,11 +142,14 @@ def dist_barrier():
 
 
 # ---------------------------------------------------------------------------- workload
-def build_layers(L, seed, log):
-    """40 resident layers of packed int4 experts, generated and quantised on the GPU."""
+def build_layers(L, seed, log, fmt="w4"):
+    """Resident layers of packed experts (int4, or NVFP4 with fmt="nvfp4"),
+    generated, quantised and packed on the GPU."""
     import torch
     import synth
     import quantized_moe_route_b200 as moe
+    if fmt == "nvfp4":
+        return build_layers_nvfp4(L, seed, log)
     gu_b, d_b = moe.moe_w4_packed_bytes(2 * F, H), moe.moe_w4_packed_bytes(H, F)
     chunk = 32
     tmp = torch.empty((chunk, 2 * F, H), dtype=torch.float32, device="cuda")
@@ -174,6 +182,41 @@ def build_layers(L, seed, log):
     return layers
 
 
+def build_layers_nvfp4(L, seed, log):
+    import torch
+    import synth
+    import quantized_moe_route_b200 as moe
+    gu_b, d_b = moe.moe_nvfp4_packed_bytes(2 * F, H), moe.moe_nvfp4_packed_bytes(H, F)
+    chunk = 32
+    tmp = torch.empty((chunk, 2 * F, H), dtype=torch.float32, device="cuda")
+    codes = torch.empty((2 * F, H), dtype=torch.uint8, device="cuda")
+    sf = torch.empty((2 * F, H // 16), dtype=torch.uint8, device="cuda")
+    layers = []
+    t0 = time.time()
+    for l in range(L):
+        gu = torch.empty(E * gu_b, dtype=torch.uint8, device="cuda")
+        dn = torch.empty(E * d_b, dtype=torch.uint8, device="cuda")
+        g_gu = torch.empty(E, dtype=torch.float32, device="cuda")
+        g_d = torch.empty(E, dtype=torch.float32, device="cuda")
+        for proj, buf, nb, (N, K), kind, gl in ((synth.PROJ_GATE_UP, gu, gu_b, (2 * F, H), moe.MOE_W4_GATE_UP, g_gu),
+                                                 (synth.PROJ_DOWN, dn, d_b, (H, F), moe.MOE_W4_PLAIN, g_d)):
+            c = codes.view(-1)[: N * K].view(N, K)
+            s = sf.view(-1)[: N * K // 16].view(N, K // 16)
+            for e0 in range(0, E, chunk):
+                w = tmp.view(-1)[: chunk * N * K].view(chunk, N, K)
+                synth.cuda_expert_weights(w, seed, l, e0, proj)
+                for i in range(chunk):
+                    e = e0 + i
+                    moe.moe_nvfp4_global(w[i], gl[e:e + 1])
+                    moe.moe_quantize_nvfp4(w[i], gl[e:e + 1], c, s)
+                    moe.moe_pack_nvfp4(c, s, kind, buf[e * nb:(e + 1) * nb])
+        layers.append((gu, dn, moe.make_nvfp4_layer(E, H, F, gu, dn, g_gu, g_d), g_gu, g_d))
+    torch.cuda.synchronize()
+    del tmp, codes, sf
+    log(f"built {L} NVFP4 layers in {time.time() - t0:.1f}s")
+    return layers
+
+
 def layer_inputs(seed, l, T):
     import synth
     x = synth.activations_bf16(seed, l, T, H)
@@ -191,7 +234,9 @@ def run_gpu(args, log):
     dev = torch.device("cuda", local)
     T = args.tokens
     seed = 1000 + rank
-    layers = build_layers(LAYERS, seed, log)
+    fmt = "nvfp4" if args.workload == "nvfp4-decode" else "w4"
+    layers = build_layers(LAYERS, seed, log, fmt)
+    decode_layer = moe.moe_decode_layer_nvfp4 if fmt == "nvfp4" else moe.moe_decode_layer_w4a16
     k = TOPK
     # per-layer device inputs (activations and router logits of every layer)
     xs, ls, uniq = [], [], []
@@ -208,7 +253,7 @@ def run_gpu(args, log):
         # one launch: route + weight-streaming expert FFN + combine
         if ev is not None:
             ev[0].record(stream)
-        moe.moe_decode_layer_w4a16(layers[l][2], xs[l], ls[l], k, y, ws, stream=stream)
+        decode_layer(layers[l][2], xs[l], ls[l], k, y, ws, stream=stream)
         if ev is not None:
             ev[1].record(stream)
 
@@ -292,7 +337,7 @@ def run_gpu(args, log):
     def e2e_step(l):
         dx.copy_(hx[l], non_blocking=True)
         dl.copy_(hl[l], non_blocking=True)
-        moe.moe_decode_layer_w4a16(layers[l][2], dx, dl, k, y, ws, stream=stream)
+        decode_layer(layers[l][2], dx, dl, k, y, ws, stream=stream)
         hy.copy_(y, non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -314,15 +359,16 @@ def run_gpu(args, log):
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "int4 weights (f16 scale/min), bf16 activations, fp32 accumulate", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "experts": E, "top_k": k, "hidden": H, "expert_width": F,
-                   "tokens_per_step": T, "resident_layers": LAYERS, "seed": 1000,
+        "dtype": DTYPE_NV if fmt == "nvfp4" else DTYPE_W4, "data": "synthetic",
+        "config": {"workload": NV_WORKLOAD if fmt == "nvfp4" else WORKLOAD, "experts": E, "top_k": k, "hidden": H,
+                   "expert_width": F, "tokens_per_step": T, "resident_layers": LAYERS, "seed": 1000,
                    "l2": f"inputs larger than L2 ({LAYERS}-layer rotation, {LAYERS * E * EXPERT_BYTES / 1e9:.1f} GB)",
                    "parallelism": f"replicas x{world}",
                    "launch": f"one kernel per step (route + FFN + combine), CUDA graphs of "
                              f"{min(K, args.graph_steps)} steps, programmatic dependent launch"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None, "kernel": "moe::decode_kernel<fused>",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": f"moe::decode_kernel<{'nvfp4' if fmt == 'nvfp4' else 'int4'}, fused>",
                      "peak_kind": peak_kind, "alg_bytes_per_launch": alg_bytes,
                      "avg_launch_us": dur_ms * 1e3, "isolated_launch_us": isolated_ms * 1e3},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2 + T * E * 4,
@@ -331,7 +377,7 @@ def run_gpu(args, log):
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(seed, T, budget_s=args.cpu_seconds, log=log)
+        out["cpu_baseline"] = cpu_baseline(seed, T, budget_s=args.cpu_seconds, log=log, fmt=fmt)
     del g_main, g_warm, g_prof, g_e2e
     if world > 1:
         import torch.distributed as dist
@@ -476,6 +522,181 @@ def run_gpu_prefill(args, log):
     return out if rank == 0 else None
 
 
+NVP_WORKLOAD = ("NVFP4 grouped prefill: 512 tokens x top-8 = 4,096 routed rows over 256 experts (router logits "
+                "N(0,1) + Zipf(1.1) expert bias), hidden 2048, expert width 512; route, permute, per-row NVFP4 "
+                "quantisation of the grouped rows, block-scaled tcgen05 grouped FFN, combine; 8 resident layers rotated")
+
+
+def run_gpu_prefill_nvfp4(args, log):
+    """Config 5's prefill leg: HBM-bound (the touched experts' 4.5-bit weights
+    dominate the bytes; the FP4 tensor cores need a few microseconds)."""
+    import torch
+    import synth
+    import quantized_moe_route_b200 as moe
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    T, k, nl = args.tokens, TOPK, args.layers
+    seed = 4000 + rank
+    layers = build_layers(nl, seed, log, "nvfp4")
+    bias = synth.zipf_bias(seed, E)
+    xs, ls, uniq = [], [], []
+    for l in range(nl):
+        xs.append(torch.from_numpy(synth.activations_bf16(seed, l, T, H).view(np.int16)).to(dev))
+        lg = (synth.router_logits(seed, l, T, E) + bias[None, :]).astype(np.float32)
+        ls.append(torch.from_numpy(lg).to(dev))
+        uniq.append(len(set(np.argsort(-lg, axis=1, kind="stable")[:, :k].ravel().tolist())))
+    R = T * k
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    sorted_rows = torch.empty(R, dtype=torch.int32, device=dev)
+    inv = torch.empty(R, dtype=torch.int32, device=dev)
+    pws = torch.empty(moe.moe_permute_workspace_bytes(T, k, E), dtype=torch.uint8, device=dev)
+    xc = torch.empty((R, H // 2), dtype=torch.uint8, device=dev)
+    xsf = torch.empty((R, H // 16), dtype=torch.uint8, device=dev)
+    xg = torch.empty(R, dtype=torch.float32, device=dev)
+    y_perm = torch.empty((R, H), dtype=torch.int16, device=dev)
+    fws = torch.empty(moe.moe_prefill_nvfp4_workspace_bytes(R, F), dtype=torch.uint8, device=dev)
+    y = torch.empty((T, H), dtype=torch.int16, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(l, ev=None, xin=None, lin=None):
+        moe.moe_route(ls[l] if lin is None else lin, k, idx, w, stream=stream)
+        moe.moe_permute(idx, E, counts, offsets, sorted_rows, inv, pws, stream=stream)
+        moe.moe_quantize_nvfp4_rows(xs[l] if xin is None else xin, xc, xsf, xg, src_rows=sorted_rows, src_div=k,
+                                    rows=R, stream=stream)
+        if ev is not None:
+            ev[0].record(stream)
+        moe.moe_ffn_grouped_prefill_nvfp4(layers[l][2], xc, xsf, xg, offsets, y_perm, fws, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        moe.moe_unpermute_combine(y_perm, w, y, inv=inv, stream=stream)
+
+    K, W = args.steps, args.warmup
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            step(i % nl)
+    torch.cuda.synchronize()
+    dist_barrier()
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        dist_barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(K):
+                step((W + i) % nl)
+            e1.record(stream)
+        e1.synchronize()
+        torch.cuda.synchronize()
+        dist_barrier()
+    ms = dist_max(e0.elapsed_time(e1))
+    tokens = K * T * world
+    value = tokens / (ms / 1e3)
+
+    # kernel-duration pass: events around the grouped FFN call (gate/up, h
+    # quantisation, down: three launches)
+    P = min(K, 50)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(P)]
+    with torch.cuda.stream(stream):
+        for i in range(P):
+            step((W + i) % nl, evs[i])
+    torch.cuda.synchronize()
+    dur_ms = sum(a.elapsed_time(b) for a, b in evs) / P
+    # algorithmic bytes of the call: touched experts' packed weights, the
+    # quantised rows in, h out (fp32) and back in, its codes out and in, y_perm out
+    act = R * (H // 2 + H // 16 + 4)
+    hq = R * (F // 2 + F // 16 + 4)
+    alg_bytes = sum(uniq[(W + i) % nl] * EXPERT_BYTES for i in range(P)) / P + act + 2 * R * F * 4 + 2 * hq + R * H * 2
+    peak, peak_kind = peaks()
+    achieved = alg_bytes / (dur_ms / 1e3) / 1e9
+    flops = R * 6.0 * H * F
+
+    import synth as _s
+    hx = [torch.from_numpy(_s.activations_bf16(seed, l, T, H).view(np.int16)).pin_memory() for l in range(nl)]
+    hl = [torch.from_numpy((_s.router_logits(seed, l, T, E) + bias[None, :]).astype(np.float32)).pin_memory()
+          for l in range(nl)]
+    hy = torch.empty((T, H), dtype=torch.int16).pin_memory()
+    dx = torch.empty((T, H), dtype=torch.int16, device=dev)
+    dl = torch.empty((T, E), dtype=torch.float32, device=dev)
+    with torch.cuda.stream(stream):
+        for i in range(2):
+            dx.copy_(hx[i % nl], non_blocking=True)
+            dl.copy_(hl[i % nl], non_blocking=True)
+            step(i % nl, xin=dx, lin=dl)
+            hy.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a0.record(stream)
+        for i in range(K):
+            dx.copy_(hx[(W + i) % nl], non_blocking=True)
+            dl.copy_(hl[(W + i) % nl], non_blocking=True)
+            step((W + i) % nl, xin=dx, lin=dl)
+            hy.copy_(y, non_blocking=True)
+        a1.record(stream)
+    a1.synchronize()
+    e2e_ms = dist_max(a0.elapsed_time(a1))
+
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": DTYPE_NV, "data": "synthetic",
+        "config": {"workload": NVP_WORKLOAD, "experts": E, "top_k": k, "hidden": H, "expert_width": F,
+                   "tokens_per_step": T, "routed_rows": R, "resident_layers": nl,
+                   "l2": f"inputs larger than L2 ({nl} layers x 453 MB of experts rotated)",
+                   "parallelism": f"replicas x{world}", "launch": "stream-ordered, PDL into the FFN kernels"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "moe::prefill_nvfp4_kernel (gate/up + h quantise + down launches)",
+                     "peak_kind": peak_kind, "alg_bytes_per_call": alg_bytes, "avg_call_us": dur_ms * 1e3,
+                     "tflops": flops / (dur_ms / 1e3) / 1e12},
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2 + T * E * 4,
+                "d2h_bytes_per_step": T * H * 2},
+        "gpu_launches": 9 * K,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline_prefill_nvfp4(seed, bias, T, budget_s=args.cpu_seconds, log=log)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return out if rank == 0 else None
+
+
+def cpu_baseline_prefill_nvfp4(seed, bias, T, budget_s, log):
+    """The oracle on sampled tokens of the NVFP4 prefill batch (tokens/s)."""
+    import oracle
+    import synth
+    import torch
+    x = synth.activations_bf16(seed, 0, T, H)
+    lg = (synth.router_logits(seed, 0, T, E) + bias[None, :]).astype(np.float32)
+    idx, _ = oracle.route(lg, TOPK)
+    toks = list(range(0, T, 61))[:6]
+    experts = {}
+    for e in sorted(set(idx[toks].ravel().tolist())):
+        wg = torch.empty((1, 2 * F, H), device="cuda")
+        wd = torch.empty((1, H, F), device="cuda")
+        synth.cuda_expert_weights(wg, seed, 0, e, synth.PROJ_GATE_UP)
+        synth.cuda_expert_weights(wd, seed, 0, e, synth.PROJ_DOWN)
+        experts[e] = (oracle_quantize(wg[0].cpu().numpy(), "nvfp4"), oracle_quantize(wd[0].cpu().numpy(), "nvfp4"))
+    t0 = time.time()
+    n = 0
+    while True:
+        t = toks[n % len(toks)]
+        oracle_forward(x[t:t + 1], lg[t:t + 1], experts, "nvfp4")
+        n += 1
+        if time.time() - t0 >= budget_s:
+            break
+    dt = time.time() - t0
+    return {"value": n / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} tokens of the {T}-token NVFP4 prefill batch ({len(toks)} distinct, all 8 experts each), "
+                      f"{dt:.1f}s"}
+
+
 def cpu_baseline_prefill(seed, bias, budget_s, log):
     """The oracle on sampled tokens of the prefill workload (rows per second
     scaled to tokens/s); weights of the sampled tokens' experts only."""
@@ -509,7 +730,28 @@ def cpu_baseline_prefill(seed, bias, budget_s, log):
 
 
 # ---------------------------------------------------------------------------- CPU oracle
-def oracle_pool(seed, T, n, log, use_gpu_generator):
+def oracle_quantize(w, fmt):
+    import oracle
+    if fmt == "nvfp4":
+        G = oracle.nvfp4_global(w)
+        return (*oracle.nvfp4_quantize(w, G), G)
+    return oracle.quantize_w4(w)
+
+
+def oracle_forward(x, lg, experts, fmt):
+    """One layer through the oracle: route, expert FFN per row, combine."""
+    import oracle
+    if fmt != "nvfp4":
+        return oracle.moe_forward_w4(x, lg, TOPK, experts)[3]
+    idx, w = oracle.route(lg, TOPK)
+    ys = []
+    for t in range(x.shape[0]):
+        Y = np.stack([oracle.expert_ffn_nvfp4(x[t], *experts[int(e)]) for e in idx[t]])
+        ys.append(oracle.combine(Y, w[t:t + 1])[0])
+    return np.stack(ys)
+
+
+def oracle_pool(seed, T, n, log, use_gpu_generator, fmt="w4"):
     """n sampled token-layers: canonical weights of their routed experts, built
     with the seeded generator and the oracle's own quantiser."""
     import oracle
@@ -531,20 +773,19 @@ def oracle_pool(seed, T, n, log, use_gpu_generator):
             else:
                 a = synth.expert_weights(seed, l, e, synth.PROJ_GATE_UP, 2 * F, H)
                 b = synth.expert_weights(seed, l, e, synth.PROJ_DOWN, H, F)
-            experts[e] = (oracle.quantize_w4(a), oracle.quantize_w4(b))
+            experts[e] = (oracle_quantize(a, fmt), oracle_quantize(b, fmt))
         pool.append((x, lg, experts))
     log(f"oracle pool of {n} token-layers built in {time.time() - t0:.1f}s")
     return pool
 
 
-def cpu_baseline(seed, T, budget_s, log):
-    import oracle
-    pool = oracle_pool(seed, T, 4, log, use_gpu_generator=True)
+def cpu_baseline(seed, T, budget_s, log, fmt="w4"):
+    pool = oracle_pool(seed, T, 4, log, use_gpu_generator=True, fmt=fmt)
     t0 = time.time()
     n = 0
     while True:
         x, lg, experts = pool[n % len(pool)]
-        oracle.moe_forward_w4(x, lg, TOPK, experts)
+        oracle_forward(x, lg, experts, fmt)
         n += 1
         if time.time() - t0 >= budget_s:
             break
@@ -589,7 +830,7 @@ def main():
     ap.add_argument("--steps", type=int, default=100000, help="timed steps")
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "nvfp4-decode", "nvfp4-prefill"])
     ap.add_argument("--tokens", type=int, default=None, help="tokens per step (decode 1, prefill 2048)")
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="resident layers the steps rotate over (40 = 18.1 GB, larger than L2)")
@@ -601,9 +842,11 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
     if args.tokens is None:
-        args.tokens = 2048 if args.workload == "prefill" else 1
+        args.tokens = {"prefill": 2048, "nvfp4-prefill": 512}.get(args.workload, 1)
     if args.workload == "prefill" and args.layers == LAYERS:
         args.layers = 4
+    if args.workload == "nvfp4-prefill" and args.layers == LAYERS:
+        args.layers = 8
 
     def log(msg):
         if not args.quiet:
@@ -613,6 +856,8 @@ def main():
         out = run_reference(args, log)
     elif args.workload == "prefill":
         out = run_gpu_prefill(args, log)
+    elif args.workload == "nvfp4-prefill":
+        out = run_gpu_prefill_nvfp4(args, log)
     else:
         out = run_gpu(args, log)
     if out is not None:

@@ -14,13 +14,16 @@
 // Per stage of 256 channels:
 //   warp 0      TMA: weight code tiles (the packed rows are stored with the
 //               128-byte swizzle already applied, so a plain box is a ready
-//               operand), weight scales, activation codes (128-byte swizzle on
-//               the fly) and scales
+//               operand), weight scales, and only the 32-row boxes of
+//               activation codes (128-byte swizzle on the fly) and scales that
+//               hold the tile's rows
 //   warp 2      rearranges the stage's scales into the tensor-memory scale
 //               layout (per 64 channels: 32 rows x {4 row groups x 4 scales})
 //   warp 1      tcgen05.cp of the scales into tensor memory, then four
 //               block-scaled MMAs per matrix (K = 64 each), commit -> stage free
-//   warps 4..7  epilogue from tensor memory (tcgen05.ld)
+//   warps 4..11 epilogue from tensor memory (tcgen05.ld), two warps per lane
+//               quarter; the down launch keeps two accumulator sets so its
+//               epilogue overlaps the next tile's MMAs
 // Every wait is bounded; a timeout raises the device error word.
 #include "common.cuh"
 #include "nvfp4.cuh"
@@ -31,7 +34,9 @@ namespace moe {
 constexpr int kNpBM = 128;   // weight rows per matrix per tile (MMA M)
 constexpr int kNpBN = 128;   // rows (tokens) per tile; the MMA's N is trimmed to the valid rows
 constexpr int kNpKT = 256;   // channels per stage: 128 code bytes per row
-constexpr int kNpThreads = 8 * 32;
+constexpr int kNpBoxRows = 32;  // activation rows per TMA box (a tile loads the boxes it needs)
+constexpr int kNpEpiWarps = 8;  // warps 4..11: two per tensor-memory lane quarter
+constexpr int kNpThreads = (4 + kNpEpiWarps) * 32;
 constexpr uint32_t kNpWaitLimit = 1u << 24;
 
 template <bool kGU>
@@ -50,14 +55,19 @@ struct NpCfg {
   static constexpr uint32_t kOffAAtom = kOffBRaw + kBRaw;
   static constexpr uint32_t kOffBAtom = kOffAAtom + kMats * 4 * kAtom;
   static constexpr uint32_t kStageBytes = (kOffBAtom + 4 * kAtom + 1023) / 1024 * 1024;
-  static constexpr uint32_t kTxBytes = kMats * (kACodes + kARaw) + kBCodes + kBRaw;
+  static constexpr uint32_t kATxBytes = kMats * (kACodes + kARaw);
+  static constexpr uint32_t kBoxTxBytes = kNpBoxRows * (128 + 16);
   static constexpr uint32_t kTailOff = kStages * kStageBytes;
   static constexpr uint32_t kSmemBytes = kTailOff + 1024 /*align slack*/ + 4096;
-  // tensor memory: accumulators [kMats][BN], then per stage the scales:
-  // A (kMats x 4 blocks of 64 channels x 4 columns), B (4 x 4 columns)
+  // tensor memory: kAcc accumulator sets of [kMats][BN] columns (down keeps
+  // two, so the epilogue of one tile overlaps the next tile's MMAs), then
+  // per stage the scales: A (kMats x 4 blocks of 64 channels x 4 columns),
+  // B (4 x 4 columns)
+  static constexpr int kAcc = kGU ? 1 : 2;
+  static constexpr uint32_t kAccCols = kMats * kNpBN;
   static constexpr uint32_t kSfCols = (kMats + 1) * 16;
   static constexpr uint32_t kTmemCols = 512;
-  static_assert(kMats * kNpBN + kStages * kSfCols <= kTmemCols, "tensor memory");
+  static_assert(kAcc * kAccCols + kStages * kSfCols <= kTmemCols, "tensor memory");
   static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
@@ -141,9 +151,9 @@ __global__ void __launch_bounds__(kNpThreads, 1)
   uint64_t *full = reinterpret_cast<uint64_t *>(tail);
   uint64_t *sfready = full + C::kStages;
   uint64_t *empty = sfready + C::kStages;
-  uint64_t *tmem_full = empty + C::kStages;
-  uint64_t *tmem_empty = tmem_full + 1;
-  uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(tmem_empty + 1);
+  uint64_t *tmem_full = empty + C::kStages;   // [kAcc]
+  uint64_t *tmem_empty = tmem_full + C::kAcc;  // [kAcc]
+  uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(tmem_empty + C::kAcc);
   volatile int *abort_s = reinterpret_cast<volatile int *>(tmem_base_s + 1);
   int *ntiles_s = const_cast<int *>(abort_s) + 1;
   int *chunk_start = ntiles_s + 1;  // [E + 1]
@@ -157,8 +167,10 @@ __global__ void __launch_bounds__(kNpThreads, 1)
       mbar_init(&sfready[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(tmem_full, 1);
-    mbar_init(tmem_empty, 128);
+    for (int b = 0; b < C::kAcc; ++b) {
+      mbar_init(&tmem_full[b], 1);
+      mbar_init(&tmem_empty[b], kNpEpiWarps * 32);
+    }
     *abort_s = 0;
     fence_mbar_init();
   }
@@ -210,7 +222,8 @@ __global__ void __launch_bounds__(kNpThreads, 1)
             break;
           }
           uint8_t *st = smem + s * C::kStageBytes;
-          mbar_arrive_expect_tx(&full[s], C::kTxBytes);
+          const int nbox = (ti.nvalid + kNpBoxRows - 1) / kNpBoxRows;
+          mbar_arrive_expect_tx(&full[s], C::kATxBytes + (uint32_t)nbox * C::kBoxTxBytes);
           for (int m = 0; m < C::kMats; ++m) {
             if (kGU) {
               tma_load_4d(st + C::kOffA + m * C::kACodes, &wmap, kt * 128, 0, m, strip0, &full[s]);
@@ -220,8 +233,12 @@ __global__ void __launch_bounds__(kNpThreads, 1)
               tma_load_2d(st + C::kOffARaw, &wsmap, kt * 256, strip0, &full[s]);
             }
           }
-          tma_load_2d(st + C::kOffB, &bmap, kt * 128, ti.row0, &full[s]);
-          tma_load_2d(st + C::kOffBRaw, &bsmap, kt * 16, ti.row0, &full[s]);
+          for (int b = 0; b < nbox; ++b) {
+            tma_load_2d(st + C::kOffB + b * kNpBoxRows * 128, &bmap, kt * 128, ti.row0 + b * kNpBoxRows,
+                        &full[s]);
+            tma_load_2d(st + C::kOffBRaw + b * kNpBoxRows * 16, &bsmap, kt * 16, ti.row0 + b * kNpBoxRows,
+                        &full[s]);
+          }
         }
       }
     }
@@ -240,15 +257,16 @@ __global__ void __launch_bounds__(kNpThreads, 1)
         }
         uint8_t *st = smem + s * C::kStageBytes;
         // weights: raw [8 strips][4 blocks of 64][16 rows][4] -> per block,
-        // word (R % 32) * 4 + R / 32 for tile row R = 16 strip + row
+        // words 4 l .. 4 l + 3 = tile rows l, l + 32, l + 64, l + 96 (row R
+        // is row R % 16 of strip R / 16)
         for (int m = 0; m < C::kMats; ++m) {
           const uint32_t *raw = reinterpret_cast<const uint32_t *>(st + C::kOffARaw + m * C::kARaw);
-          uint32_t *atom = reinterpret_cast<uint32_t *>(st + C::kOffAAtom + m * 4 * C::kAtom);
-#pragma unroll 4
-          for (int idx = lane; idx < 512; idx += 32) {
-            const int i = idx >> 6, c = (idx >> 4) & 3, r = idx & 15, R = 16 * i + r;
-            atom[c * 128 + (R & 31) * 4 + (R >> 5)] = raw[idx];
-          }
+          uint4 *atom = reinterpret_cast<uint4 *>(st + C::kOffAAtom + m * 4 * C::kAtom);
+          const int rbase = (lane >> 4) * 64 + (lane & 15);
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            atom[c * 32 + lane] = make_uint4(raw[rbase + c * 16], raw[rbase + 128 + c * 16],
+                                             raw[rbase + 256 + c * 16], raw[rbase + 384 + c * 16]);
         }
         // activations: raw [128 rows][4 blocks][4] -> per block, row n at
         // 16 (n % 32) + 4 (n / 32): lane l moves rows l, l+32, l+64, l+96
@@ -273,7 +291,9 @@ __global__ void __launch_bounds__(kNpThreads, 1)
       for (int t = blockIdx.x; t < ntiles && !*abort_s; t += G, ++tcount) {
         const NpTile ti = np_tile(t, a.n_sub, chunk_start, a.E, a.offsets);
         const uint32_t idesc = idesc_nvf4((ti.nvalid + 15) & ~15);
-        if (!mbar_wait_bounded(tmem_empty, (tcount & 1u) ^ 1u, kNpWaitLimit)) {
+        const int ab = tcount % C::kAcc;
+        const uint32_t acc0 = tmem_base + ab * C::kAccCols;
+        if (!mbar_wait_bounded(&tmem_empty[ab], ((tcount / C::kAcc) & 1u) ^ 1u, kNpWaitLimit)) {
           fail();
           break;
         }
@@ -289,7 +309,7 @@ __global__ void __launch_bounds__(kNpThreads, 1)
           }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + s * C::kStageBytes);
-          const uint32_t sf0 = tmem_base + C::kMats * kNpBN + s * C::kSfCols;
+          const uint32_t sf0 = tmem_base + C::kAcc * C::kAccCols + s * C::kSfCols;
 #pragma unroll
           for (int m = 0; m < C::kMats; ++m)
 #pragma unroll
@@ -305,31 +325,33 @@ __global__ void __launch_bounds__(kNpThreads, 1)
 #pragma unroll
             for (int m = 0; m < C::kMats; ++m) {
               const uint64_t adesc = smem_desc_sw128(sa + C::kOffA + m * C::kACodes + kb * 32);
-              tc_mma_nvf4(tmem_base + m * kNpBN, adesc, bdesc, idesc, sf0 + m * 16 + kb * 4,
+              tc_mma_nvf4(acc0 + m * kNpBN, adesc, bdesc, idesc, sf0 + m * 16 + kb * 4,
                           sf0 + C::kMats * 16 + kb * 4, (kt | kb) ? 1u : 0u);
             }
           }
           tc_commit(&empty[s]);  // stage (and its tensor-memory scales) free once these MMAs are done
         }
         if (!ok) break;
-        tc_commit(tmem_full);
+        tc_commit(&tmem_full[ab]);
       }
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // tensor-memory lane quarter of this warp
+    const int q = warp & 3;            // tensor-memory lane quarter of this warp
+    const int half = (warp - 4) >> 2;  // the two warps of a quarter take alternate 16-column chunks
     uint32_t tcount = 0;
     for (int t = blockIdx.x; t < ntiles; t += G, ++tcount) {
       const NpTile ti = np_tile(t, a.n_sub, chunk_start, a.E, a.offsets);
-      if (!mbar_wait_bounded(tmem_full, tcount & 1u, kNpWaitLimit) || *abort_s) {
+      const int ab = tcount % C::kAcc;
+      if (!mbar_wait_bounded(&tmem_full[ab], (tcount / C::kAcc) & 1u, kNpWaitLimit) || *abort_s) {
         if (lane == 0 && !*abort_s) fail();
         break;
       }
       tc_fence_after();
       const int wrow = ti.sub * kNpBM + q * 32 + lane;  // feature (gate/up) or output channel (down)
-      const uint32_t trow = tmem_base + ((uint32_t)(q * 32) << 16);
+      const uint32_t trow = tmem_base + ab * C::kAccCols + ((uint32_t)(q * 32) << 16);
       const float wG = a.w_G[ti.e];
-      for (int c0 = 0; c0 < ti.nvalid; c0 += 16) {
+      for (int c0 = 16 * half; c0 < ti.nvalid; c0 += 32) {
         uint32_t v0[16], v1[16];
         tmem_ld16(trow + c0, v0);
         if (kGU) tmem_ld16(trow + kNpBN + c0, v1);
@@ -341,7 +363,7 @@ __global__ void __launch_bounds__(kNpThreads, 1)
             if (kGU) {
               const float g = __fmul_rn(__uint_as_float(v0[c]), gs);
               const float u = __fmul_rn(__uint_as_float(v1[c]), gs);
-              a.h_out[(size_t)p * a.ld_out + wrow] = g / (1.0f + expf(-g)) * u;
+              a.h_out[(size_t)p * a.ld_out + wrow] = __fdividef(g, 1.0f + __expf(-g)) * u;
             } else {
               a.y_out[(size_t)p * a.ld_out + wrow] =
                   f32_to_bf16_bits(__fmul_rn(__uint_as_float(v0[c]), gs));
@@ -350,7 +372,7 @@ __global__ void __launch_bounds__(kNpThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(tmem_empty);
+      mbar_arrive(&tmem_empty[ab]);
     }
   }
   tc_fence_before();
@@ -401,16 +423,16 @@ static bool make_weight_maps(CUtensorMap *codes, CUtensorMap *scales, const void
          encode(scales, base + (size_t)8 * K, 2, sd, ss, sbx, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-// Activation maps: codes [rows][K/2] as 128 rows x 128 bytes with the
-// 128-byte swizzle; scales [rows][K/16] as 128 rows x 16 bytes.
+// Activation maps: codes [rows][K/2] as boxes of 32 rows x 128 bytes with
+// the 128-byte swizzle; scales [rows][K/16] as 32 rows x 16 bytes.
 static bool make_act_maps(CUtensorMap *codes, CUtensorMap *scales, const uint8_t *c,
                           const uint8_t *sf, int rows, int K) {
   cuuint64_t cd[2] = {(cuuint64_t)K / 2, (cuuint64_t)rows};
   cuuint64_t cs[1] = {(cuuint64_t)K / 2};
-  cuuint32_t cb[2] = {128, kNpBN};
+  cuuint32_t cb[2] = {128, kNpBoxRows};
   cuuint64_t sd[2] = {(cuuint64_t)K / 16, (cuuint64_t)rows};
   cuuint64_t ss[1] = {(cuuint64_t)K / 16};
-  cuuint32_t sbx[2] = {16, kNpBN};
+  cuuint32_t sbx[2] = {16, kNpBoxRows};
   return encode(codes, c, 2, cd, cs, cb, CU_TENSOR_MAP_SWIZZLE_128B) &&
          encode(scales, sf, 2, sd, ss, sbx, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
