@@ -490,11 +490,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
   if (tid < 32) emask[tid] = 0u;
   for (int i = tid; i < kDecMaxRows * 8; i += kDecThreads) rmask[i] = 0u;
   pdl_wait();  // inputs of this call may come from the previous kernel
-  if (tid == 0) {
-    unsigned int ep = a.ctrl[0] + 1u;  // this call's epoch; never 0 (zeroed words never match)
-    misc[2] = (int)(ep == 0u ? 1u : ep);
+  // The loads this setup needs go out together: x straight into shared
+  // memory (int4; asynchronous), the call counter, the router logits.
+  if (!kFp4) {
+    for (int v = tid; v < T * H / 8; v += kDecThreads) cp_async_16(x_s + 8 * v, a.x + 8 * v);
+    cp_async_commit();
   }
-  __syncthreads();
+  const unsigned int ctrl0 = tid == kDecThreads - 1 ? a.ctrl[0] : 0u;
+  __syncthreads();  // barrier initialisation and table clears are visible
 
   auto item_of = [&](int item, int nA, bool *isA, int *slot, int *sub) {
     if (item < nA) {
@@ -543,6 +546,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
     ridx[tid] = e;
     atomicOr(&emask[e >> 5], 1u << (e & 31));
   }
+  if (tid == kDecThreads - 1) {
+    const unsigned int ep = ctrl0 + 1u;  // this call's epoch; never 0 (zeroed words never match)
+    misc[2] = (int)(ep == 0u ? 1u : ep);
+  }
   __syncthreads();
   if (warp == 0) {
     uint32_t m = emask[lane];
@@ -564,11 +571,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
       const uint64_t pol = policy_evict_first();
       for (int q = 0; q < min(myCount, a.nstages); ++q) issue(blockIdx.x + q * G, nA, q, pol);
     }
-  } else if (!kFp4) {
-    const int vec = T * H / 8;  // activations into shared memory
-    for (int v = tid - 32; v < vec; v += kDecThreads - 32)
-      reinterpret_cast<uint4 *>(x_s)[v] = reinterpret_cast<const uint4 *>(a.x)[v];
   }
+  if (!kFp4) cp_async_wait_all();  // this thread's x copies
   __syncthreads();
   pdl_launch_dependents();
   // rows of each slot as a bit set; activation group sums

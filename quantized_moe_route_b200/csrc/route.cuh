@@ -15,62 +15,65 @@ constexpr int kRouteMaxPerLane = 32;  // E <= 1024
 
 // One warp, one token.  Lane l owns experts l, l + 32, l + 64, ...
 // (coalesced loads).  Each of the k rounds takes the warp-wide maximum
-// (value, then lowest id) of the not-yet-taken experts; only the winning lane
+// (value, then lowest id) of the not-yet-taken experts with two single-
+// instruction warp reductions (max of an order-preserving integer key of the
+// logit, then min of the ids holding that key); only the winning lane
 // rescans its own entries.  Weights are exp(l_j - max) / sum over the
 // selected of exp(l_j' - max): the renormalised softmax restricted to the
 // selection.  Lane j < k returns the j-th selection in *idx_j, *w_j.
+
+// Unsigned key ordered like the float (both zeros map to one key); 0 is
+// below every finite logit and marks "nothing left".
+__device__ __forceinline__ uint32_t route_key(float f) {
+  const uint32_t b = f == 0.f ? 0u : __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float route_key_value(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
 template <int PER>
 __device__ __forceinline__ void route_token_warp(const float *__restrict__ l, int E, int k,
                                                  int *idx_j, float *w_j) {
   const int lane = threadIdx.x & 31;
-  float v[PER];
+  uint32_t key[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int e = lane + 32 * i;
-    v[i] = e < E ? l[e] : -INFINITY;
+    key[i] = e < E ? route_key(l[e]) : 0u;
   }
   uint32_t taken = 0;  // bit i: expert lane + 32 i already selected
   // local best of the untaken entries: entries visited in increasing id and
-  // strict > keeps the lowest id among equals; -1 = nothing left
-  auto local_best = [&](float &bv, int &bi) {
-    bv = -INFINITY;
-    bi = -1;
+  // strict > keeps the lowest id among equal keys; key 0 = nothing left
+  auto local_best = [&](uint32_t &bk, int &bi) {
+    bk = 0u;
+    bi = 0;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !((taken >> i) & 1u) && (bi < 0 || v[i] > bv)) {
-        bv = v[i];
-        bi = e;
+      if (!((taken >> i) & 1u) && key[i] > bk) {
+        bk = key[i];
+        bi = lane + 32 * i;
       }
     }
   };
-  float bv;
+  uint32_t bk;
   int bi;
-  local_best(bv, bi);
+  local_best(bk, bi);
   float top = 0.f, denom = 0.f, my_w = 0.f;
   int my_idx = 0;
   for (int j = 0; j < k; ++j) {
-    // warp arg-max: larger value, then lower id; exhausted lanes carry INT_MAX
-    float rv = bv;
-    int ri = bi < 0 ? 0x7fffffff : bi;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, rv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, ri, o);
-      if (oi != 0x7fffffff && (ri == 0x7fffffff || ov > rv || (ov == rv && oi < ri))) {
-        rv = ov;
-        ri = oi;
-      }
-    }
-    if ((ri & 31) == lane) {
+    const uint32_t kmax = __reduce_max_sync(0xffffffffu, bk);
+    const uint32_t ri = __reduce_min_sync(0xffffffffu, (bk == kmax && bk != 0u) ? (uint32_t)bi : 0xffffffffu);
+    if ((int)(ri & 31u) == lane) {
       taken |= 1u << (ri >> 5);
-      local_best(bv, bi);
+      local_best(bk, bi);
     }
+    const float rv = route_key_value(kmax);
     if (j == 0) top = rv;
     const float ex = expf(rv - top);
     denom += ex;
     if (lane == j) {
-      my_idx = ri;
+      my_idx = (int)ri;
       my_w = ex;
     }
   }
