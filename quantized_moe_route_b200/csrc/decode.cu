@@ -186,10 +186,19 @@ __device__ __forceinline__ void fold(float acc[4], const float d[4], const float
   acc[3] = __fmaf_rn(A.c1, xs[3], __fmaf_rn(A.s1, d[3], acc[3]));
 }
 
+// Shared-memory order of the 64 activations of a group (int4 path): channel
+// k = 16 j + 8 hi + 2 t + lo sits at 16 t + 4 j + 2 hi + lo, so lane t's B
+// fragments of the group's four k16 steps are 16 consecutive values (two
+// 16-byte loads).
+__host__ __device__ constexpr int w4_kpos(int k) {
+  return 16 * ((k & 7) >> 1) + 4 * (k >> 4) + 2 * ((k >> 3) & 1) + (k & 1);
+}
+
 // One warp: NG 64-channel groups and NMAT matrices (gate and up, or down) of
 // 16 rows each, against up to 16 activation rows held in shared memory as
-// bf16 [n][ld], whose per-group sums are gsum[n][g].  The A fragments of a
-// group are built once and reused for both token blocks.
+// bf16 [n][ld] in w4_kpos order, whose per-group sums are gsum[n][g].  The A
+// fragments of a group are built once and reused for both token blocks.
+// Columns n >= ntok read row tok_of[0]; their results are never used.
 template <int NB, int NMAT, int NG>
 __device__ __forceinline__ void group_mma(const uint8_t *const (&blk)[NG][NMAT],
                                           const uint16_t *act, int ld, const int (&gidx)[NG],
@@ -212,20 +221,16 @@ __device__ __forceinline__ void group_mma(const uint8_t *const (&blk)[NG][NMAT],
 #pragma unroll
   for (int nb = 0; nb < NB; ++nb) {
     const int n = nb * 8 + gi;  // this lane's B column (token slot)
-    const bool live = n < ntok;
-    const uint16_t *arow = act + (size_t)(live ? tok_of[n] : 0) * ld + 2 * t4;
+    const uint16_t *arow = act + (size_t)tok_of[n < ntok ? n : 0] * ld + 16 * t4;
     const int na = nb * 8 + 2 * t4, nb1 = na + 1;  // this lane's D columns
+    const float *ga = gsum + (size_t)tok_of[na < ntok ? na : 0] * gsum_ld;
+    const float *gb = gsum + (size_t)tok_of[nb1 < ntok ? nb1 : 0] * gsum_ld;
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
-      uint32_t b[4][2];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint16_t *p = arow + 64 * gidx[g] + 16 * j;
-        b[j][0] = live ? *reinterpret_cast<const uint32_t *>(p) : 0u;
-        b[j][1] = live ? *reinterpret_cast<const uint32_t *>(p + 8) : 0u;
-      }
-      const float xa = na < ntok ? gsum[(size_t)tok_of[na] * gsum_ld + gidx[g]] : 0.f;
-      const float xb = nb1 < ntok ? gsum[(size_t)tok_of[nb1] * gsum_ld + gidx[g]] : 0.f;
+      const uint4 q0 = *reinterpret_cast<const uint4 *>(arow + 64 * gidx[g]);
+      const uint4 q1 = *reinterpret_cast<const uint4 *>(arow + 64 * gidx[g] + 8);
+      const uint32_t b[4][2] = {{q0.x, q0.y}, {q0.z, q0.w}, {q1.x, q1.y}, {q1.z, q1.w}};
+      const float xa = ga[gidx[g]], xb = gb[gidx[g]];
       const float xs[4] = {xa, xb, xa, xb};
 #pragma unroll
       for (int m = 0; m < NMAT; ++m) {
@@ -281,19 +286,32 @@ __device__ __forceinline__ void frag_to_red(float *red, const float acc[2][4], i
 
 // Sums of 64 consecutive bf16 values: rows [nrows][ld] -> out[n][g] for the
 // first ngroups groups; eight threads per sum, one 16-byte vector each.
-// `t` / `nthreads`: this thread's index among the participating threads.
-__device__ __forceinline__ void group_sums(const uint16_t *rows, int nrows, int ld, int ngroups,
+// `t` / `nthreads`: this thread's index among the participating threads
+// (a multiple of 32).  With kReorder, the group is also rewritten in place in
+// w4_kpos order (the eight threads of a group share a warp).
+template <bool kReorder = false>
+__device__ __forceinline__ void group_sums(uint16_t *rows, int nrows, int ld, int ngroups,
                                            float *out, int t, int nthreads) {
   const int tasks = nrows * ngroups * 8;
   for (int v = t; v < ((tasks + nthreads - 1) / nthreads) * nthreads; v += nthreads) {
     float s = 0.f;
     const int task = v >> 3, part = v & 7;
+    uint16_t *grp = rows;
+    uint32_t u[4] = {0u, 0u, 0u, 0u};
     if (v < tasks) {
       const int n = task / ngroups, g = task % ngroups;
-      const uint4 q = *reinterpret_cast<const uint4 *>(rows + (size_t)n * ld + 64 * g + 8 * part);
-      const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+      grp = rows + (size_t)n * ld + 64 * g;
+      const uint4 q = *reinterpret_cast<const uint4 *>(grp + 8 * part);
+      u[0] = q.x, u[1] = q.y, u[2] = q.z, u[3] = q.w;
 #pragma unroll
       for (int i = 0; i < 4; ++i) s += __uint_as_float(u[i] << 16) + __uint_as_float(u[i] & 0xFFFF0000u);
+    }
+    if (kReorder) {
+      __syncwarp();  // the whole group is in registers before any of it moves
+      if (v < tasks)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)  // channels 8 part + 2 i, + 1
+          *reinterpret_cast<uint32_t *>(grp + w4_kpos(8 * part + 2 * i)) = u[i];
     }
     s += __shfl_xor_sync(0xffffffffu, s, 1);
     s += __shfl_xor_sync(0xffffffffu, s, 2);
@@ -583,7 +601,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
     atomicOr(&rmask[my_slot * 8 + (tid >> 5)], 1u << (tid & 31));
   }
   if (!kFp4) {
-    group_sums(x_s, T, H, Gh, xsum_s, tid, kDecThreads);
+    group_sums<true>(x_s, T, H, Gh, xsum_s, tid, kDecThreads);
   } else if (warp < T) {  // warp t quantises token t: x_s = E2M1 * S_b (f16), xsum_s[t] = G
     const uint16_t *xr = a.x + (size_t)warp * H;
     const float G = nvfp4_row_f16(
@@ -677,7 +695,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
           const unsigned long long w =
               ld_relaxed_u64(a.hbuf + (size_t)slot_rows[r0 + n] * F + f);
           if ((unsigned int)(w & 0xFFFFFFFFull) != epoch) mine = false;
-          else if (!kFp4) h_s[(size_t)n * F + f] = (uint16_t)(w >> 32);
+          else if (!kFp4) h_s[(size_t)n * F + (f & ~63) + w4_kpos(f & 63)] = (uint16_t)(w >> 32);
         }
         ready = !team_or(bar_id, !mine);
         if (ready || ++spins > (1u << 20)) break;
