@@ -812,19 +812,28 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
           const int t = slot_rows[r0 + n] / k;
           if (maxslot[t] != slot) continue;
           float acc = 0.f;
-          for (int j = 0; j < k && ok; ++j) {
-            const unsigned long long *wp = a.ybuf + (size_t)(t * k + j) * H + kDecOutRows * sub + c;
-            unsigned long long wv = ld_relaxed_u64(wp);
-            uint32_t spins = 0;
-            while ((unsigned int)(wv & 0xFFFFFFFFull) != epoch) {
-              if (++spins > (1u << 22)) {
-                ok = false;
-                break;
+          const unsigned long long *wp0 = a.ybuf + (size_t)t * k * H + kDecOutRows * sub + c;
+          for (int j0 = 0; j0 < k && ok; j0 += 8) {
+            // the (up to) eight rows' words are requested together, then
+            // summed in j order; a word of an earlier call is polled again
+            unsigned long long wv[8];
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj)
+              wv[jj] = j0 + jj < k ? ld_relaxed_u64(wp0 + (size_t)(j0 + jj) * H) : 0ull;
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+              if (j0 + jj >= k || !ok) break;
+              uint32_t spins = 0;
+              while ((unsigned int)(wv[jj] & 0xFFFFFFFFull) != epoch) {
+                if (++spins > (1u << 22)) {
+                  ok = false;
+                  break;
+                }
+                __nanosleep(64);
+                wv[jj] = ld_relaxed_u64(wp0 + (size_t)(j0 + jj) * H);
               }
-              __nanosleep(64);
-              wv = ld_relaxed_u64(wp);
+              acc = __fadd_rn(acc, __fmul_rn(rw[t * k + j0 + jj], __uint_as_float((uint32_t)(wv[jj] >> 32))));
             }
-            acc = __fadd_rn(acc, __fmul_rn(rw[t * k + j], __uint_as_float((uint32_t)(wv >> 32))));
           }
           a.y[(size_t)t * H + kDecOutRows * sub + c] = f32_to_bf16_bits(acc);
         }
