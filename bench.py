@@ -42,6 +42,10 @@ NV_WORKLOAD = ("NVFP4 single-layer decode: 256 experts, top-8, hidden 2048, expe
                "E2M1 weights with E4M3 scales per 16 channels and fp32 per-matrix globals, x and h quantised "
                "per token/row in the kernel; steps rotate over 40 resident NVFP4 layers (18.1 GB)")
 DTYPE_W4 = "int4 weights (f16 scale/min), bf16 activations, fp32 accumulate"
+# dram__bytes_read.sum + dram__bytes_write.sum of one decode launch at 1 token,
+# from the ncu captures summarised in profiles/ (taken on the current kernels;
+# set to None whenever the kernel changes)
+DECODE_TRAFFIC = {"w4": 14242560, "nvfp4": 14254336}
 DTYPE_NV = "nvfp4 weights and activations (e2m1 + e4m3/16 + fp32 global), fp32 accumulate"
 
 
@@ -367,7 +371,11 @@ def run_gpu(args, log):
                    "launch": f"one kernel per step (route + FFN + combine), CUDA graphs of "
                              f"{min(K, args.graph_steps)} steps, programmatic dependent launch"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak,
+                     "traffic": DECODE_TRAFFIC.get(fmt) if T == 1 else None,
+                     "traffic_source": ("ncu capture, one launch at 1 token: profiles/decode_kernel_"
+                                        + ("nvfp4_" if fmt == "nvfp4" else "") + "single_layer_T1.md")
+                     if T == 1 else "not captured at this batch size",
                      "kernel": f"moe::decode_kernel<{'nvfp4' if fmt == 'nvfp4' else 'int4'}, fused>",
                      "peak_kind": peak_kind, "alg_bytes_per_launch": alg_bytes,
                      "avg_launch_us": dur_ms * 1e3, "isolated_launch_us": isolated_ms * 1e3},
