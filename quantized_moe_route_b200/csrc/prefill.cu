@@ -296,26 +296,34 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           const uint2 cw = *reinterpret_cast<const uint2 *>(blk + 16 * lane + 8 * wh);
           const uint32_t sm0 = *reinterpret_cast<const uint32_t *>(blk + kBlkCodeBytes + 4 * gi);
           const uint32_t sm1 = *reinterpret_cast<const uint32_t *>(blk + kBlkCodeBytes + 4 * (gi + 8));
-          // fp32 q * s + m computed as (128 + q) * s + (m - 128 s): the code
-          // becomes the bf16 value 128 + q by OR-ing 0x4300, and a bf16 is the
-          // top half of an fp32; m - 128 s is formed once per row and group
-          float sc[2], of[2];
+          // fp32 q * s + m with one rounding, as the format defines it.  A
+          // nibble at bit p <= 16 of a word, OR-ed into the exponent pattern
+          // (150 - p) << 23, is the fp32 value 2^(23 - p) + q exactly, so one
+          // integer op per code (plus one shift per word for the nibbles at
+          // 20, 24, 28) and an exact subtraction give q in fp32.
+          float sc[2], mn[2];
           sc[0] = f16_bits_to_f32((uint16_t)(sm0 & 0xFFFFu));
           sc[1] = f16_bits_to_f32((uint16_t)(sm1 & 0xFFFFu));
-          of[0] = __fmaf_rn(-128.f, sc[0], f16_bits_to_f32((uint16_t)(sm0 >> 16)));
-          of[1] = __fmaf_rn(-128.f, sc[1], f16_bits_to_f32((uint16_t)(sm1 >> 16)));
+          mn[0] = f16_bits_to_f32((uint16_t)(sm0 >> 16));
+          mn[1] = f16_bits_to_f32((uint16_t)(sm1 >> 16));
           uint8_t *rowp[2] = {atile + ((rb + gi) >> 3) * 1024 + gi * 128,
                               atile + ((rb + gi + 8) >> 3) * 1024 + gi * 128};
           const uint32_t wx = (uint32_t)wh << 6;
 #pragma unroll
           for (int jj = 0; jj < 2; ++jj) {
             const uint32_t w = jj ? cw.y : cw.x;
+            const uint32_t w12 = w >> 12;  // nibbles 20, 24, 28 at 8, 12, 16
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {  // shift 4 i: hr = i & 1, hk = i >> 1
+            for (int i = 0; i < 4; ++i) {  // nibble 4 i (channel k) and 4 i + 16 (k + 1): hr = i & 1, hk = i >> 1
               const int hr = i & 1, hk = i >> 1;
-              const uint32_t v = ((w >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
-              const float lo = __fmaf_rn(__uint_as_float(v << 16), sc[hr], of[hr]);
-              const float hi = __fmaf_rn(__uint_as_float(v & 0xFFFF0000u), sc[hr], of[hr]);
+              const int p = 4 * i, ph = p + 16;  // ph: 16 from w, else from w12 at ph - 12
+              const float vlo = __uint_as_float((w & (0xFu << p)) | ((150u - p) << 23));
+              const float vhi = ph == 16 ? __uint_as_float((w & 0xF0000u) | (134u << 23))
+                                         : __uint_as_float((w12 & (0xFu << (ph - 12))) | ((150u - (ph - 12)) << 23));
+              const float qlo = __fsub_rn(vlo, (float)(1u << (23 - p)));
+              const float qhi = __fsub_rn(vhi, ph == 16 ? 128.0f : (float)(1u << (23 - (ph - 12))));
+              const float lo = __fmaf_rn(qlo, sc[hr], mn[hr]);
+              const float hi = __fmaf_rn(qhi, sc[hr], mn[hr]);
               *reinterpret_cast<__nv_bfloat162 *>(rowp[hr] + (koff[jj][hk] ^ wx)) = __floats2bfloat162_rn(lo, hi);
             }
           }
