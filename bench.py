@@ -130,13 +130,21 @@ def dist_setup():
 
 
 def dist_max(v: float) -> float:
+    """Max of a per-rank value over all ranks (the slowest rank's time)."""
     import torch
     import torch.distributed as dist
     if not dist.is_initialized():
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank: int, world: int, max_ms: float) -> float:
+    """Whole-job throughput of independent replicas: every rank's units over
+    the slowest rank's time (weak scaling; no data-path exchange)."""
+    return units_per_rank * world / (max_ms / 1e3)
 
 
 def dist_barrier():
@@ -309,7 +317,7 @@ def run_gpu(args, log):
         dist_barrier()
     ms = dist_max(e0.elapsed_time(e1))
     tokens = K * T * world
-    value = tokens / (ms / 1e3)
+    value = job_throughput(K * T, world, ms)
 
     # Each step is exactly one launch of the decode kernel, so the timed
     # region over K is that kernel's average launch duration (back to back,
@@ -459,7 +467,7 @@ def run_gpu_prefill(args, log):
         dist_barrier()
     ms = dist_max(e0.elapsed_time(e1))
     tokens = K * T * world
-    value = tokens / (ms / 1e3)
+    value = job_throughput(K * T, world, ms)
 
     # kernel-duration pass: events around the two grouped-GEMM launches
     P = min(K, 50)
@@ -602,7 +610,7 @@ def run_gpu_prefill_nvfp4(args, log):
         dist_barrier()
     ms = dist_max(e0.elapsed_time(e1))
     tokens = K * T * world
-    value = tokens / (ms / 1e3)
+    value = job_throughput(K * T, world, ms)
 
     # kernel-duration pass: events around the grouped FFN call (gate/up, h
     # quantisation, down: three launches)
