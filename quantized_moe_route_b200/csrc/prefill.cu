@@ -39,21 +39,25 @@ constexpr uint32_t kPfWaitLimit = 1u << 24;
 // MMA).
 template <bool kGU>
 struct PfCfg {
-  static constexpr int kMats = kGU ? 2 : 1;
+  // two 128-row MMA blocks per tile share each activation tile: gate and up
+  // of 128 features, or 256 consecutive outputs of the down matrix (which
+  // halves the down launch's re-reads of h)
+  static constexpr int kMats = 2;
   static constexpr uint32_t kRawBytes = kMats * 8 * kBlkBytes;              // 8 strips per matrix
   static constexpr uint32_t kRawStride = (kRawBytes + 127) / 128 * 128;
   static constexpr uint32_t kABytes = kMats * kPfBM * kPfBK * 2;            // bf16 tiles
   static constexpr uint32_t kBBytes = kPfBN * kPfBK * 2;                    // activation tile
-  static constexpr int kRawStages = kGU ? 6 : 10;
+  static constexpr int kRawStages = 6;
   static constexpr int kAStages = 2;
   static constexpr int kBStages = 3;
-  static constexpr uint32_t kTmemCols = kGU ? 2 * kPfBN : kPfBN;  // 512 or 256 (powers of two)
+  static constexpr uint32_t kTmemCols = kMats * kPfBN;  // 512: the two accumulators
   // layout: [A ring][B ring][raw ring], 1024-aligned tiles
   static constexpr uint32_t kAOff = 0;
   static constexpr uint32_t kBOff = kAOff + kAStages * kABytes;
   static constexpr uint32_t kRawOff = kBOff + kBStages * kBBytes;
   static constexpr uint32_t kTailOff = kRawOff + kRawStages * kRawStride;
   static constexpr uint32_t kSmemBytes = kTailOff + 1024 /*align slack*/ + 4096;
+  static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
 struct PrefillArgs {
@@ -63,7 +67,7 @@ struct PrefillArgs {
   uint16_t *out;           // gate/up: h [rows][F]; down: y_perm [rows][H]
   int *err;
   int E, K, rows;
-  int n_sub;               // weight tiles per row chunk: F/128 (gate/up) or H/128 (down)
+  int n_sub;               // weight tiles per row chunk: F/128 (gate/up) or H/256 (down)
   int ld_out;              // F (gate/up) or H (down)
   int F;                   // gate/up: features per matrix (strip index of the up half)
 };
@@ -186,7 +190,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             for (int i = 0; i < 8; ++i) {
               // gate/up: strip 2 r is gate, 2 r + 1 up, of 16-feature block r
               const int srow = ti.sub * 8 + i;
-              const int strip = kGU ? 2 * srow + m : srow;
+              const int strip = kGU ? 2 * srow + m : ti.sub * 16 + m * 8 + i;
               bulk_g2s(raw + (m * 8 + i) * kBlkBytes, wexp + ((size_t)strip * KB + kb) * kBlkBytes,
                        kBlkBytes, &raw_full[s]);
             }
@@ -343,24 +347,26 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         break;
       }
       tc_fence_after();
-      const int feat = ti.sub * kPfBM + quarter * 32 + lane;  // this thread's weight row
+      // this thread's weight row: gate/up feature, or the first block's
+      // output channel (the second block's is 128 further)
+      const int feat = ti.sub * (kGU ? kPfBM : 2 * kPfBM) + quarter * 32 + lane;
       const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16);
       for (int c0 = cgrp * 16; c0 < kPfBN; c0 += 64) {
         if (c0 >= ti.nvalid) break;  // uniform across the warp
         uint32_t v0[16], v1[16];
         tmem_ld16(trow + c0, v0);
-        if (kGU) tmem_ld16(trow + kPfBN + c0, v1);
+        tmem_ld16(trow + kPfBN + c0, v1);
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           if (c0 + c < ti.nvalid) {
-            float y;
+            uint16_t *orow = a.out + (size_t)(ti.row0 + c0 + c) * a.ld_out;
             if (kGU) {
               const float g = __uint_as_float(v0[c]), u = __uint_as_float(v1[c]);
-              y = g / (1.0f + __expf(-g)) * u;
+              orow[feat] = f32_to_bf16_bits(g / (1.0f + __expf(-g)) * u);
             } else {
-              y = __uint_as_float(v0[c]);
+              orow[feat] = f32_to_bf16_bits(__uint_as_float(v0[c]));
+              orow[feat + kPfBM] = f32_to_bf16_bits(__uint_as_float(v1[c]));
             }
-            a.out[(size_t)(ti.row0 + c0 + c) * a.ld_out + feat] = f32_to_bf16_bits(y);
           }
         }
       }
@@ -442,7 +448,7 @@ extern "C" MOE_API moe_status moe_ffn_grouped_prefill(const moe_w4_layer *layer,
   if (!layer || rows < 0) return MOE_ERR_INVALID_ARG;
   const int E = layer->E, H = layer->H, F = layer->F;
   if (E <= 0 || H <= 0 || F <= 0) return MOE_ERR_INVALID_ARG;
-  if (H % kPfBM || F % kPfBM || E > 960) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (H % (2 * kPfBM) || F % kPfBM || E > 960) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (rows == 0) return MOE_OK;
   if (!layer->gate_up || !layer->down || !x_perm || !offsets || !y_perm) return MOE_ERR_INVALID_ARG;
   if (!ws || ws_bytes < moe_prefill_workspace_bytes(rows, F)) return MOE_ERR_WORKSPACE;
@@ -478,7 +484,7 @@ extern "C" MOE_API moe_status moe_ffn_grouped_prefill(const moe_w4_layer *layer,
   dn.w_stride = w4_packed_bytes(H, F);
   dn.out = y_perm;
   dn.K = F;
-  dn.n_sub = H / kPfBM;
+  dn.n_sub = H / (2 * kPfBM);
   dn.ld_out = H;
   return prefill_launch<false>(dn, hmap, s);
 }

@@ -65,7 +65,7 @@ def test_no_op_calls_leave_outputs_untouched():
                                   moe._p(ws), ws.numel(), None)
     assert st == moe.MOE_OK
     assert L.moe_route(moe._p(lg), 0, 8, 2, None, None, None) == moe.MOE_OK
-    pf = moe.moe_w4_layer(8, 128, 128, 16, 16)  # a shape the prefill tiles (F % 128 == 0)
+    pf = moe.moe_w4_layer(8, 256, 128, 16, 16)  # a shape the prefill tiles (H % 256, F % 128)
     assert L.moe_ffn_grouped_prefill(ctypes.byref(pf), None, None, 0, None, None, 0, None) == moe.MOE_OK
     assert L.moe_unpermute_combine(None, 0, None, None, 0, 2, 128, None, None) == moe.MOE_OK
     torch.cuda.synchronize()
