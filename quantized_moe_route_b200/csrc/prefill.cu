@@ -70,6 +70,7 @@ struct PrefillArgs {
   int n_sub;               // weight tiles per row chunk: F/128 (gate/up) or H/256 (down)
   int ld_out;              // F (gate/up) or H (down)
   int F;                   // gate/up: features per matrix (strip index of the up half)
+  int spe;                 // strip pairs (gate/up) or strips (down) per expert
 };
 
 // ---------------------------------------------------------------- tiles
@@ -97,7 +98,8 @@ __device__ __forceinline__ TileInfo tile_info(int t, int n_sub, const int *chunk
 
 template <bool kGU>
 __global__ void __launch_bounds__(kPfThreads, 1)
-    prefill_kernel(PrefillArgs a, const __grid_constant__ CUtensorMap act_map) {
+    prefill_kernel(PrefillArgs a, const __grid_constant__ CUtensorMap act_map,
+                   const __grid_constant__ CUtensorMap w_map) {
   using C = PfCfg<kGU>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -176,7 +178,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       uint32_t it = 0;
       for (int t = blockIdx.x; t < ntiles && !*abort_s; t += G) {
         const TileInfo ti = tile_info(t, a.n_sub, chunk_start, a.E, a.offsets);
-        const uint8_t *wexp = a.w + (size_t)ti.e * a.w_stride;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % C::kRawStages;
           const uint32_t ph = (it / C::kRawStages) & 1u;
@@ -186,14 +187,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
           uint8_t *raw = smem + C::kRawOff + s * C::kRawStride;
           mbar_arrive_expect_tx(&raw_full[s], C::kRawBytes);
-          for (int m = 0; m < C::kMats; ++m)
-            for (int i = 0; i < 8; ++i) {
-              // gate/up: strip 2 r is gate, 2 r + 1 up, of 16-feature block r
-              const int srow = ti.sub * 8 + i;
-              const int strip = kGU ? 2 * srow + m : ti.sub * 16 + m * 8 + i;
-              bulk_g2s(raw + (m * 8 + i) * kBlkBytes, wexp + ((size_t)strip * KB + kb) * kBlkBytes,
-                       kBlkBytes, &raw_full[s]);
-            }
+          // one box per matrix: block kb of 8 strips.  gate/up: strip 2 r is
+          // gate, 2 r + 1 up, of 16-feature block r (coordinates: strip pair,
+          // gate/up); down: strips 16 sub + 8 m + i
+          for (int m = 0; m < C::kMats; ++m) {
+            if (kGU)
+              tma_load_4d(raw + m * 8 * kBlkBytes, &w_map, 0, kb, m, ti.e * a.spe + ti.sub * 8, &raw_full[s]);
+            else
+              tma_load_3d(raw + m * 8 * kBlkBytes, &w_map, 0, kb, ti.e * a.spe + ti.sub * 16 + m * 8,
+                          &raw_full[s]);
+          }
         }
       }
     }
@@ -397,8 +400,34 @@ static bool make_act_map(CUtensorMap *map, const void *base, int rows, int cols)
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Packed int4 weights of all E experts as 32-bit words: one 576-byte block
+// (144 words) x K/64 blocks per strip x strips.  gate/up: strips as
+// {gate, up} x strip pairs, box = block kb of 8 gate (or up) strips; down:
+// box = block kb of 8 consecutive strips.
+static bool make_w4_map(CUtensorMap *map, const void *base, int E, int N, int K, bool gate_up) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t KB = (cuuint64_t)K / kGroup, strip = KB * kBlkBytes;
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  if (gate_up) {
+    cuuint64_t dims[4] = {kBlkBytes / 4, KB, 2, (cuuint64_t)E * (N / 32)};
+    cuuint64_t strides[3] = {kBlkBytes, strip, 2 * strip};
+    cuuint32_t box[4] = {kBlkBytes / 4, 1, 1, 8};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  }
+  cuuint64_t dims[3] = {kBlkBytes / 4, KB, (cuuint64_t)E * (N / 16)};
+  cuuint64_t strides[2] = {kBlkBytes, strip};
+  cuuint32_t box[3] = {kBlkBytes / 4, 1, 8};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <bool kGU>
-static moe_status prefill_launch(const PrefillArgs &a, const CUtensorMap &map, cudaStream_t stream) {
+static moe_status prefill_launch(const PrefillArgs &a, const CUtensorMap &map, const CUtensorMap &wmap,
+                                 cudaStream_t stream) {
   using C = PfCfg<kGU>;
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
@@ -423,7 +452,7 @@ static moe_status prefill_launch(const PrefillArgs &a, const CUtensorMap &map, c
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_kernel<kGU>, a, map);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_kernel<kGU>, a, map, wmap);
   if (e != cudaSuccess) {
     set_cuda_error(e);
     return MOE_ERR_CUDA;
@@ -459,8 +488,10 @@ extern "C" MOE_API moe_status moe_ffn_grouped_prefill(const moe_w4_layer *layer,
   int *err = device_error_word();
   if (!err) return MOE_ERR_CUDA;
   uint16_t *h = static_cast<uint16_t *>(ws);
-  CUtensorMap xmap, hmap;
-  if (!make_act_map(&xmap, x_perm, rows, H) || !make_act_map(&hmap, h, rows, F)) {
+  CUtensorMap xmap, hmap, gumap, dnmap;
+  if (!make_act_map(&xmap, x_perm, rows, H) || !make_act_map(&hmap, h, rows, F) ||
+      !make_w4_map(&gumap, layer->gate_up, E, 2 * F, H, true) ||
+      !make_w4_map(&dnmap, layer->down, E, H, F, false)) {
     set_cuda_error(cudaErrorInvalidValue);
     return MOE_ERR_CUDA;
   }
@@ -477,7 +508,8 @@ extern "C" MOE_API moe_status moe_ffn_grouped_prefill(const moe_w4_layer *layer,
   gu.n_sub = F / kPfBM;
   gu.ld_out = F;
   gu.F = F;
-  moe_status st = prefill_launch<true>(gu, xmap, s);
+  gu.spe = F / 16;  // strip pairs per expert
+  moe_status st = prefill_launch<true>(gu, xmap, gumap, s);
   if (st != MOE_OK) return st;
   PrefillArgs dn = gu;
   dn.w = static_cast<const uint8_t *>(layer->down);
@@ -486,5 +518,6 @@ extern "C" MOE_API moe_status moe_ffn_grouped_prefill(const moe_w4_layer *layer,
   dn.K = F;
   dn.n_sub = H / (2 * kPfBM);
   dn.ld_out = H;
-  return prefill_launch<false>(dn, hmap, s);
+  dn.spe = H / 16;  // strips per expert
+  return prefill_launch<false>(dn, hmap, dnmap, s);
 }
