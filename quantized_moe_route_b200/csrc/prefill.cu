@@ -47,15 +47,17 @@ struct PfCfg {
   static constexpr uint32_t kRawStride = (kRawBytes + 127) / 128 * 128;
   static constexpr uint32_t kABytes = kMats * kPfBM * kPfBK * 2;            // bf16 tiles
   static constexpr uint32_t kBBytes = kPfBN * kPfBK * 2;                    // activation tile
-  static constexpr int kRawStages = 6;
+  static constexpr int kRawStages = 4;
   static constexpr int kAStages = 2;
   static constexpr int kBStages = 3;
   static constexpr uint32_t kTmemCols = kMats * kPfBN;  // 512: the two accumulators
-  // layout: [A ring][B ring][raw ring], 1024-aligned tiles
+  // layout: [A ring][B ring][raw ring][epilogue staging], 1024-aligned tiles
   static constexpr uint32_t kAOff = 0;
   static constexpr uint32_t kBOff = kAOff + kAStages * kABytes;
   static constexpr uint32_t kRawOff = kBOff + kBStages * kBBytes;
-  static constexpr uint32_t kTailOff = kRawOff + kRawStages * kRawStride;
+  static constexpr uint32_t kEpiOff = kRawOff + kRawStages * kRawStride;
+  static constexpr uint32_t kEpiBytes = kPfDqWarps * 16 * 32 * 2;  // per warp: 16 rows x 32 outputs, bf16
+  static constexpr uint32_t kTailOff = kEpiOff + kEpiBytes;
   static constexpr uint32_t kSmemBytes = kTailOff + 1024 /*align slack*/ + 4096;
   static_assert(kSmemBytes <= 232448, "shared memory");
 };
@@ -350,27 +352,40 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         break;
       }
       tc_fence_after();
-      // this thread's weight row: gate/up feature, or the first block's
-      // output channel (the second block's is 128 further)
-      const int feat = ti.sub * (kGU ? kPfBM : 2 * kPfBM) + quarter * 32 + lane;
       const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16);
+      // each warp turns its 32 outputs x 16 rows around in shared memory and
+      // writes them as 16-byte vectors (row c: 64 bytes from 4 lanes)
+      uint16_t *stage = reinterpret_cast<uint16_t *>(smem + C::kEpiOff) + dw * 16 * 32;
+      const int fbase = ti.sub * (kGU ? kPfBM : 2 * kPfBM) + quarter * 32;  // first output of this warp
       for (int c0 = cgrp * 16; c0 < kPfBN; c0 += 64) {
         if (c0 >= ti.nvalid) break;  // uniform across the warp
         uint32_t v0[16], v1[16];
         tmem_ld16(trow + c0, v0);
         tmem_ld16(trow + kPfBN + c0, v1);
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          if (c0 + c < ti.nvalid) {
-            uint16_t *orow = a.out + (size_t)(ti.row0 + c0 + c) * a.ld_out;
+        for (int blk = 0; blk < (kGU ? 1 : 2); ++blk) {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            float y;
             if (kGU) {
               const float g = __uint_as_float(v0[c]), u = __uint_as_float(v1[c]);
-              orow[feat] = f32_to_bf16_bits(g / (1.0f + __expf(-g)) * u);
+              y = g / (1.0f + __expf(-g)) * u;
             } else {
-              orow[feat] = f32_to_bf16_bits(__uint_as_float(v0[c]));
-              orow[feat + kPfBM] = f32_to_bf16_bits(__uint_as_float(v1[c]));
+              y = __uint_as_float(blk ? v1[c] : v0[c]);
+            }
+            stage[c * 32 + lane] = f32_to_bf16_bits(y);
+          }
+          __syncwarp();
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const int q = lane + 32 * r, c = q >> 2, part = q & 3;
+            if (c0 + c < ti.nvalid) {
+              const uint4 v = *reinterpret_cast<const uint4 *>(stage + c * 32 + 8 * part);
+              *reinterpret_cast<uint4 *>(a.out + (size_t)(ti.row0 + c0 + c) * a.ld_out + fbase +
+                                         blk * kPfBM + 8 * part) = v;
             }
           }
+          __syncwarp();
         }
       }
       tc_fence_before();
