@@ -45,7 +45,7 @@ DTYPE_W4 = "int4 weights (f16 scale/min), bf16 activations, fp32 accumulate"
 # dram__bytes_read.sum + dram__bytes_write.sum of one decode launch at 1 token,
 # from the ncu captures summarised in profiles/ (taken on the current kernels;
 # set to None whenever the kernel changes)
-DECODE_TRAFFIC = {"w4": 14242560, "nvfp4": 14254336}
+DECODE_TRAFFIC = {"w4": 14242560, "nvfp4": None}
 DTYPE_NV = "nvfp4 weights and activations (e2m1 + e4m3/16 + fp32 global), fp32 accumulate"
 
 

@@ -110,8 +110,10 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int fmt, int T, int H, 
   L.x = take((uint32_t)T * H * 2, 16);
   // int4: 64-channel group sums of x and of each team's h;
   // NVFP4: the row globals of x and of each team's h
-  L.xsum = take(fmt == kFmtW4 ? (uint32_t)T * (H / 64) * 4 : (uint32_t)T * 4, 16);
-  L.hsum = take(fmt == kFmtW4 ? 2u * T * (F / 64) * 4 : 2u * T * 4, 16);
+  // NVFP4: the row globals of x and of each team's h, each followed by the
+  // rows' maxima (as bits)
+  L.xsum = take(fmt == kFmtW4 ? (uint32_t)T * (H / 64) * 4 : 2u * T * 4, 16);
+  L.hsum = take(fmt == kFmtW4 ? 2u * T * (F / 64) * 4 : 2u * 2u * T * 4, 16);
   L.bars = take((uint32_t)nstages * 8, 8);
   L.meta = take(3600 * 4, 16);  // routing tables + 256 x 8 row-set words
   L.total = o;
@@ -403,6 +405,60 @@ __device__ __forceinline__ float nvfp4_row_f16(Load load, int nb, uint16_t *out)
   return G;
 }
 
+// Cooperative form of nvfp4_row_f16 for values already in registers: the
+// participating threads (index t of nthreads, a multiple of 32) hold channel
+// pairs P = t + nthreads * i (i < MAXP) of `rows` rows of K channels, pair P
+// being row P / (K/2), channels 2 (P % (K/2)) and + 1, in hv[i].  A 16-value
+// block is 8 consecutive lanes, a warp's 32 pairs lie in one row.  rowmax
+// [rows] (shared, zeroed by the caller before the last barrier) collects
+// the row maxima; between the two halves the caller's barrier `sync` runs.
+// Same fp32 decisions as nvfp4_row_f16.
+template <int MAXP, class Sync>
+__device__ __forceinline__ void nvfp4_pairs_f16(const float2 (&hv)[MAXP], int rows, int K, int t,
+                                                int nthreads, unsigned int *rowmax, float *Gout,
+                                                uint16_t *out, Sync sync) {
+  const int lane = threadIdx.x & 31, half = K / 2, total = rows * half;
+  float bmax[MAXP];
+#pragma unroll
+  for (int i = 0; i < MAXP; ++i) {
+    const int P = t + nthreads * i;
+    float m = P < total ? fmaxf(fabsf(hv[i].x), fabsf(hv[i].y)) : 0.f;
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+    bmax[i] = m;
+    float r = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+    r = fmaxf(r, __shfl_xor_sync(0xffffffffu, r, 16));
+    if (lane == 0 && P < total) atomicMax(&rowmax[P / half], __float_as_uint(r));
+  }
+  sync();
+#pragma unroll
+  for (int i = 0; i < MAXP; ++i) {
+    const int P = t + nthreads * i;
+    if (P >= total) continue;
+    const int n = P / half, c2 = 2 * (P % half);  // first channel of the pair
+    const float amax = __uint_as_float(rowmax[n]);
+    const float G = amax == 0.f ? 1.0f : __fdiv_rn(amax, 2688.0f);
+    if (c2 == 0) Gout[n] = G;
+    const __nv_fp8_storage_t s8 = __nv_cvt_float_to_fp8(__fdiv_rn(bmax[i], __fmul_rn(6.0f, G)),
+                                                        __NV_SATFINITE, __NV_E4M3);
+    const float sb = __half2float(__half(__nv_cvt_fp8_to_halfraw(s8, __NV_E4M3)));
+    const float scale = __fmul_rn(sb, G);
+    const float v2[2] = {hv[i].x, hv[i].y};
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const __nv_fp4_storage_t c = __nv_cvt_float_to_fp4(__fdiv_rn(v2[j], scale), __NV_E2M1,
+                                                         cudaRoundNearest);
+      const float e = __half2float(__half(__nv_cvt_fp4_to_halfraw(c, __NV_E2M1)));
+      const float q = sb == 0.f ? 0.f : __fmul_rn(e, sb);
+      // tensor-core k order inside the 16-channel block (inverse of nv_perm)
+      const int ch = (c2 + j) & 15;
+      const int kap = ((ch & 1) << 3) | (((ch >> 3) & 1) << 2) | (((ch >> 1) & 1) << 1) | ((ch >> 2) & 1);
+      out[(size_t)n * K + ((c2 + j) & ~15) + kap] = __half_as_ushort(__float2half_rn(q));
+    }
+  }
+}
+
 // One warp, one 64-channel chunk g of NMAT NVFP4 strips (K channels each)
 // against up to 16 activation rows act[n][ld] (f16 in tensor-core k order):
 // acc += S_b * (sum over the block of code * 2^-14 * activation), block by
@@ -505,6 +561,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
     fence_mbar_init();
   }
   if (tid < kDecMaxTok) ident[tid] = tid;
+  if (kFp4 && tid < T) reinterpret_cast<unsigned int *>(xsum_s)[T + tid] = 0u;  // x row maxima
   if (tid < 32) emask[tid] = 0u;
   for (int i = tid; i < kDecMaxRows * 8; i += kDecThreads) rmask[i] = 0u;
   pdl_wait();  // inputs of this call may come from the previous kernel
@@ -602,6 +659,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
   }
   if (!kFp4) {
     group_sums<true>(x_s, T, H, Gh, xsum_s, tid, kDecThreads);
+  } else if (T * H / 2 <= 8 * kDecThreads) {  // all warps: channel pairs in registers
+    float2 hv[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int P = tid + kDecThreads * i;
+      hv[i] = make_float2(0.f, 0.f);
+      if (P < T * H / 2) {
+        const uint32_t u = reinterpret_cast<const uint32_t *>(a.x)[P];  // channels 2P, 2P + 1 of x
+        hv[i] = make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+      }
+    }
+    nvfp4_pairs_f16<8>(hv, T, H, tid, kDecThreads, reinterpret_cast<unsigned int *>(xsum_s) + T, xsum_s, x_s,
+                       [] { __syncthreads(); });
   } else if (warp < T) {  // warp t quantises token t: x_s = E2M1 * S_b (f16), xsum_s[t] = G
     const uint16_t *xr = a.x + (size_t)warp * H;
     const float G = nvfp4_row_f16(
@@ -665,7 +735,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
   const int myCount = (int)blockIdx.x < nItems ? (nItems - 1 - (int)blockIdx.x) / G + 1 : 0;
   const uint64_t pol = policy_evict_first();
   int *tok_list = tok_lists[team];
-  float *hsum_s = reinterpret_cast<float *>(smem + L.hsum) + (size_t)team * T * (kFp4 ? 1 : Gf);
+  float *hsum_s = reinterpret_cast<float *>(smem + L.hsum) + (size_t)team * T * (kFp4 ? 2 : Gf);
+  unsigned int *hrowmax = reinterpret_cast<unsigned int *>(hsum_s + T);  // NVFP4 only
 
   // ---- team `team` runs the CTA's items q = team, team + 2, ...
   bool aborted = false;
@@ -686,10 +757,29 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
       // (bounded: only a broken contract waits for seconds), into the bf16
       // tile that sits behind the weights in this stage
       const int words = ntok * F;
+      // NVFP4 with few enough values: channel pairs kept in registers for
+      // the quantisation (no second pass over the words)
+      const bool regs = kFp4 && words / 2 <= 8 * kTeamThreads;
+      float2 hv[8];
+      if (kFp4 && ttid < ntok) hrowmax[ttid] = 0u;
       uint32_t spins = 0;
       bool ready = false;
       while (true) {
         bool mine = true;
+        if (regs) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int P = ttid + kTeamThreads * i;
+            if (P < words / 2) {
+              const int n = P / (F / 2), f = 2 * (P % (F / 2));
+              const unsigned long long *wp = a.hbuf + (size_t)slot_rows[r0 + n] * F + f;
+              const unsigned long long w0 = ld_relaxed_u64(wp), w1 = ld_relaxed_u64(wp + 1);
+              if ((unsigned int)(w0 & 0xFFFFFFFFull) != epoch || (unsigned int)(w1 & 0xFFFFFFFFull) != epoch)
+                mine = false;
+              hv[i] = make_float2(__uint_as_float((uint32_t)(w0 >> 32)), __uint_as_float((uint32_t)(w1 >> 32)));
+            }
+          }
+        } else
         for (int v = ttid; v < words; v += kTeamThreads) {
           const int n = v / F, f = v % F;
           const unsigned long long w =
@@ -708,6 +798,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
       }
       if (!kFp4) {
         group_sums(h_s, ntok, F, Gf, hsum_s, ttid, kTeamThreads);
+      } else if (regs) {
+        nvfp4_pairs_f16<8>(hv, ntok, F, ttid, kTeamThreads, hrowmax, hsum_s, h_s, [&] { team_sync(bar_id); });
+        team_sync(bar_id);
       } else {  // warp per row: h (fp32) -> NVFP4 -> E2M1 * S_b in h_s, G in hsum_s
         for (int n = tw; n < ntok; n += kTeamWarps) {
           const unsigned long long *hr = a.hbuf + (size_t)slot_rows[r0 + n] * F;
