@@ -3,23 +3,26 @@
 // Prefill groups the rows of a batch by routed expert ("drama-rs", sections
 // "Apple Silicon (MLX)" and "Layout": prefill runs a grouped MoE); every
 // expert's rows then form a dense contraction with that expert's weights.
-// Two launches of one kernel template:
+// Two launches of one kernel template, each tile two 128-row MMA blocks that
+// share the activation tile:
 //   gate/up:  D_gate, D_up [128 features][BN rows] = W [128][H] . X[BN][H]^T,
 //             epilogue h = SiLU(D_gate) * D_up -> bf16 workspace [rows][F]
-//   down:     D [128 outputs][BN rows] = W_down [128][F] . h[BN][F]^T
+//   down:     D_0, D_1 [2 x 128 outputs][BN rows] = W_down [256][F] . h[BN][F]^T
 //             epilogue -> y_perm bf16 [rows][H]
-// The weights are the MMA's A operand (M = 128 rows of one matrix), the rows
-// of an expert its B operand (N = BN tokens), so a few-row expert wastes N,
-// not M.
+// The weights are the MMA's A operand (M = 128 rows per block), the rows of
+// an expert its B operand (N = BN tokens), so a few-row expert wastes N, not
+// M.
 //
 // Per 64-channel k block (one quantisation group):
-//   producer warp:   bulk copies of the packed int4 blocks, TMA (128-byte
-//                    swizzle) of the activation tile
-//   dequant warps:   int4 -> bf16 (fp32 q*s+m, rounded to nearest even) into
-//                    the 128-byte-swizzled K-major smem layout the MMA reads
+//   producer warp:   one TMA box per matrix of packed int4 blocks (8 strips),
+//                    TMA (128-byte swizzle) of the activation tile
+//   dequant warps:   int4 -> bf16 (fp32 q*s+m with one rounding, then nearest
+//                    even) into the 128-byte-swizzled K-major smem layout the
+//                    MMA reads
 //   MMA thread:      tcgen05.mma kind::f16 (bf16 x bf16 -> fp32 in tensor
 //                    memory), four k16 steps per block, commit -> stage free
-// then the dequant warps run the epilogue from tensor memory (tcgen05.ld).
+// then the dequant warps run the epilogue from tensor memory (tcgen05.ld),
+// turning 32 outputs x 16 rows around in shared memory for 16-byte stores.
 // Every wait is bounded; a timeout raises the device error word.
 #include "common.cuh"
 #include "tcgen05.cuh"
