@@ -229,6 +229,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
+      const uint64_t adesc0 = smem_desc_sw128(smem_u32(smem + C::kAOff));
+      const uint64_t bdesc0 = smem_desc_sw128(smem_u32(smem + C::kBOff));
       uint32_t it = 0, tcount = 0;
       for (int t = blockIdx.x; t < ntiles && !*abort_s; t += G, ++tcount) {
         const TileInfo ti = tile_info(t, a.n_sub, chunk_start, a.E, a.offsets);
@@ -249,16 +251,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t at = smem_u32(smem + C::kAOff + sa * C::kABytes);
-          const uint32_t bt = smem_u32(smem + C::kBOff + sb * C::kBBytes);
+          // descriptors: the start-address field counts 16-byte units, so an
+          // offset inside shared memory is added to it directly
+          const uint64_t at = adesc0 + ((uint32_t)sa * C::kABytes >> 4);
+          const uint64_t bt = bdesc0 + ((uint32_t)sb * C::kBBytes >> 4);
 #pragma unroll
           for (int kk = 0; kk < kPfBK / 16; ++kk) {
-            const uint64_t bdesc = smem_desc_sw128(bt + kk * 32);
 #pragma unroll
-            for (int m = 0; m < C::kMats; ++m) {
-              const uint64_t adesc = smem_desc_sw128(at + m * (kPfBM * 128) + kk * 32);
-              tc_mma_bf16(tmem_base + m * kPfBN, adesc, bdesc, idesc, (kb | kk) ? 1u : 0u);
-            }
+            for (int m = 0; m < C::kMats; ++m)
+              tc_mma_bf16(tmem_base + m * kPfBN, at + ((m * (kPfBM * 128) + kk * 32) >> 4), bt + (kk * 32 >> 4),
+                          idesc, (kb | kk) ? 1u : 0u);
           }
           tc_commit(&a_empty[sa]);  // both operand stages are free once these MMAs have read them
           tc_commit(&b_empty[sb]);
@@ -273,15 +275,22 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int quarter = warp & 3;       // TMEM lanes this warp may read
     const int cgrp = dw >> 2;           // epilogue: column group of this warp
     const int gi = lane >> 2, t4 = lane & 3;
-    // Swizzled byte offsets inside a 128-byte row of the pair (16 j + 2 t4 + 8 hk,
-    // +1): 16-byte chunk (2 j + hk) xor gi, byte 4 t4.  Rows g and g + 8 of a
-    // block have the same swizzle phase gi.  (Words 2 and 3 differ from words 0
-    // and 1 only in chunk bit 2: xor 64.)
-    uint32_t koff[2][2];
+    // This warp converts 16-row block rbk of both matrices in every k block:
+    // words 2 wh and 2 wh + 1 of every lane's 16-byte fragment.
+    const int rbk = dw >> 1, wh = dw & 1;
+    // Byte offset of this lane's bf16 pair (channels 16 j + 2 t4 + 8 hk, +1;
+    // j = 2 wh + jj) of row rbk * 16 + gi inside a matrix tile: 8-row atoms of
+    // 1024 bytes, 128-byte rows, 16-byte chunk (2 j + hk) xor gi.  Row
+    // rbk * 16 + gi + 8 is the next atom (+ 1024).
+    uint32_t soff[2][2];
 #pragma unroll
-    for (int j = 0; j < 2; ++j)
+    for (int jj = 0; jj < 2; ++jj)
 #pragma unroll
-      for (int hk = 0; hk < 2; ++hk) koff[j][hk] = (uint32_t)((((2 * j + hk) ^ gi) << 4) | (t4 << 2));
+      for (int hk = 0; hk < 2; ++hk)
+        soff[jj][hk] = (uint32_t)(rbk * 2048 + gi * 128 + ((((2 * (2 * wh + jj) + hk) ^ gi) << 4) | (t4 << 2)));
+    const uint32_t smem_s = smem_u32(smem);
+    const uint32_t code_off = (uint32_t)(rbk * kBlkBytes + 16 * lane + 8 * wh);
+    const uint32_t scale_off = (uint32_t)(rbk * kBlkBytes + kBlkCodeBytes + 4 * gi);
     uint32_t it = 0, tcount = 0;
     for (int t = blockIdx.x; t < ntiles; t += G, ++tcount) {
       const TileInfo ti = tile_info(t, a.n_sub, chunk_start, a.E, a.offsets);
@@ -296,18 +305,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           ok = false;
           break;
         }
-        const uint8_t *raw = smem + C::kRawOff + sr * C::kRawStride;
-        uint8_t *atiles = smem + C::kAOff + sa * C::kABytes;
-        // units (block b, word half wh): matrix b / 8, 16-row block b % 8,
-        // words 2 wh and 2 wh + 1 of every lane
-        for (int u = dw; u < C::kMats * 16; u += kPfDqWarps) {
-          const int b = u >> 1, wh = u & 1;
-          const uint8_t *blk = raw + b * kBlkBytes;
-          const int m = b >> 3, rb = (b & 7) * 16;
-          uint8_t *atile = atiles + m * (kPfBM * 128);
-          const uint2 cw = *reinterpret_cast<const uint2 *>(blk + 16 * lane + 8 * wh);
-          const uint32_t sm0 = *reinterpret_cast<const uint32_t *>(blk + kBlkCodeBytes + 4 * gi);
-          const uint32_t sm1 = *reinterpret_cast<const uint32_t *>(blk + kBlkCodeBytes + 4 * (gi + 8));
+        const uint32_t raw_s = smem_s + C::kRawOff + (uint32_t)sr * C::kRawStride;
+        const uint32_t at_s = smem_s + C::kAOff + (uint32_t)sa * C::kABytes;
+#pragma unroll
+        for (int m = 0; m < C::kMats; ++m) {
+          const uint32_t blk_s = raw_s + (uint32_t)(m * 8 * kBlkBytes);
+          const uint2 cw = lds_v2(blk_s + code_off);
+          const uint32_t sm0 = lds_b32(blk_s + scale_off), sm1 = lds_b32(blk_s + scale_off + 32);
           // fp32 q * s + m with one rounding, as the format defines it.  A
           // nibble at bit p <= 16 of a word, OR-ed into the exponent pattern
           // (150 - p) << 23, is the fp32 value 2^(23 - p) + q exactly, so one
@@ -318,9 +322,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           sc[1] = f16_bits_to_f32((uint16_t)(sm1 & 0xFFFFu));
           mn[0] = f16_bits_to_f32((uint16_t)(sm0 >> 16));
           mn[1] = f16_bits_to_f32((uint16_t)(sm1 >> 16));
-          uint8_t *rowp[2] = {atile + ((rb + gi) >> 3) * 1024 + gi * 128,
-                              atile + ((rb + gi + 8) >> 3) * 1024 + gi * 128};
-          const uint32_t wx = (uint32_t)wh << 6;
+          const uint32_t tile_s = at_s + (uint32_t)(m * (kPfBM * 128));
 #pragma unroll
           for (int jj = 0; jj < 2; ++jj) {
             const uint32_t w = jj ? cw.y : cw.x;
@@ -334,9 +336,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                                          : __uint_as_float((w12 & (0xFu << (ph - 12))) | ((150u - (ph - 12)) << 23));
               const float qlo = __fsub_rn(vlo, (float)(1u << (23 - p)));
               const float qhi = __fsub_rn(vhi, ph == 16 ? 128.0f : (float)(1u << (23 - (ph - 12))));
-              const float lo = __fmaf_rn(qlo, sc[hr], mn[hr]);
-              const float hi = __fmaf_rn(qhi, sc[hr], mn[hr]);
-              *reinterpret_cast<__nv_bfloat162 *>(rowp[hr] + (koff[jj][hk] ^ wx)) = __floats2bfloat162_rn(lo, hi);
+              sts_b32(tile_s + soff[jj][hk] + hr * 1024,
+                      cvt_bf16x2(__fmaf_rn(qlo, sc[hr], mn[hr]), __fmaf_rn(qhi, sc[hr], mn[hr])));
             }
           }
         }
@@ -372,7 +373,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             float y;
             if (kGU) {
               const float g = __uint_as_float(v0[c]), u = __uint_as_float(v1[c]);
-              y = g / (1.0f + __expf(-g)) * u;
+              y = __fdividef(g, 1.0f + __expf(-g)) * u;  // 0 once exp(-g) overflows
             } else {
               y = __uint_as_float(blk ? v1[c] : v0[c]);
             }
