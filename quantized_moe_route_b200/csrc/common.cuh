@@ -114,6 +114,25 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
   return false;
 }
 
+// Bounded wait for warps that have nothing else to do: each poll suspends
+// the thread until the phase completes or about hint_ns have passed, so a
+// waiting warp takes few issue slots.  At most `limit` polls.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t limit,
+                                                uint32_t hint_ns = 10000u) {
+  for (uint32_t i = 0; i < limit; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
+
 // Order this thread's generic-proxy shared-memory accesses before later
 // async-proxy accesses (bulk/TMA copies, tensor-core operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {

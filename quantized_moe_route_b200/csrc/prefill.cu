@@ -35,7 +35,7 @@ constexpr int kPfThreads = (3 + kPfDqWarps) * 32;  // warp 0 int4 producer, 1 MM
 constexpr int kPfBM = 128;       // weight rows per matrix per tile
 constexpr int kPfBN = 256;       // rows (tokens) per tile (the MMA's N is trimmed to the valid rows)
 constexpr int kPfBK = 64;        // k block = one quantisation group
-constexpr uint32_t kPfWaitLimit = 1u << 24;
+constexpr uint32_t kPfWaitPolls = 1u << 18;  // sleeping polls of up to 10 us: a bound of seconds
 
 // Three rings: packed int4 blocks (deep: hides HBM latency, released by the
 // dequant warps), bf16 weight tiles (dequant -> MMA), activation tiles (TMA ->
@@ -186,7 +186,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % C::kRawStages;
           const uint32_t ph = (it / C::kRawStages) & 1u;
-          if (!mbar_wait_bounded(&raw_empty[s], ph ^ 1u, kPfWaitLimit)) {
+          if (!mbar_wait_sleep(&raw_empty[s], ph ^ 1u, kPfWaitPolls)) {
             fail();
             break;
           }
@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % C::kBStages;
           const uint32_t ph = (it / C::kBStages) & 1u;
-          if (!mbar_wait_bounded(&b_empty[s], ph ^ 1u, kPfWaitLimit)) {
+          if (!mbar_wait_sleep(&b_empty[s], ph ^ 1u, kPfWaitPolls)) {
             fail();
             break;
           }
@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       for (int t = blockIdx.x; t < ntiles && !*abort_s; t += G, ++tcount) {
         const TileInfo ti = tile_info(t, a.n_sub, chunk_start, a.E, a.offsets);
         const uint32_t idesc = idesc_bf16_f32((ti.nvalid + 15) & ~15);  // N: valid rows, rounded to 16
-        if (!mbar_wait_bounded(tmem_empty, (tcount & 1u) ^ 1u, kPfWaitLimit)) {
+        if (!mbar_wait_sleep(tmem_empty, (tcount & 1u) ^ 1u, kPfWaitPolls)) {
           fail();
           break;
         }
@@ -244,8 +244,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int sa = it % C::kAStages, sb = it % C::kBStages;
           const uint32_t pa = (it / C::kAStages) & 1u, pb = (it / C::kBStages) & 1u;
-          if (!mbar_wait_bounded(&b_full[sb], pb, kPfWaitLimit) ||
-              !mbar_wait_bounded(&a_full[sa], pa, kPfWaitLimit)) {
+          if (!mbar_wait_sleep(&b_full[sb], pb, kPfWaitPolls) ||
+              !mbar_wait_sleep(&a_full[sa], pa, kPfWaitPolls)) {
             fail();
             ok = false;
             break;
@@ -298,8 +298,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       for (int kb = 0; kb < KB; ++kb, ++it) {
         const int sr = it % C::kRawStages, sa = it % C::kAStages;
         const uint32_t pr = (it / C::kRawStages) & 1u, pa = (it / C::kAStages) & 1u;
-        const bool landed = mbar_wait_bounded(&raw_full[sr], pr, kPfWaitLimit) &&
-                            mbar_wait_bounded(&a_empty[sa], pa ^ 1u, kPfWaitLimit);
+        const bool landed = mbar_wait_sleep(&raw_full[sr], pr, kPfWaitPolls) &&
+                            mbar_wait_sleep(&a_empty[sa], pa ^ 1u, kPfWaitPolls);
         if (!landed || *abort_s) {
           if (!landed) fail();
           ok = false;
@@ -351,7 +351,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (!ok) break;
       // ---- epilogue: accumulators of this tile; the four warps of a lane
       // quarter split the columns
-      if (!mbar_wait_bounded(tmem_full, tcount & 1u, kPfWaitLimit)) {
+      if (!mbar_wait_sleep(tmem_full, tcount & 1u, kPfWaitPolls)) {
         fail();
         break;
       }
@@ -364,8 +364,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       for (int c0 = cgrp * 16; c0 < kPfBN; c0 += 64) {
         if (c0 >= ti.nvalid) break;  // uniform across the warp
         uint32_t v0[16], v1[16];
-        tmem_ld16(trow + c0, v0);
-        tmem_ld16(trow + kPfBN + c0, v1);
+        tmem_ld16_async(trow + c0, v0);
+        tmem_ld16_async(trow + kPfBN + c0, v1);
+        tmem_ld_wait();
+        tmem_regs_after_wait(v0);
+        tmem_regs_after_wait(v1);
 #pragma unroll
         for (int blk = 0; blk < (kGU ? 1 : 2); ++blk) {
 #pragma unroll
