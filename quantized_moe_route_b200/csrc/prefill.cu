@@ -312,32 +312,43 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           const uint32_t blk_s = raw_s + (uint32_t)(m * 8 * kBlkBytes);
           const uint2 cw = lds_v2(blk_s + code_off);
           const uint32_t sm0 = lds_b32(blk_s + scale_off), sm1 = lds_b32(blk_s + scale_off + 32);
-          // fp32 q * s + m with one rounding, as the format defines it.  A
-          // nibble at bit p <= 16 of a word, OR-ed into the exponent pattern
-          // (150 - p) << 23, is the fp32 value 2^(23 - p) + q exactly, so one
-          // integer op per code (plus one shift per word for the nibbles at
-          // 20, 24, 28) and an exact subtraction give q in fp32.
-          float sc[2], mn[2];
+          // q * s + m in fp32 from one FMA per code.  A nibble at bit p of a
+          // word, OR-ed into the exponent pattern (150 - p) << 23, is the fp32
+          // value v = 2^K + q (K = 23 - p), and v * s + (m - 2^K s) = q s + m.
+          // The codes are first brought to bit 8, 12 or 16 (K = 15, 11, 7), so
+          // the constant m - 2^K s is exact unless m and 2^K s lie more than
+          // 2^11 apart in magnitude, and otherwise off by at most 2^-24 2^K |s|
+          // (<= 2^-9 |s|, far below the bf16 rounding that follows).
+          float sc[2], mn[2], c8[2], c12[2], c16[2];
           sc[0] = f16_bits_to_f32((uint16_t)(sm0 & 0xFFFFu));
           sc[1] = f16_bits_to_f32((uint16_t)(sm1 & 0xFFFFu));
           mn[0] = f16_bits_to_f32((uint16_t)(sm0 >> 16));
           mn[1] = f16_bits_to_f32((uint16_t)(sm1 >> 16));
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            c8[r] = __fmaf_rn(-32768.0f, sc[r], mn[r]);
+            c12[r] = __fmaf_rn(-2048.0f, sc[r], mn[r]);
+            c16[r] = __fmaf_rn(-128.0f, sc[r], mn[r]);
+          }
           const uint32_t tile_s = at_s + (uint32_t)(m * (kPfBM * 128));
 #pragma unroll
           for (int jj = 0; jj < 2; ++jj) {
             const uint32_t w = jj ? cw.y : cw.x;
-            const uint32_t w12 = w >> 12;  // nibbles 20, 24, 28 at 8, 12, 16
+            const uint32_t wl = w << 8;   // nibbles 0, 1 at bits 8, 12
+            const uint32_t wr = w >> 12;  // nibbles 5, 6, 7 at bits 8, 12, 16
+            // nibble i (channel k) and i + 4 (k + 1) of pair i: hr = i & 1, hk = i >> 1
+            const float v[4][2] = {
+                {__uint_as_float((wl & 0x00000F00u) | (142u << 23)), __uint_as_float((w & 0x000F0000u) | (134u << 23))},
+                {__uint_as_float((wl & 0x0000F000u) | (138u << 23)), __uint_as_float((wr & 0x00000F00u) | (142u << 23))},
+                {__uint_as_float((w & 0x00000F00u) | (142u << 23)), __uint_as_float((wr & 0x0000F000u) | (138u << 23))},
+                {__uint_as_float((w & 0x0000F000u) | (138u << 23)), __uint_as_float((wr & 0x000F0000u) | (134u << 23))}};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {  // nibble 4 i (channel k) and 4 i + 16 (k + 1): hr = i & 1, hk = i >> 1
+            for (int i = 0; i < 4; ++i) {
               const int hr = i & 1, hk = i >> 1;
-              const int p = 4 * i, ph = p + 16;  // ph: 16 from w, else from w12 at ph - 12
-              const float vlo = __uint_as_float((w & (0xFu << p)) | ((150u - p) << 23));
-              const float vhi = ph == 16 ? __uint_as_float((w & 0xF0000u) | (134u << 23))
-                                         : __uint_as_float((w12 & (0xFu << (ph - 12))) | ((150u - (ph - 12)) << 23));
-              const float qlo = __fsub_rn(vlo, (float)(1u << (23 - p)));
-              const float qhi = __fsub_rn(vhi, ph == 16 ? 128.0f : (float)(1u << (23 - (ph - 12))));
+              const float clo = i == 0 || i == 2 ? c8[hr] : c12[hr];
+              const float chi = i == 0 || i == 3 ? c16[hr] : (i == 1 ? c8[hr] : c12[hr]);
               sts_b32(tile_s + soff[jj][hk] + hr * 1024,
-                      cvt_bf16x2(__fmaf_rn(qlo, sc[hr], mn[hr]), __fmaf_rn(qhi, sc[hr], mn[hr])));
+                      cvt_bf16x2(__fmaf_rn(v[i][0], sc[hr], clo), __fmaf_rn(v[i][1], sc[hr], chi)));
             }
           }
         }
