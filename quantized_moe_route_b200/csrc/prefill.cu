@@ -234,7 +234,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       uint32_t it = 0, tcount = 0;
       for (int t = blockIdx.x; t < ntiles && !*abort_s; t += G, ++tcount) {
         const TileInfo ti = tile_info(t, a.n_sub, chunk_start, a.E, a.offsets);
-        const uint32_t idesc = idesc_bf16_f32((ti.nvalid + 15) & ~15);  // N: valid rows, rounded to 16
+        // A tile of at most 128 rows is issued transposed (rows on M, the 256
+        // weight rows on N): one MMA per k16 step instead of two.  An MMA
+        // costs about as much at N = 16 as at N = 200, so this halves the
+        // tensor time of the many few-row tiles.
+        const bool swapped = ti.nvalid <= kPfBM;
+        const uint32_t idesc = idesc_bf16_f32(swapped ? C::kMats * kPfBM : (ti.nvalid + 15) & ~15);
         if (!mbar_wait_sleep(tmem_empty, (tcount & 1u) ^ 1u, kPfWaitPolls)) {
           fail();
           break;
@@ -255,12 +260,20 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           // offset inside shared memory is added to it directly
           const uint64_t at = adesc0 + ((uint32_t)sa * C::kABytes >> 4);
           const uint64_t bt = bdesc0 + ((uint32_t)sb * C::kBBytes >> 4);
+          if (swapped) {
+            // D [128 rows][256 weight rows] = X [128][16] . W [256][16]^T: the two
+            // 128-row weight tiles are contiguous, one 256-row operand
 #pragma unroll
-          for (int kk = 0; kk < kPfBK / 16; ++kk) {
+            for (int kk = 0; kk < kPfBK / 16; ++kk)
+              tc_mma_bf16(tmem_base, bt + (kk * 32 >> 4), at + (kk * 32 >> 4), idesc, (kb | kk) ? 1u : 0u);
+          } else {
 #pragma unroll
-            for (int m = 0; m < C::kMats; ++m)
-              tc_mma_bf16(tmem_base + m * kPfBN, at + ((m * (kPfBM * 128) + kk * 32) >> 4), bt + (kk * 32 >> 4),
-                          idesc, (kb | kk) ? 1u : 0u);
+            for (int kk = 0; kk < kPfBK / 16; ++kk) {
+#pragma unroll
+              for (int m = 0; m < C::kMats; ++m)
+                tc_mma_bf16(tmem_base + m * kPfBN, at + ((m * (kPfBM * 128) + kk * 32) >> 4), bt + (kk * 32 >> 4),
+                            idesc, (kb | kk) ? 1u : 0u);
+            }
           }
           tc_commit(&a_empty[sa]);  // both operand stages are free once these MMAs have read them
           tc_commit(&b_empty[sb]);
@@ -368,42 +381,79 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       tc_fence_after();
       const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16);
-      // each warp turns its 32 outputs x 16 rows around in shared memory and
-      // writes them as 16-byte vectors (row c: 64 bytes from 4 lanes)
-      uint16_t *stage = reinterpret_cast<uint16_t *>(smem + C::kEpiOff) + dw * 16 * 32;
-      const int fbase = ti.sub * (kGU ? kPfBM : 2 * kPfBM) + quarter * 32;  // first output of this warp
-      for (int c0 = cgrp * 16; c0 < kPfBN; c0 += 64) {
-        if (c0 >= ti.nvalid) break;  // uniform across the warp
-        uint32_t v0[16], v1[16];
-        tmem_ld16_async(trow + c0, v0);
-        tmem_ld16_async(trow + kPfBN + c0, v1);
-        tmem_ld_wait();
-        tmem_regs_after_wait(v0);
-        tmem_regs_after_wait(v1);
+      if (ti.nvalid <= kPfBM) {
+        // transposed accumulators: lane quarter q holds rows 32 q + lane, the
+        // columns are the tile's 256 weight rows (gate then up, or 256
+        // consecutive outputs); the four warps of a quarter split the
+        // columns and every thread writes a stretch of its own row
+        const int r = quarter * 32 + lane;
+        const bool live = r < ti.nvalid;
+        uint16_t *orow = a.out + (size_t)(ti.row0 + (live ? r : 0)) * a.ld_out + ti.sub * (kGU ? kPfBM : 2 * kPfBM);
 #pragma unroll
-        for (int blk = 0; blk < (kGU ? 1 : 2); ++blk) {
+        for (int h = 0; h < 2; ++h) {
+          const int c0 = kGU ? cgrp * 32 + 16 * h : cgrp * 64 + 32 * h;
+          uint32_t v0[16], v1[16];
+          tmem_ld16_async(trow + c0, v0);                     // gate (or outputs c0 ..)
+          tmem_ld16_async(trow + (kGU ? kPfBM : 16) + c0, v1);  // up (or outputs c0 + 16 ..)
+          tmem_ld_wait();
+          tmem_regs_after_wait(v0);
+          tmem_regs_after_wait(v1);
+          uint32_t pk[kGU ? 8 : 16];
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            float y;
+          for (int c = 0; c < (kGU ? 8 : 16); ++c) {
             if (kGU) {
-              const float g = __uint_as_float(v0[c]), u = __uint_as_float(v1[c]);
-              y = __fdividef(g, 1.0f + __expf(-g)) * u;  // 0 once exp(-g) overflows
+              const float g0 = __uint_as_float(v0[2 * c]), g1 = __uint_as_float(v0[2 * c + 1]);
+              const float u0 = __uint_as_float(v1[2 * c]), u1 = __uint_as_float(v1[2 * c + 1]);
+              pk[c] = cvt_bf16x2(__fdividef(g0, 1.0f + __expf(-g0)) * u0, __fdividef(g1, 1.0f + __expf(-g1)) * u1);
             } else {
-              y = __uint_as_float(blk ? v1[c] : v0[c]);
+              const uint32_t *v = c < 8 ? v0 : v1;
+              pk[c] = cvt_bf16x2(__uint_as_float(v[(2 * c) & 15]), __uint_as_float(v[(2 * c + 1) & 15]));
             }
-            stage[c * 32 + lane] = f32_to_bf16_bits(y);
           }
-          __syncwarp();
+          if (live) {
 #pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            const int q = lane + 32 * r, c = q >> 2, part = q & 3;
-            if (c0 + c < ti.nvalid) {
-              const uint4 v = *reinterpret_cast<const uint4 *>(stage + c * 32 + 8 * part);
-              *reinterpret_cast<uint4 *>(a.out + (size_t)(ti.row0 + c0 + c) * a.ld_out + fbase +
-                                         blk * kPfBM + 8 * part) = v;
-            }
+            for (int q = 0; q < (kGU ? 2 : 4); ++q)
+              *reinterpret_cast<uint4 *>(orow + c0 + 8 * q) = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
           }
-          __syncwarp();
+        }
+      } else {
+        // each warp turns its 32 outputs x 16 rows around in shared memory and
+        // writes them as 16-byte vectors (row c: 64 bytes from 4 lanes)
+        uint16_t *stage = reinterpret_cast<uint16_t *>(smem + C::kEpiOff) + dw * 16 * 32;
+        const int fbase = ti.sub * (kGU ? kPfBM : 2 * kPfBM) + quarter * 32;  // first output of this warp
+        for (int c0 = cgrp * 16; c0 < kPfBN; c0 += 64) {
+          if (c0 >= ti.nvalid) break;  // uniform across the warp
+          uint32_t v0[16], v1[16];
+          tmem_ld16_async(trow + c0, v0);
+          tmem_ld16_async(trow + kPfBN + c0, v1);
+          tmem_ld_wait();
+          tmem_regs_after_wait(v0);
+          tmem_regs_after_wait(v1);
+#pragma unroll
+          for (int blk = 0; blk < (kGU ? 1 : 2); ++blk) {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              float y;
+              if (kGU) {
+                const float g = __uint_as_float(v0[c]), u = __uint_as_float(v1[c]);
+                y = __fdividef(g, 1.0f + __expf(-g)) * u;  // 0 once exp(-g) overflows
+              } else {
+                y = __uint_as_float(blk ? v1[c] : v0[c]);
+              }
+              stage[c * 32 + lane] = f32_to_bf16_bits(y);
+            }
+            __syncwarp();
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+              const int q = lane + 32 * r, c = q >> 2, part = q & 3;
+              if (c0 + c < ti.nvalid) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(stage + c * 32 + 8 * part);
+                *reinterpret_cast<uint4 *>(a.out + (size_t)(ti.row0 + c0 + c) * a.ld_out + fbase +
+                                           blk * kPfBM + 8 * part) = v;
+              }
+            }
+            __syncwarp();
+          }
         }
       }
       tc_fence_before();
