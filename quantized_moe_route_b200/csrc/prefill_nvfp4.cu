@@ -37,7 +37,7 @@ constexpr int kNpKT = 256;   // channels per stage: 128 code bytes per row
 constexpr int kNpBoxRows = 32;  // activation rows per TMA box (a tile loads the boxes it needs)
 constexpr int kNpEpiWarps = 8;  // warps 4..11: two per tensor-memory lane quarter
 constexpr int kNpThreads = (4 + kNpEpiWarps) * 32;
-constexpr uint32_t kNpWaitLimit = 1u << 24;
+constexpr uint32_t kNpWaitPolls = 1u << 18;  // sleeping polls of up to 10 us: a bound of seconds
 
 template <bool kGU>
 struct NpCfg {
@@ -217,7 +217,7 @@ __global__ void __launch_bounds__(kNpThreads, 1)
         for (int kt = 0; kt < KT; ++kt, ++it) {
           const int s = it % C::kStages;
           const uint32_t ph = (it / C::kStages) & 1u;
-          if (!mbar_wait_bounded(&empty[s], ph ^ 1u, kNpWaitLimit)) {
+          if (!mbar_wait_sleep(&empty[s], ph ^ 1u, kNpWaitPolls)) {
             fail();
             break;
           }
@@ -250,7 +250,7 @@ __global__ void __launch_bounds__(kNpThreads, 1)
       for (int kt = 0; kt < KT; ++kt, ++it) {
         const int s = it % C::kStages;
         const uint32_t ph = (it / C::kStages) & 1u;
-        if (!mbar_wait_bounded(&full[s], ph, kNpWaitLimit) || *abort_s) {
+        if (!mbar_wait_sleep(&full[s], ph, kNpWaitPolls) || *abort_s) {
           if (lane == 0 && !*abort_s) fail();
           ok = false;
           break;
@@ -287,13 +287,16 @@ __global__ void __launch_bounds__(kNpThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
+      // descriptors: the start-address field counts 16-byte units, so an
+      // offset inside shared memory is added to it directly
+      const uint64_t dsw0 = smem_desc_sw128(smem_u32(smem)), dpl0 = smem_desc_plain(smem_u32(smem));
       uint32_t it = 0, tcount = 0;
       for (int t = blockIdx.x; t < ntiles && !*abort_s; t += G, ++tcount) {
         const NpTile ti = np_tile(t, a.n_sub, chunk_start, a.E, a.offsets);
         const uint32_t idesc = idesc_nvf4((ti.nvalid + 15) & ~15);
         const int ab = tcount % C::kAcc;
         const uint32_t acc0 = tmem_base + ab * C::kAccCols;
-        if (!mbar_wait_bounded(&tmem_empty[ab], ((tcount / C::kAcc) & 1u) ^ 1u, kNpWaitLimit)) {
+        if (!mbar_wait_sleep(&tmem_empty[ab], ((tcount / C::kAcc) & 1u) ^ 1u, kNpWaitPolls)) {
           fail();
           break;
         }
@@ -302,33 +305,31 @@ __global__ void __launch_bounds__(kNpThreads, 1)
         for (int kt = 0; kt < KT; ++kt, ++it) {
           const int s = it % C::kStages;
           const uint32_t ph = (it / C::kStages) & 1u;
-          if (!mbar_wait_bounded(&sfready[s], ph, kNpWaitLimit)) {
+          if (!mbar_wait_sleep(&sfready[s], ph, kNpWaitPolls)) {
             fail();
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + s * C::kStageBytes);
+          const uint32_t so = (uint32_t)s * C::kStageBytes;  // stage offset
+          const uint64_t sw = dsw0 + (so >> 4), pl = dpl0 + (so >> 4);
           const uint32_t sf0 = tmem_base + C::kAcc * C::kAccCols + s * C::kSfCols;
 #pragma unroll
           for (int m = 0; m < C::kMats; ++m)
 #pragma unroll
             for (int kb = 0; kb < 4; ++kb)
-              tc_cp_32x128b_x4(sf0 + m * 16 + kb * 4,
-                               smem_desc_plain(sa + C::kOffAAtom + (m * 4 + kb) * C::kAtom));
+              tc_cp_32x128b_x4(sf0 + m * 16 + kb * 4, pl + ((C::kOffAAtom + (m * 4 + kb) * C::kAtom) >> 4));
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb)
-            tc_cp_32x128b_x4(sf0 + C::kMats * 16 + kb * 4, smem_desc_plain(sa + C::kOffBAtom + kb * C::kAtom));
+            tc_cp_32x128b_x4(sf0 + C::kMats * 16 + kb * 4, pl + ((C::kOffBAtom + kb * C::kAtom) >> 4));
+          // one accumulator's four MMAs, then the other's
 #pragma unroll
-          for (int kb = 0; kb < 4; ++kb) {
-            const uint64_t bdesc = smem_desc_sw128(sa + C::kOffB + kb * 32);
+          for (int m = 0; m < C::kMats; ++m)
 #pragma unroll
-            for (int m = 0; m < C::kMats; ++m) {
-              const uint64_t adesc = smem_desc_sw128(sa + C::kOffA + m * C::kACodes + kb * 32);
-              tc_mma_nvf4(acc0 + m * kNpBN, adesc, bdesc, idesc, sf0 + m * 16 + kb * 4,
+            for (int kb = 0; kb < 4; ++kb)
+              tc_mma_nvf4(acc0 + m * kNpBN, sw + ((C::kOffA + m * C::kACodes + kb * 32) >> 4),
+                          sw + ((C::kOffB + kb * 32) >> 4), idesc, sf0 + m * 16 + kb * 4,
                           sf0 + C::kMats * 16 + kb * 4, (kt | kb) ? 1u : 0u);
-            }
-          }
           tc_commit(&empty[s]);  // stage (and its tensor-memory scales) free once these MMAs are done
         }
         if (!ok) break;
@@ -343,7 +344,7 @@ __global__ void __launch_bounds__(kNpThreads, 1)
     for (int t = blockIdx.x; t < ntiles; t += G, ++tcount) {
       const NpTile ti = np_tile(t, a.n_sub, chunk_start, a.E, a.offsets);
       const int ab = tcount % C::kAcc;
-      if (!mbar_wait_bounded(&tmem_full[ab], (tcount / C::kAcc) & 1u, kNpWaitLimit) || *abort_s) {
+      if (!mbar_wait_sleep(&tmem_full[ab], (tcount / C::kAcc) & 1u, kNpWaitPolls) || *abort_s) {
         if (lane == 0 && !*abort_s) fail();
         break;
       }
