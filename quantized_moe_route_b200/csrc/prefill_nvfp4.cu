@@ -354,13 +354,18 @@ __global__ void __launch_bounds__(kNpThreads, 1)
       const float wG = a.w_G[ti.e];
       for (int c0 = 16 * half; c0 < ti.nvalid; c0 += 32) {
         uint32_t v0[16], v1[16];
-        tmem_ld16(trow + c0, v0);
-        if (kGU) tmem_ld16(trow + kNpBN + c0, v1);
+        tmem_ld16_async(trow + c0, v0);
+        if (kGU) tmem_ld16_async(trow + kNpBN + c0, v1);
+        // the 16 rows' activation globals: one load per lane, then broadcast
+        const float gl = lane < 16 && c0 + lane < ti.nvalid ? __fmul_rn(a.act_G[ti.row0 + c0 + lane], wG) : 0.f;
+        tmem_ld_wait();
+        tmem_regs_after_wait(v0);
+        if (kGU) tmem_regs_after_wait(v1);
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
+          const float gs = __shfl_sync(0xffffffffu, gl, c);
           if (c0 + c < ti.nvalid) {
             const int p = ti.row0 + c0 + c;
-            const float gs = __fmul_rn(a.act_G[p], wG);
             if (kGU) {
               const float g = __fmul_rn(__uint_as_float(v0[c]), gs);
               const float u = __fmul_rn(__uint_as_float(v1[c]), gs);
