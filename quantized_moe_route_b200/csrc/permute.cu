@@ -1,11 +1,15 @@
 // permute.cu -- group the T*k routed rows by expert ("drama-rs", section
 // "Apple Silicon (MLX)": prefill groups rows by routed expert).
 //
-// Three stream-ordered kernels, no global atomics:
+// Stream-ordered kernels, no global atomics:
 //   1. per-chunk expert histograms (shared-memory counters),
 //   2. one block: totals, exclusive scan -> offsets, per-chunk bases,
 //   3. per chunk: stable ranks with warp match + popc, scatter of
-//      sorted_rows / inv, and the optional gather of x rows into x_perm.
+//      sorted_rows / inv,
+//   4. optional: the gather of x rows into x_perm, one warp per destination
+//      row, many rows in flight across the whole GPU.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace moe {
@@ -83,15 +87,11 @@ __global__ void perm_scan_kernel(const int32_t *__restrict__ hist, int nchunks, 
   }
 }
 
-// One warp assigns positions to the chunk's rows 32 at a time, in row order;
-// then the whole block copies the activation rows.
-__global__ void perm_scatter_kernel(const int32_t *__restrict__ idx, int R, int E, int k,
+// One warp assigns positions to the chunk's rows 32 at a time, in row order.
+__global__ void perm_scatter_kernel(const int32_t *__restrict__ idx, int R, int E,
                                     const int32_t *__restrict__ base,
-                                    int32_t *__restrict__ sorted_rows, int32_t *__restrict__ inv,
-                                    const uint16_t *__restrict__ x, int H,
-                                    uint16_t *__restrict__ x_perm) {
+                                    int32_t *__restrict__ sorted_rows, int32_t *__restrict__ inv) {
   extern __shared__ int32_t run[];  // [E] running position per expert
-  __shared__ int32_t pos_of[kPermChunk];
   const int r0 = blockIdx.x * kPermChunk;
   const int nrows = min(R - r0, kPermChunk);
   for (int e = threadIdx.x; e < E; e += blockDim.x) run[e] = base[(size_t)blockIdx.x * E + e];
@@ -108,7 +108,6 @@ __global__ void perm_scatter_kernel(const int32_t *__restrict__ idx, int R, int 
       if (valid) {
         const int rank = __popc(peers & ((1u << lane) - 1u));
         const int p = run[e] + rank;
-        pos_of[i] = p;
         sorted_rows[p] = r0 + i;
         inv[r0 + i] = p;
       }
@@ -117,14 +116,35 @@ __global__ void perm_scatter_kernel(const int32_t *__restrict__ idx, int R, int 
       __syncwarp();
     }
   }
-  __syncthreads();
-  if (!x_perm) return;
+}
+
+// x_perm[p] = x[sorted_rows[p] / k] for the offsets[E] grouped rows: warp w
+// of the grid copies rows w, w + nwarps, ...; each lane moves up to eight
+// 16-byte vectors of a row at once (all loads before the stores).
+__global__ void perm_gather_kernel(const int32_t *__restrict__ sorted_rows,
+                                   const int32_t *__restrict__ offsets, int E, int k,
+                                   const uint16_t *__restrict__ x, int H,
+                                   uint16_t *__restrict__ x_perm) {
+  const int lane = threadIdx.x & 31;
+  const int nwarps = (int)(gridDim.x * blockDim.x) >> 5;
+  const int total = offsets[E];
   const int vec = H / 8;  // 16-byte vectors per row
-  for (int i = 0; i < nrows; ++i) {
-    if ((unsigned)idx[r0 + i] >= (unsigned)E) continue;
-    const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)((r0 + i) / k) * H);
-    uint4 *dst = reinterpret_cast<uint4 *>(x_perm + (size_t)pos_of[i] * H);
-    for (int v = threadIdx.x; v < vec; v += blockDim.x) dst[v] = src[v];
+  for (int p = (int)(blockIdx.x * blockDim.x + threadIdx.x) >> 5; p < total; p += nwarps) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)(sorted_rows[p] / k) * H);
+    uint4 *dst = reinterpret_cast<uint4 *>(x_perm + (size_t)p * H);
+    for (int v0 = 0; v0 < vec; v0 += 8 * 32) {
+      uint4 buf[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int v = v0 + 32 * j + lane;
+        if (v < vec) buf[j] = src[v];
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int v = v0 + 32 * j + lane;
+        if (v < vec) dst[v] = buf[j];
+      }
+    }
   }
 }
 
@@ -175,6 +195,13 @@ extern "C" MOE_API moe_status moe_permute(const int32_t *idx, int T, int k, int 
   perm_scan_kernel<<<1, 1024, shE, s>>>(hist, nch, E, counts, offsets, base);
   st = launch_status();
   if (st != MOE_OK) return st;
-  perm_scatter_kernel<<<nch, 256, shE, s>>>(idx, R, E, k, base, sorted_rows, inv, x, H, x_perm);
+  perm_scatter_kernel<<<nch, 256, shE, s>>>(idx, R, E, base, sorted_rows, inv);
+  st = launch_status();
+  if (st != MOE_OK || !gather) return st;
+  int dev = 0, nsm = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const int blocks = (int)std::min<long long>((R + 7) / 8, 8LL * nsm);  // 8 warps per block
+  perm_gather_kernel<<<blocks, 256, 0, s>>>(sorted_rows, offsets, E, k, x, H, x_perm);
   return launch_status();
 }
