@@ -17,41 +17,27 @@ __global__ void combine_kernel(const void *__restrict__ Y, const int32_t *__rest
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  // up to eight of the k rows in flight at once; the sum still runs j = 0, 1, ...
-  for (int j0 = 0; j0 < k; j0 += 8) {
-    size_t p[8];
-    float wj[8];
+  for (int j = 0; j < k; ++j) {
+    const int r = t * k + j;
+    const size_t p = inv ? (size_t)inv[r] : (size_t)r;
+    const float wj = w[r];
+    float v[8];
+    if (kBf16In) {
+      uint4 q = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(Y) + p * H + c0);
+      const uint32_t u[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj) {
-      const int r = t * k + min(j0 + jj, k - 1);
-      p[jj] = inv ? (size_t)inv[r] : (size_t)r;
-      wj[jj] = w[r];
-    }
-    float v[8][8];
-#pragma unroll
-    for (int jj = 0; jj < 8; ++jj) {
-      if (j0 + jj >= k) break;
-      if (kBf16In) {
-        const uint4 q = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(Y) + p[jj] * H + c0);
-        const uint32_t u[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          v[jj][2 * i] = __uint_as_float(u[i] << 16);
-          v[jj][2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
-        }
-      } else {
-        const float4 *src = reinterpret_cast<const float4 *>(static_cast<const float *>(Y) + p[jj] * H + c0);
-        const float4 a = src[0], b = src[1];
-        v[jj][0] = a.x; v[jj][1] = a.y; v[jj][2] = a.z; v[jj][3] = a.w;
-        v[jj][4] = b.x; v[jj][5] = b.y; v[jj][6] = b.z; v[jj][7] = b.w;
+      for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(u[i] << 16);
+        v[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
       }
+    } else {
+      const float4 *src = reinterpret_cast<const float4 *>(static_cast<const float *>(Y) + p * H + c0);
+      float4 a = src[0], b = src[1];
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+      v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
     }
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj) {
-      if (j0 + jj >= k) break;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], __fmul_rn(wj[jj], v[jj][i]));
-    }
+    for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], __fmul_rn(wj, v[i]));
   }
   uint4 o;
   o.x = pack_bf16x2(acc[0], acc[1]);
