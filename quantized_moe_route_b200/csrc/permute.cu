@@ -28,23 +28,35 @@ __global__ void perm_hist_kernel(const int32_t *__restrict__ idx, int R, int E,
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(size_t)blockIdx.x * E + e] = sh[e];
 }
 
-// One block of up to 1024 threads; thread e walks the chunks of expert e.
-__global__ void perm_scan_kernel(const int32_t *__restrict__ hist, int nchunks, int E,
+// One block of 1024 threads.  Each expert's chunks are split among S
+// consecutive threads (S a power of two, S * E <= 1024 where E allows): every
+// thread sums a contiguous range of chunks, the S partial sums are combined
+// with warp shuffles (totals, then the per-chunk running bases).
+__global__ void perm_scan_kernel(const int32_t *__restrict__ hist, int nchunks, int E, int S,
                                  int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
                                  int32_t *__restrict__ base) {
   extern __shared__ int32_t sh[];  // [E] totals then scanned
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int s = 0;
-    for (int c = 0; c < nchunks; ++c) s += hist[(size_t)c * E + e];
-    sh[e] = s;
-    counts[e] = s;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int per = (nchunks + S - 1) / S;  // chunks of one thread
+  const int ngroups = (E * S + blockDim.x - 1) / blockDim.x;
+  for (int g = 0; g < ngroups; ++g) {
+    const int idx = g * blockDim.x + threadIdx.x;
+    const int e = idx / S, part = idx % S;
+    int sum = 0;
+    if (e < E)
+      for (int c = part * per; c < min(nchunks, (part + 1) * per); ++c) sum += hist[(size_t)c * E + e];
+    int tot = sum;
+    for (int o = 1; o < S; o <<= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+    if (e < E && part == 0) {
+      sh[e] = tot;
+      counts[e] = tot;
+    }
   }
   __syncthreads();
   // block-wide exclusive scan of sh[0..E), 1024 entries per pass
   __shared__ int32_t warp_sum[32];
   __shared__ int32_t carry;
   if (threadIdx.x == 0) carry = 0;
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   for (int e0 = 0; e0 < E; e0 += blockDim.x) {
     __syncthreads();
     const int e = e0 + threadIdx.x;
@@ -77,12 +89,26 @@ __global__ void perm_scan_kernel(const int32_t *__restrict__ hist, int nchunks, 
   }
   __syncthreads();
   if (threadIdx.x == 0) offsets[E] = carry;
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int run = sh[e];
-    for (int c = 0; c < nchunks; ++c) {
-      base[(size_t)c * E + e] = run;
-      run += hist[(size_t)c * E + e];
+  // base[c][e] = offsets[e] + sum over c' < c of hist[c'][e]: each thread
+  // starts its chunk range after the ranges of the lower parts
+  for (int g = 0; g < ngroups; ++g) {
+    const int idx = g * blockDim.x + threadIdx.x;
+    const int e = idx / S, part = idx % S;
+    const int c0 = part * per, c1 = min(nchunks, (part + 1) * per);
+    int sum = 0;
+    if (e < E)
+      for (int c = c0; c < c1; ++c) sum += hist[(size_t)c * E + e];
+    int incl = sum;  // inclusive scan over the S parts of this expert
+    for (int o = 1; o < S; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (part >= o) incl += n;
+    }
+    if (e < E) {
+      int run = sh[e] + incl - sum;
+      for (int c = c0; c < c1; ++c) {
+        base[(size_t)c * E + e] = run;
+        run += hist[(size_t)c * E + e];
+      }
     }
   }
 }
@@ -192,7 +218,9 @@ extern "C" MOE_API moe_status moe_permute(const int32_t *idx, int T, int k, int 
   perm_hist_kernel<<<nch, 256, shE, s>>>(idx, R, E, hist);
   moe_status st = launch_status();
   if (st != MOE_OK) return st;
-  perm_scan_kernel<<<1, 1024, shE, s>>>(hist, nch, E, counts, offsets, base);
+  int S = 1;  // threads per expert in the scan: a power of two, S * E <= 1024, S <= 32
+  while (S < 32 && 2 * S * E <= 1024 && S < nch) S *= 2;
+  perm_scan_kernel<<<1, 1024, shE, s>>>(hist, nch, E, S, counts, offsets, base);
   st = launch_status();
   if (st != MOE_OK) return st;
   perm_scatter_kernel<<<nch, 256, shE, s>>>(idx, R, E, base, sorted_rows, inv);

@@ -122,7 +122,9 @@ def _idx_for(T, k, E, mode, seed):
 @pytest.mark.parametrize("T,k,E,mode", [
     (4, 2, 8, "plain"), (1, 8, 256, "plain"), (3, 8, 256, "plain"), (17, 8, 256, "plain"),
     (2048, 8, 256, "zipf"), (512, 8, 256, "zipf"), (100, 1, 256, "one_expert"), (0, 8, 256, "plain"),
-    (33, 2, 8, "plain")])
+    (33, 2, 8, "plain"),
+    # the scan splits each expert's chunks among 8 threads here, and needs two passes over E here
+    (1024, 4, 64, "zipf"), (256, 8, 2048, "plain")])
 def test_permute_matches_oracle_bit_exact(T, k, E, mode):
     H = 128
     idx = _idx_for(T, k, E, mode, 3)
