@@ -13,6 +13,7 @@ __global__ void combine_kernel(const void *__restrict__ Y, const int32_t *__rest
                                uint16_t *__restrict__ y) {
   const int t = blockIdx.y;
   const int c0 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  grid_dep_wait();
   if (t >= T || c0 >= H) return;
   float acc[8];
 #pragma unroll
@@ -45,6 +46,7 @@ __global__ void combine_kernel(const void *__restrict__ Y, const int32_t *__rest
   o.z = pack_bf16x2(acc[4], acc[5]);
   o.w = pack_bf16x2(acc[6], acc[7]);
   *reinterpret_cast<uint4 *>(y + (size_t)t * H + c0) = o;
+  grid_dep_trigger();
 }
 
 }  // namespace moe
@@ -63,9 +65,6 @@ extern "C" MOE_API moe_status moe_unpermute_combine(const void *Y, int y_dtype, 
   if (T > 65535) return MOE_ERR_UNSUPPORTED_SHAPE;
   const int threads = 128;
   dim3 grid((H / 8 + threads - 1) / threads, T);
-  if (y_dtype == 1)
-    combine_kernel<true><<<grid, threads, 0, as_stream(stream)>>>(Y, inv, w, T, k, H, y);
-  else
-    combine_kernel<false><<<grid, threads, 0, as_stream(stream)>>>(Y, inv, w, T, k, H, y);
-  return launch_status();
+  return launch_pdl(y_dtype == 1 ? combine_kernel<true> : combine_kernel<false>, grid, dim3(threads), 0,
+                    as_stream(stream), Y, inv, w, T, k, H, y);
 }

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/moe.h"
 
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
@@ -19,6 +21,30 @@ void set_cuda_error(cudaError_t e);
 moe_status launch_status();  // checks cudaGetLastError after a launch
 
 inline cudaStream_t as_stream(moe_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Launch with programmatic stream serialization: the kernel may begin while
+// the previous kernel on the stream drains, so it calls grid_dep_wait()
+// before it reads anything earlier work wrote.  Returns the launch status.
+template <typename... KArgs, typename... Args>
+inline moe_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                             Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e != cudaSuccess) {
+    set_cuda_error(e);
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
 
 // Device error word (one per device, cleared by moe_device_error).
 enum : int {
@@ -73,6 +99,12 @@ __host__ __device__ inline void w4_block_pos(int r, int c, int *lane, int *word,
 
 // ---------------------------------------------------------------- device side
 #ifdef __CUDACC__
+
+// Programmatic dependent launch: wait until the previous kernel on the
+// stream has completed and its writes are visible; let the next kernel on the
+// stream begin launching (it still waits for this one before reading).
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

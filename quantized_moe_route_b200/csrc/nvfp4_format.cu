@@ -129,6 +129,7 @@ __global__ void quantize_rows_kernel(const void *__restrict__ xv, int R, int K,
                                      float *__restrict__ Gout) {
   const int p = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
+  grid_dep_wait();
   if (p >= R) return;
   const int src = rows ? rows[p] / div : p;
   const int nb = K / 16;
@@ -177,6 +178,7 @@ __global__ void quantize_rows_kernel(const void *__restrict__ xv, int R, int K,
     for (int i = 0; i < 8; ++i) w[i / 4] |= (uint32_t)(c[2 * i] | (c[2 * i + 1] << 4)) << (8 * (i % 4));
     *reinterpret_cast<uint2 *>(codes + (size_t)p * (K / 2) + 8 * blk) = make_uint2(w[0], w[1]);
   }
+  grid_dep_trigger();
 }
 
 static moe_status nvfp4_check_shape(int N, int K, int kind) {
@@ -270,11 +272,6 @@ extern "C" MOE_API moe_status moe_quantize_nvfp4_rows(const void *x, int x_dtype
     return MOE_ERR_INVALID_ARG;
   const int warps = 8;
   const unsigned grid = (unsigned)((rows + warps - 1) / warps);
-  if (x_dtype == 0)
-    quantize_rows_kernel<false><<<grid, 32 * warps, 0, as_stream(stream)>>>(x, rows, K, src_rows,
-                                                                          src_div, codes, sf, G);
-  else
-    quantize_rows_kernel<true><<<grid, 32 * warps, 0, as_stream(stream)>>>(x, rows, K, src_rows,
-                                                                         src_div, codes, sf, G);
-  return launch_status();
+  return launch_pdl(x_dtype == 0 ? quantize_rows_kernel<false> : quantize_rows_kernel<true>, dim3(grid),
+                    dim3(32 * warps), 0, as_stream(stream), x, rows, K, src_rows, src_div, codes, sf, G);
 }

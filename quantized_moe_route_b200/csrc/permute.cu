@@ -18,6 +18,7 @@ constexpr int kPermChunk = 256;  // rows per chunk (one block each)
 
 __global__ void perm_hist_kernel(const int32_t *__restrict__ idx, int R, int E,
                                  int32_t *__restrict__ hist) {
+  grid_dep_wait();
   extern __shared__ int32_t sh[];
   for (int e = threadIdx.x; e < E; e += blockDim.x) sh[e] = 0;
   __syncthreads();
@@ -26,6 +27,7 @@ __global__ void perm_hist_kernel(const int32_t *__restrict__ idx, int R, int E,
     if ((unsigned)idx[r] < (unsigned)E) atomicAdd(&sh[idx[r]], 1);  // ids outside [0, E) are skipped
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(size_t)blockIdx.x * E + e] = sh[e];
+  grid_dep_trigger();
 }
 
 // One block of 1024 threads.  Each expert's chunks are split among S
@@ -35,6 +37,7 @@ __global__ void perm_hist_kernel(const int32_t *__restrict__ idx, int R, int E,
 __global__ void perm_scan_kernel(const int32_t *__restrict__ hist, int nchunks, int E, int S,
                                  int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
                                  int32_t *__restrict__ base) {
+  grid_dep_wait();
   extern __shared__ int32_t sh[];  // [E] totals then scanned
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int per = (nchunks + S - 1) / S;  // chunks of one thread
@@ -111,12 +114,14 @@ __global__ void perm_scan_kernel(const int32_t *__restrict__ hist, int nchunks, 
       }
     }
   }
+  grid_dep_trigger();
 }
 
 // One warp assigns positions to the chunk's rows 32 at a time, in row order.
 __global__ void perm_scatter_kernel(const int32_t *__restrict__ idx, int R, int E,
                                     const int32_t *__restrict__ base,
                                     int32_t *__restrict__ sorted_rows, int32_t *__restrict__ inv) {
+  grid_dep_wait();
   extern __shared__ int32_t run[];  // [E] running position per expert
   const int r0 = blockIdx.x * kPermChunk;
   const int nrows = min(R - r0, kPermChunk);
@@ -124,9 +129,18 @@ __global__ void perm_scatter_kernel(const int32_t *__restrict__ idx, int R, int 
   __syncthreads();
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
-    for (int i0 = 0; i0 < nrows; i0 += 32) {
+    int ids[kPermChunk / 32];  // the chunk's expert ids, all loads issued up front
+#pragma unroll
+    for (int s8 = 0; s8 < kPermChunk / 32; ++s8) {
+      const int i = 32 * s8 + lane;
+      ids[s8] = i < nrows ? idx[r0 + i] : -1;
+    }
+#pragma unroll
+    for (int s8 = 0; s8 < kPermChunk / 32; ++s8) {
+      const int i0 = 32 * s8;
+      if (i0 >= nrows) break;
       const int i = i0 + lane;
-      const int ei = i < nrows ? idx[r0 + i] : -1;
+      const int ei = ids[s8];
       const bool valid = (unsigned)ei < (unsigned)E;  // ids outside [0, E) are skipped
       const int e = valid ? ei : -1 - lane;           // invalid lanes never match
       const uint32_t active = __ballot_sync(0xffffffffu, valid);
@@ -142,6 +156,7 @@ __global__ void perm_scatter_kernel(const int32_t *__restrict__ idx, int R, int 
       __syncwarp();
     }
   }
+  grid_dep_trigger();
 }
 
 // x_perm[p] = x[sorted_rows[p] / k] for the offsets[E] grouped rows: warp w
@@ -151,6 +166,7 @@ __global__ void perm_gather_kernel(const int32_t *__restrict__ sorted_rows,
                                    const int32_t *__restrict__ offsets, int E, int k,
                                    const uint16_t *__restrict__ x, int H,
                                    uint16_t *__restrict__ x_perm) {
+  grid_dep_wait();
   const int lane = threadIdx.x & 31;
   const int nwarps = (int)(gridDim.x * blockDim.x) >> 5;
   const int total = offsets[E];
@@ -172,6 +188,7 @@ __global__ void perm_gather_kernel(const int32_t *__restrict__ sorted_rows,
       }
     }
   }
+  grid_dep_trigger();
 }
 
 }  // namespace moe
@@ -215,21 +232,19 @@ extern "C" MOE_API moe_status moe_permute(const int32_t *idx, int T, int k, int 
   int32_t *hist = static_cast<int32_t *>(ws);
   int32_t *base = hist + (size_t)nch * E;
   const size_t shE = sizeof(int32_t) * (size_t)E;
-  perm_hist_kernel<<<nch, 256, shE, s>>>(idx, R, E, hist);
-  moe_status st = launch_status();
+  moe_status st = launch_pdl(perm_hist_kernel, dim3(nch), dim3(256), shE, s, idx, R, E, hist);
   if (st != MOE_OK) return st;
   int S = 1;  // threads per expert in the scan: a power of two, S * E <= 1024, S <= 32
   while (S < 32 && 2 * S * E <= 1024 && S < nch) S *= 2;
-  perm_scan_kernel<<<1, 1024, shE, s>>>(hist, nch, E, S, counts, offsets, base);
-  st = launch_status();
+  st = launch_pdl(perm_scan_kernel, dim3(1), dim3(1024), shE, s, hist, nch, E, S, counts, offsets, base);
   if (st != MOE_OK) return st;
-  perm_scatter_kernel<<<nch, 256, shE, s>>>(idx, R, E, base, sorted_rows, inv);
-  st = launch_status();
+  st = launch_pdl(perm_scatter_kernel, dim3(nch), dim3(256), shE, s, idx, R, E, (const int32_t *)base,
+                  sorted_rows, inv);
   if (st != MOE_OK || !gather) return st;
   int dev = 0, nsm = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   const int blocks = (int)std::min<long long>((R + 7) / 8, 8LL * nsm);  // 8 warps per block
-  perm_gather_kernel<<<blocks, 256, 0, s>>>(sorted_rows, offsets, E, k, x, H, x_perm);
-  return launch_status();
+  return launch_pdl(perm_gather_kernel, dim3(blocks), dim3(256), 0, s, (const int32_t *)sorted_rows,
+                    (const int32_t *)offsets, E, k, x, H, x_perm);
 }

@@ -14,6 +14,7 @@ __global__ void route_kernel(const float *__restrict__ logits, int T, int E, int
                              int32_t *__restrict__ idx, float *__restrict__ w) {
   const int warps = blockDim.x / 32;
   const int t = blockIdx.x * warps + threadIdx.x / 32;
+  grid_dep_wait();
   if (t >= T) return;
   const int lane = threadIdx.x & 31;
   int my_idx;
@@ -23,6 +24,7 @@ __global__ void route_kernel(const float *__restrict__ logits, int T, int E, int
     idx[(size_t)t * k + lane] = my_idx;
     w[(size_t)t * k + lane] = my_w;
   }
+  grid_dep_trigger();
 }
 
 }  // namespace moe
@@ -39,11 +41,7 @@ extern "C" MOE_API moe_status moe_route(const float *logits, int T, int E, int k
   const dim3 grid((T + warps - 1) / warps);
   cudaStream_t s = as_stream(stream);
   const int per = (E + 31) / 32;
-  if (per <= 1) route_kernel<1><<<grid, threads, 0, s>>>(logits, T, E, k, idx, w);
-  else if (per <= 2) route_kernel<2><<<grid, threads, 0, s>>>(logits, T, E, k, idx, w);
-  else if (per <= 4) route_kernel<4><<<grid, threads, 0, s>>>(logits, T, E, k, idx, w);
-  else if (per <= 8) route_kernel<8><<<grid, threads, 0, s>>>(logits, T, E, k, idx, w);
-  else if (per <= 16) route_kernel<16><<<grid, threads, 0, s>>>(logits, T, E, k, idx, w);
-  else route_kernel<32><<<grid, threads, 0, s>>>(logits, T, E, k, idx, w);
-  return launch_status();
+  auto kern = per <= 1 ? route_kernel<1> : per <= 2 ? route_kernel<2> : per <= 4 ? route_kernel<4>
+             : per <= 8 ? route_kernel<8> : per <= 16 ? route_kernel<16> : route_kernel<32>;
+  return launch_pdl(kern, grid, dim3(threads), 0, s, logits, T, E, k, idx, w);
 }
