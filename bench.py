@@ -45,8 +45,11 @@ DTYPE_W4 = "int4 weights (f16 scale/min), bf16 activations, fp32 accumulate"
 # dram__bytes_read.sum + dram__bytes_write.sum of one decode launch at 1 token,
 # from the ncu captures summarised in profiles/ (taken on the current kernels;
 # set to None whenever the kernel changes)
-DECODE_TRAFFIC = {"w4": 14242560, "nvfp4": None}
+DECODE_TRAFFIC = {"w4": 14242560, "nvfp4": 14289152}
 DTYPE_NV = "nvfp4 weights and activations (e2m1 + e4m3/16 + fp32 global), fp32 accumulate"
+# the same for the prefill FFN kernels: both launches of one layer at the bench's
+# token count (the bench's first layer), from profiles/prefill_*.md
+PREFILL_TRAFFIC = {"w4": 285511168, "nvfp4": 139914752}
 
 
 # ---------------------------------------------------------------------------- helpers
@@ -521,12 +524,14 @@ def run_gpu_prefill(args, log):
                    "l2": "inputs larger than L2 (453 MB of experts per layer, 67 MB permuted rows)",
                    "parallelism": f"replicas x{world}", "launch": "stream-ordered, PDL into the FFN kernels"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak, "traffic": PREFILL_TRAFFIC["w4"],
+                     "traffic_source": "ncu capture of the gate/up and down launches of one layer (2048 tokens): "
+                                       "profiles/prefill_kernel_grouped_2048tok.md",
                      "kernel": "moe::prefill_kernel (gate/up + down launches)", "peak_kind": peak_kind,
                      "alg_flop_per_launch_pair": flops, "avg_pair_us": dur_ms * 1e3},
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2 + T * E * 4,
                 "d2h_bytes_per_step": T * H * 2},
-        "gpu_launches": 7 * K,
+        "gpu_launches": 8 * K,  # route, histogram, scan, scatter, gather, gate/up, down, combine
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -665,7 +670,10 @@ def run_gpu_prefill_nvfp4(args, log):
                    "l2": f"inputs larger than L2 ({nl} layers x 453 MB of experts rotated)",
                    "parallelism": f"replicas x{world}", "launch": "stream-ordered, PDL into the FFN kernels"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak, "traffic": PREFILL_TRAFFIC["nvfp4"],
+                     "traffic_source": "ncu capture of the gate/up and down launches of one layer (512 tokens; "
+                                       "the h quantise launch between them is not included): "
+                                       "profiles/prefill_nvfp4_kernel_grouped_512tok.md",
                      "kernel": "moe::prefill_nvfp4_kernel (gate/up + h quantise + down launches)",
                      "peak_kind": peak_kind, "alg_bytes_per_call": alg_bytes, "avg_call_us": dur_ms * 1e3,
                      "tflops": flops / (dur_ms / 1e3) / 1e12},
