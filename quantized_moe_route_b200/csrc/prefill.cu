@@ -61,7 +61,8 @@ struct PfCfg {
   static constexpr uint32_t kEpiOff = kRawOff + kRawStages * kRawStride;
   static constexpr uint32_t kEpiBytes = kPfDqWarps * 16 * 32 * 2;  // per warp: 16 rows x 32 outputs, bf16
   static constexpr uint32_t kTailOff = kEpiOff + kEpiBytes;
-  static constexpr uint32_t kSmemBytes = kTailOff + 1024 /*align slack*/ + 4096;
+  // tail: barriers, TMEM address and flags, then two chunk tables of E + 1 ints (E <= 960)
+  static constexpr uint32_t kSmemBytes = kTailOff + 1024 /*align slack*/ + 8192;
   static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
@@ -79,27 +80,42 @@ struct PrefillArgs {
 };
 
 // ---------------------------------------------------------------- tiles
-// Tile t of a CTA: row chunk t / n_sub (chunks of kPfBN rows, expert after
-// expert), weight tile t % n_sub.  chunk_start[e] = first chunk of expert e.
+// Row chunks of kPfBN rows, expert by expert.  A chunk of more than 128
+// rows is "heavy" (two MMAs per k16 step), one of at most 128 rows "light"
+// (one transposed MMA): an expert has n / 256 full chunks, plus a heavy or
+// a light partial chunk.  Tiles are numbered heavy chunks first, then light
+// ones, each chunk's n_sub weight tiles consecutive; heavy_start[e] /
+// light_start[e] = first heavy / light chunk of expert e (exclusive scans).
 struct TileInfo {
   int e, row0, nvalid, sub;
 };
-__device__ __forceinline__ TileInfo tile_info(int t, int n_sub, const int *chunk_start, int E,
-                                              const int32_t *offsets) {
-  const int chunk = t / n_sub;
-  int lo = 0, hi = E - 1;  // last expert with chunk_start[e] <= chunk
+__device__ __forceinline__ int last_at_or_below(const int *start, int E, int c) {
+  int lo = 0, hi = E - 1;  // last expert with start[e] <= c
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (chunk_start[mid] <= chunk) lo = mid;
+    if (start[mid] <= c) lo = mid;
     else hi = mid - 1;
   }
+  return lo;
+}
+__device__ __forceinline__ TileInfo tile_info(int t, int n_sub, const int *heavy_start,
+                                              const int *light_start, int E, const int32_t *offsets) {
+  const int chunk = t / n_sub, nheavy = heavy_start[E];
   TileInfo ti;
-  ti.e = lo;
-  ti.row0 = offsets[lo] + (chunk - chunk_start[lo]) * kPfBN;
-  ti.nvalid = min(kPfBN, offsets[lo + 1] - ti.row0);
+  if (chunk < nheavy) {
+    ti.e = last_at_or_below(heavy_start, E, chunk);
+    ti.row0 = offsets[ti.e] + (chunk - heavy_start[ti.e]) * kPfBN;
+  } else {
+    ti.e = last_at_or_below(light_start, E, chunk - nheavy);
+    ti.row0 = offsets[ti.e] + (offsets[ti.e + 1] - offsets[ti.e]) / kPfBN * kPfBN;  // the partial chunk
+  }
+  ti.nvalid = min(kPfBN, offsets[ti.e + 1] - ti.row0);
   ti.sub = t % n_sub;
   return ti;
 }
+// The i-th tile of CTA b: passes of G tiles, alternately in and against CTA
+// order, so the heavy tiles at the front spread evenly over the CTAs.
+__device__ __forceinline__ int cta_tile(int i, int b, int G) { return i * G + ((i & 1) ? G - 1 - b : b); }
 
 template <bool kGU>
 __global__ void __launch_bounds__(kPfThreads, 1)
@@ -120,7 +136,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(tmem_empty + 1);
   volatile int *abort_s = reinterpret_cast<volatile int *>(tmem_base_s + 1);
   int *ntiles_s = const_cast<int *>(abort_s) + 1;
-  int *chunk_start = ntiles_s + 1;  // [E + 1]
+  int *heavy_start = ntiles_s + 1;   // [E + 1]
+  int *light_start = heavy_start + (a.E + 1);  // [E + 1]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int KB = a.K / kPfBK;
@@ -145,25 +162,34 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   }
   if (warp == 1) tmem_alloc(tmem_base_s, C::kTmemCols);
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  // chunk table: chunk_start[e] = sum over e' < e of ceil(rows(e') / BN)
+  // chunk tables: exclusive scans of each expert's heavy and light chunks
   if (warp == 0) {
-    int carry = 0;
+    int hcarry = 0, lcarry = 0;
     for (int e0 = 0; e0 < a.E; e0 += 32) {
       const int e = e0 + lane;
-      const int n = e < a.E ? a.offsets[e + 1] - a.offsets[e] : 0;
-      const int c = (max(n, 0) + kPfBN - 1) / kPfBN;
-      int incl = c;
+      const int n = e < a.E ? max(a.offsets[e + 1] - a.offsets[e], 0) : 0;
+      const int rem = n % kPfBN;
+      const int hc = n / kPfBN + (rem > kPfBM ? 1 : 0), lc = (rem > 0 && rem <= kPfBM) ? 1 : 0;
+      int hi = hc, li = lc;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
+        const int hv = __shfl_up_sync(0xffffffffu, hi, o), lv = __shfl_up_sync(0xffffffffu, li, o);
+        if (lane >= o) {
+          hi += hv;
+          li += lv;
+        }
       }
-      if (e < a.E) chunk_start[e] = carry + incl - c;
-      carry += __shfl_sync(0xffffffffu, incl, 31);
+      if (e < a.E) {
+        heavy_start[e] = hcarry + hi - hc;
+        light_start[e] = lcarry + li - lc;
+      }
+      hcarry += __shfl_sync(0xffffffffu, hi, 31);
+      lcarry += __shfl_sync(0xffffffffu, li, 31);
     }
     if (lane == 0) {
-      chunk_start[a.E] = carry;
-      *ntiles_s = carry * a.n_sub;
+      heavy_start[a.E] = hcarry;
+      light_start[a.E] = lcarry;
+      *ntiles_s = (hcarry + lcarry) * a.n_sub;
     }
   }
   tc_fence_before();
@@ -181,8 +207,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // ------------------------------------------------------------ int4 producer
     if (lane == 0) {
       uint32_t it = 0;
-      for (int t = blockIdx.x; t < ntiles && !*abort_s; t += G) {
-        const TileInfo ti = tile_info(t, a.n_sub, chunk_start, a.E, a.offsets);
+      for (int i = 0, t = cta_tile(0, blockIdx.x, G); t < ntiles && !*abort_s; t = cta_tile(++i, blockIdx.x, G)) {
+        const TileInfo ti = tile_info(t, a.n_sub, heavy_start, light_start, a.E, a.offsets);
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % C::kRawStages;
           const uint32_t ph = (it / C::kRawStages) & 1u;
@@ -209,8 +235,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // ------------------------------------------------------------ activation producer
     if (lane == 0) {
       uint32_t it = 0;
-      for (int t = blockIdx.x; t < ntiles && !*abort_s; t += G) {
-        const TileInfo ti = tile_info(t, a.n_sub, chunk_start, a.E, a.offsets);
+      for (int i = 0, t = cta_tile(0, blockIdx.x, G); t < ntiles && !*abort_s; t = cta_tile(++i, blockIdx.x, G)) {
+        const TileInfo ti = tile_info(t, a.n_sub, heavy_start, light_start, a.E, a.offsets);
         const int nbox = (ti.nvalid + 63) / 64;  // whole 64-row boxes covering the valid rows
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % C::kBStages;
@@ -232,8 +258,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const uint64_t adesc0 = smem_desc_sw128(smem_u32(smem + C::kAOff));
       const uint64_t bdesc0 = smem_desc_sw128(smem_u32(smem + C::kBOff));
       uint32_t it = 0, tcount = 0;
-      for (int t = blockIdx.x; t < ntiles && !*abort_s; t += G, ++tcount) {
-        const TileInfo ti = tile_info(t, a.n_sub, chunk_start, a.E, a.offsets);
+      for (int i = 0, t = cta_tile(0, blockIdx.x, G); t < ntiles && !*abort_s;
+           t = cta_tile(++i, blockIdx.x, G), ++tcount) {
+        const TileInfo ti = tile_info(t, a.n_sub, heavy_start, light_start, a.E, a.offsets);
         // A tile of at most 128 rows is issued transposed (rows on M, the 256
         // weight rows on N): one MMA per k16 step instead of two.  An MMA
         // costs about as much at N = 16 as at N = 200, so this halves the
@@ -306,8 +333,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const uint32_t code_off = (uint32_t)(rbk * kBlkBytes + 16 * lane + 8 * wh);
     const uint32_t scale_off = (uint32_t)(rbk * kBlkBytes + kBlkCodeBytes + 4 * gi);
     uint32_t it = 0, tcount = 0;
-    for (int t = blockIdx.x; t < ntiles; t += G, ++tcount) {
-      const TileInfo ti = tile_info(t, a.n_sub, chunk_start, a.E, a.offsets);
+    for (int i = 0, t = cta_tile(0, blockIdx.x, G); t < ntiles; t = cta_tile(++i, blockIdx.x, G), ++tcount) {
+      const TileInfo ti = tile_info(t, a.n_sub, heavy_start, light_start, a.E, a.offsets);
       bool ok = true;
       for (int kb = 0; kb < KB; ++kb, ++it) {
         const int sr = it % C::kRawStages, sa = it % C::kAStages;
