@@ -6,10 +6,10 @@
 // routed experts", section "Quantization") both operands of every expert's
 // contraction are E2M1 codes with one E4M3 scale per 16 input channels, which
 // the sm_100 tensor cores consume as they are: no dequantisation anywhere.
-//   gate/up:  D_gate, D_up [128 features][N rows] = W [128][H] . X[N][H]^T,
+//   gate/up:  D_gate, D_up [128 features][N <= 64 rows] = W [128][H] . X[N][H]^T,
 //             epilogue g, u = D * G_x * G_w; h = SiLU(g) * u -> fp32 [rows][F]
 //   (h is re-quantised per row to NVFP4 between the two launches)
-//   down:     D [128 outputs][N rows] = W_down [128][F] . h[N][F]^T,
+//   down:     D [128 outputs][N <= 128 rows] = W_down [128][F] . h[N][F]^T,
 //             epilogue y = D * G_h * G_w -> bf16 y_perm [rows][H]
 // Per stage of 256 channels:
 //   warp 0      TMA: weight code tiles (the packed rows are stored with the
@@ -22,8 +22,9 @@
 //   warp 1      tcgen05.cp of the scales into tensor memory, then four
 //               block-scaled MMAs per matrix (K = 64 each), commit -> stage free
 //   warps 4..11 epilogue from tensor memory (tcgen05.ld), two warps per lane
-//               quarter; the down launch keeps two accumulator sets so its
-//               epilogue overlaps the next tile's MMAs
+//               quarter; both launches keep two accumulator sets (gate/up
+//               tiles of 64 rows, down tiles of 128) so the epilogue of one
+//               tile overlaps the next tile's MMAs
 // Every wait is bounded; a timeout raises the device error word.
 #include "common.cuh"
 #include "nvfp4.cuh"
@@ -32,7 +33,7 @@
 namespace moe {
 
 constexpr int kNpBM = 128;   // weight rows per matrix per tile (MMA M)
-constexpr int kNpBN = 128;   // rows (tokens) per tile; the MMA's N is trimmed to the valid rows
+constexpr int kNpBN = 128;   // most rows (tokens) a tile's activation buffers hold
 constexpr int kNpKT = 256;   // channels per stage: 128 code bytes per row
 constexpr int kNpBoxRows = 32;  // activation rows per TMA box (a tile loads the boxes it needs)
 constexpr int kNpEpiWarps = 8;  // warps 4..11: two per tensor-memory lane quarter
@@ -42,6 +43,11 @@ constexpr uint32_t kNpWaitPolls = 1u << 18;  // sleeping polls of up to 10 us: a
 template <bool kGU>
 struct NpCfg {
   static constexpr int kMats = kGU ? 2 : 1;
+  // rows per tile; the MMA's N is trimmed to the valid rows.  Gate/up tiles
+  // take 64 rows so that two accumulator sets fit in tensor memory beside
+  // the per-stage scales, and the epilogue of one tile overlaps the next
+  // tile's MMAs.
+  static constexpr int kBN = kGU ? 64 : 128;
   static constexpr int kStages = kGU ? 3 : 5;
   static constexpr uint32_t kACodes = kNpBM * 128;  // 16 KB per matrix
   static constexpr uint32_t kBCodes = kNpBN * 128;  // 16 KB
@@ -63,8 +69,8 @@ struct NpCfg {
   // two, so the epilogue of one tile overlaps the next tile's MMAs), then
   // per stage the scales: A (kMats x 4 blocks of 64 channels x 4 columns),
   // B (4 x 4 columns)
-  static constexpr int kAcc = kGU ? 1 : 2;
-  static constexpr uint32_t kAccCols = kMats * kNpBN;
+  static constexpr int kAcc = 2;
+  static constexpr uint32_t kAccCols = kMats * kBN;
   static constexpr uint32_t kSfCols = (kMats + 1) * 16;
   static constexpr uint32_t kTmemCols = 512;
   static_assert(kAcc * kAccCols + kStages * kSfCols <= kTmemCols, "tensor memory");
@@ -121,7 +127,7 @@ struct NpTile {
   int e, row0, nvalid, sub;
 };
 __device__ __forceinline__ NpTile np_tile(int t, int n_sub, const int *chunk_start, int E,
-                                          const int32_t *offsets) {
+                                          const int32_t *offsets, int bn) {
   const int chunk = t / n_sub;
   int lo = 0, hi = E - 1;  // last expert with chunk_start[e] <= chunk
   while (lo < hi) {
@@ -131,8 +137,8 @@ __device__ __forceinline__ NpTile np_tile(int t, int n_sub, const int *chunk_sta
   }
   NpTile ti;
   ti.e = lo;
-  ti.row0 = offsets[lo] + (chunk - chunk_start[lo]) * kNpBN;
-  ti.nvalid = min(kNpBN, offsets[lo + 1] - ti.row0);
+  ti.row0 = offsets[lo] + (chunk - chunk_start[lo]) * bn;
+  ti.nvalid = min(bn, offsets[lo + 1] - ti.row0);
   ti.sub = t % n_sub;
   return ti;
 }
@@ -181,7 +187,7 @@ __global__ void __launch_bounds__(kNpThreads, 1)
     for (int e0 = 0; e0 < a.E; e0 += 32) {
       const int e = e0 + lane;
       const int n = e < a.E ? a.offsets[e + 1] - a.offsets[e] : 0;
-      const int c = (max(n, 0) + kNpBN - 1) / kNpBN;
+      const int c = (max(n, 0) + C::kBN - 1) / C::kBN;
       int incl = c;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -212,7 +218,7 @@ __global__ void __launch_bounds__(kNpThreads, 1)
     if (lane == 0) {
       uint32_t it = 0;
       for (int t = blockIdx.x; t < ntiles && !*abort_s; t += G) {
-        const NpTile ti = np_tile(t, a.n_sub, chunk_start, a.E, a.offsets);
+        const NpTile ti = np_tile(t, a.n_sub, chunk_start, a.E, a.offsets, C::kBN);
         const int strip0 = ti.e * a.spe + 8 * ti.sub;  // first strip (pair) of the weight tile
         for (int kt = 0; kt < KT; ++kt, ++it) {
           const int s = it % C::kStages;
@@ -292,7 +298,7 @@ __global__ void __launch_bounds__(kNpThreads, 1)
       const uint64_t dsw0 = smem_desc_sw128(smem_u32(smem)), dpl0 = smem_desc_plain(smem_u32(smem));
       uint32_t it = 0, tcount = 0;
       for (int t = blockIdx.x; t < ntiles && !*abort_s; t += G, ++tcount) {
-        const NpTile ti = np_tile(t, a.n_sub, chunk_start, a.E, a.offsets);
+        const NpTile ti = np_tile(t, a.n_sub, chunk_start, a.E, a.offsets, C::kBN);
         const uint32_t idesc = idesc_nvf4((ti.nvalid + 15) & ~15);
         const int ab = tcount % C::kAcc;
         const uint32_t acc0 = tmem_base + ab * C::kAccCols;
@@ -327,7 +333,7 @@ __global__ void __launch_bounds__(kNpThreads, 1)
           for (int m = 0; m < C::kMats; ++m)
 #pragma unroll
             for (int kb = 0; kb < 4; ++kb)
-              tc_mma_nvf4(acc0 + m * kNpBN, sw + ((C::kOffA + m * C::kACodes + kb * 32) >> 4),
+              tc_mma_nvf4(acc0 + m * C::kBN, sw + ((C::kOffA + m * C::kACodes + kb * 32) >> 4),
                           sw + ((C::kOffB + kb * 32) >> 4), idesc, sf0 + m * 16 + kb * 4,
                           sf0 + C::kMats * 16 + kb * 4, (kt | kb) ? 1u : 0u);
           tc_commit(&empty[s]);  // stage (and its tensor-memory scales) free once these MMAs are done
@@ -342,7 +348,7 @@ __global__ void __launch_bounds__(kNpThreads, 1)
     const int half = (warp - 4) >> 2;  // the two warps of a quarter take alternate 16-column chunks
     uint32_t tcount = 0;
     for (int t = blockIdx.x; t < ntiles; t += G, ++tcount) {
-      const NpTile ti = np_tile(t, a.n_sub, chunk_start, a.E, a.offsets);
+      const NpTile ti = np_tile(t, a.n_sub, chunk_start, a.E, a.offsets, C::kBN);
       const int ab = tcount % C::kAcc;
       if (!mbar_wait_sleep(&tmem_full[ab], (tcount / C::kAcc) & 1u, kNpWaitPolls) || *abort_s) {
         if (lane == 0 && !*abort_s) fail();
@@ -355,7 +361,7 @@ __global__ void __launch_bounds__(kNpThreads, 1)
       for (int c0 = 16 * half; c0 < ti.nvalid; c0 += 32) {
         uint32_t v0[16], v1[16];
         tmem_ld16_async(trow + c0, v0);
-        if (kGU) tmem_ld16_async(trow + kNpBN + c0, v1);
+        if (kGU) tmem_ld16_async(trow + C::kBN + c0, v1);
         // the 16 rows' activation globals: one load per lane, then broadcast
         const float gl = lane < 16 && c0 + lane < ti.nvalid ? __fmul_rn(a.act_G[ti.row0 + c0 + lane], wG) : 0.f;
         tmem_ld_wait();
