@@ -33,7 +33,6 @@
 namespace moe {
 
 constexpr int kNpBM = 128;   // weight rows per matrix per tile (MMA M)
-constexpr int kNpBN = 128;   // most rows (tokens) a tile's activation buffers hold
 constexpr int kNpKT = 256;   // channels per stage: 128 code bytes per row
 constexpr int kNpBoxRows = 32;  // activation rows per TMA box (a tile loads the boxes it needs)
 constexpr int kNpEpiWarps = 8;  // warps 4..11: two per tensor-memory lane quarter
@@ -48,11 +47,13 @@ struct NpCfg {
   // the per-stage scales, and the epilogue of one tile overlaps the next
   // tile's MMAs.
   static constexpr int kBN = kGU ? 64 : 128;
-  static constexpr int kStages = kGU ? 3 : 5;
+  static constexpr int kStages = kGU ? 4 : 5;
   static constexpr uint32_t kACodes = kNpBM * 128;  // 16 KB per matrix
-  static constexpr uint32_t kBCodes = kNpBN * 128;  // 16 KB
+  static constexpr uint32_t kBCodes = kBN * 128;    // 8 or 16 KB
   static constexpr uint32_t kARaw = 8 * 256;        // 8 strips x (4 x 64 scale bytes)
-  static constexpr uint32_t kBRaw = kNpBN * 16;     // [rows][16 scale bytes]
+  // [rows][16 scale bytes]; the rearrangement reads 128 rows, past the end
+  // of a 64-row buffer into the stage's own atom area (rows it never uses)
+  static constexpr uint32_t kBRaw = kBN * 16;
   static constexpr uint32_t kAtom = 512;            // 128 rows x 4 scales, tensor-memory order
   static constexpr uint32_t kOffA = 0;
   static constexpr uint32_t kOffB = kOffA + kMats * kACodes;
