@@ -351,6 +351,15 @@ __global__ void __launch_bounds__(kNpThreads, 1)
     for (int t = blockIdx.x; t < ntiles; t += G, ++tcount) {
       const NpTile ti = np_tile(t, a.n_sub, chunk_start, a.E, a.offsets, C::kBN);
       const int ab = tcount % C::kAcc;
+      // the tile's activation globals times the expert's weight global,
+      // loaded while the MMAs run: lane l holds rows l, l + 32, ...
+      const float wG = a.w_G[ti.e];
+      float gl[C::kBN / 32];
+#pragma unroll
+      for (int i = 0; i < C::kBN / 32; ++i) {
+        const int r = 32 * i + lane;
+        gl[i] = r < ti.nvalid ? __fmul_rn(a.act_G[ti.row0 + r], wG) : 0.f;
+      }
       if (!mbar_wait_sleep(&tmem_full[ab], (tcount / C::kAcc) & 1u, kNpWaitPolls) || *abort_s) {
         if (lane == 0 && !*abort_s) fail();
         break;
@@ -358,19 +367,19 @@ __global__ void __launch_bounds__(kNpThreads, 1)
       tc_fence_after();
       const int wrow = ti.sub * kNpBM + q * 32 + lane;  // feature (gate/up) or output channel (down)
       const uint32_t trow = tmem_base + ab * C::kAccCols + ((uint32_t)(q * 32) << 16);
-      const float wG = a.w_G[ti.e];
-      for (int c0 = 16 * half; c0 < ti.nvalid; c0 += 32) {
+#pragma unroll
+      for (int i = 0; i < C::kBN / 32; ++i) {
+        const int c0 = 32 * i + 16 * half;  // rows c0 .. c0 + 15
+        if (c0 >= ti.nvalid) break;
         uint32_t v0[16], v1[16];
         tmem_ld16_async(trow + c0, v0);
         if (kGU) tmem_ld16_async(trow + C::kBN + c0, v1);
-        // the 16 rows' activation globals: one load per lane, then broadcast
-        const float gl = lane < 16 && c0 + lane < ti.nvalid ? __fmul_rn(a.act_G[ti.row0 + c0 + lane], wG) : 0.f;
         tmem_ld_wait();
         tmem_regs_after_wait(v0);
         if (kGU) tmem_regs_after_wait(v1);
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          const float gs = __shfl_sync(0xffffffffu, gl, c);
+          const float gs = __shfl_sync(0xffffffffu, gl[i], 16 * half + c);
           if (c0 + c < ti.nvalid) {
             const int p = ti.row0 + c0 + c;
             if (kGU) {
