@@ -76,6 +76,20 @@ def test_prefill_ragged_single_rows():
     _check(3, 32, 256, 128, 7, 3)
 
 
+def test_prefill_chunk_boundaries():
+    """Experts whose row counts sit on either side of the 128-row (one or two
+    MMAs per k step) and 256-row (chunk) boundaries, in one batch: the tile
+    schedule numbers the chunks of more than 128 rows first."""
+    counts = [0, 1, 127, 128, 129, 255, 256, 257, 384, 385, 513, 16]
+    E, k = len(counts), 1
+    owner = np.repeat(np.arange(E), counts)
+    owner = owner[np.random.default_rng(5).permutation(owner.size)]  # rows of an expert interleaved
+    logits = synth.router_logits(5, 0, owner.size, E)
+    logits[np.arange(owner.size), owner] += 100.0
+    offsets = _check(5, E, 256, 128, owner.size, k, logits=logits.astype(np.float32))
+    assert np.array_equal(np.diff(offsets), counts)
+
+
 def test_prefill_full_shape_sampled_tokens():
     """2048 tokens, 256 experts (Zipf-skewed), top-8, hidden 2048, width 512:
     every routing/permutation output exact, 64 sampled tokens against the oracle."""

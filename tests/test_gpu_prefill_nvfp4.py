@@ -104,6 +104,19 @@ def test_nvfp4_prefill_ragged_rows():
     _check(12, 32, 256, 512, 7, 3)
 
 
+def test_nvfp4_prefill_tile_boundaries():
+    """Experts whose row counts sit on either side of the 64-row gate/up and
+    128-row down tile sizes, in one batch."""
+    counts = [0, 1, 63, 64, 65, 127, 128, 129, 200, 3]
+    E, k = len(counts), 1
+    owner = np.repeat(np.arange(E), counts)
+    owner = owner[np.random.default_rng(6).permutation(owner.size)]
+    logits = synth.router_logits(6, 0, owner.size, E)
+    logits[np.arange(owner.size), owner] += 100.0
+    g = _check(6, E, 256, 256, owner.size, k, logits=logits.astype(np.float32))
+    assert np.array_equal(np.diff(g["offsets"]), counts)
+
+
 def test_nvfp4_prefill_one_expert_all_rows():
     T, E, k = 300, 8, 1
     logits = synth.router_logits(13, 0, T, E)
