@@ -239,6 +239,71 @@ def layer_inputs(seed, l, T):
     return x, logits
 
 
+def pipelined_e2e(torch, dev, stream, run_step, host_in, T, H, E, K, W, nl):
+    """End-to-end time (ms) of K stream-ordered steps through the C ABI
+    with host buffers.  Every step copies its inputs (x then the logits, one
+    pinned buffer per layer) host -> device and its result y device -> host.
+    The copies run on two copy streams beside the neighbouring steps' kernels;
+    device inputs and outputs are double-buffered, and the kernels stay in
+    order on `stream`.  Returns the H2D bytes per step too."""
+    xb = T * H * 2
+    nbytes = host_in[0].numel()
+    dxl = [torch.empty(nbytes, dtype=torch.uint8, device=dev) for _ in range(2)]
+    dx = [b[:xb].view(torch.int16).view(T, H) for b in dxl]
+    dl = [b[xb:].view(torch.float32).view(T, E) for b in dxl]
+    dy = [torch.empty((T, H), dtype=torch.int16, device=dev) for _ in range(2)]
+    hy = [torch.empty((T, H), dtype=torch.int16).pin_memory() for _ in range(2)]
+    cs, ds = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_k = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def steps(n, first):
+        cs.wait_stream(stream)
+        ds.wait_stream(stream)
+        for i in range(n):
+            l, b = (first + i) % nl, i % 2
+            if i >= 2:
+                cs.wait_event(ev_k[b])  # the step that read this input buffer is done
+            with torch.cuda.stream(cs):
+                dxl[b].copy_(host_in[l], non_blocking=True)
+                ev_in[b].record(cs)
+            stream.wait_event(ev_in[b])
+            if i >= 2:
+                stream.wait_event(ev_out[b])  # this output buffer's last result has been read
+            with torch.cuda.stream(stream):
+                run_step(l, dx[b], dl[b], dy[b])
+            ev_k[b].record(stream)
+            ds.wait_event(ev_k[b])
+            with torch.cuda.stream(ds):
+                hy[b].copy_(dy[b], non_blocking=True)
+                ev_out[b].record(ds)
+        stream.wait_stream(cs)
+        stream.wait_stream(ds)
+
+    steps(2, 0)
+    torch.cuda.synchronize()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    steps(K, W)
+    a1.record(stream)
+    a1.synchronize()
+    return a0.elapsed_time(a1), nbytes
+
+
+def pinned_inputs(torch, x_list, lg_list):
+    """One pinned host buffer per layer: the bf16 activations, then the fp32 logits."""
+    out = []
+    for x, lg in zip(x_list, lg_list):
+        xb = np.ascontiguousarray(x).view(np.uint8).reshape(-1)
+        lb = np.ascontiguousarray(lg, dtype=np.float32).view(np.uint8).reshape(-1)
+        buf = torch.empty(xb.size + lb.size, dtype=torch.uint8).pin_memory()
+        buf[:xb.size].copy_(torch.from_numpy(xb))
+        buf[xb.size:].copy_(torch.from_numpy(lb))
+        out.append(buf)
+    return out
+
+
 def run_gpu(args, log):
     global LAYERS
     LAYERS = args.layers
@@ -341,25 +406,66 @@ def run_gpu(args, log):
     peak, peak_kind = peaks()
     achieved = alg_bytes / (dur_ms / 1e3) / 1e9
 
-    # end to end through the C ABI with host buffers: H2D of the step's inputs
-    # from pinned memory and D2H of its result, every step
-    hx = [torch.from_numpy(layer_inputs(seed, l, T)[0].view(np.int16)).pin_memory() for l in range(LAYERS)]
-    hl = [torch.from_numpy(layer_inputs(seed, l, T)[1]).pin_memory() for l in range(LAYERS)]
-    hy = torch.empty((T, H), dtype=torch.int16).pin_memory()
-    dx = torch.empty((T, H), dtype=torch.int16, device=dev)
-    dl = torch.empty((T, E), dtype=torch.float32, device=dev)
+    # end to end through the C ABI with host buffers: every step copies its
+    # inputs (x and the logits, one pinned buffer) host -> device and its
+    # result y device -> host.  The copies run on two copy streams and
+    # overlap the neighbouring steps' kernels (double-buffered device inputs
+    # and outputs); the kernels stay in order on the decode stream.
+    xl_bytes = T * H * 2 + T * E * 4
+    hxl = []
+    for l in range(LAYERS):
+        x, lg = layer_inputs(seed, l, T)
+        buf = torch.empty(xl_bytes, dtype=torch.uint8).pin_memory()
+        buf[:T * H * 2].copy_(torch.from_numpy(x.view(np.uint8).reshape(-1)))
+        buf[T * H * 2:].copy_(torch.from_numpy(lg.view(np.uint8).reshape(-1)))
+        hxl.append(buf)
+    hy = [torch.empty((T, H), dtype=torch.int16).pin_memory() for _ in range(2)]
+    dxl = [torch.empty(xl_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
+    dx = [b[:T * H * 2].view(torch.int16).view(T, H) for b in dxl]
+    dl = [b[T * H * 2:].view(torch.float32).view(T, E) for b in dxl]
+    dy = [torch.empty((T, H), dtype=torch.int16, device=dev) for _ in range(2)]
+    cs, ds = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_k = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step(l):
-        dx.copy_(hx[l], non_blocking=True)
-        dl.copy_(hl[l], non_blocking=True)
-        decode_layer(layers[l][2], dx, dl, k, y, ws, stream=stream)
-        hy.copy_(y, non_blocking=True)
+    def e2e_steps(n, first):
+        cs.wait_stream(stream)
+        ds.wait_stream(stream)
+        for i in range(n):
+            l, b = (first + i) % LAYERS, i % 2
+            if i >= 2:
+                cs.wait_event(ev_k[b])  # the kernel that read this input buffer is done
+            with torch.cuda.stream(cs):
+                dxl[b].copy_(hxl[l], non_blocking=True)
+                ev_in[b].record(cs)
+            stream.wait_event(ev_in[b])
+            if i >= 2:
+                stream.wait_event(ev_out[b])  # this output buffer's last result has been read
+            decode_layer(layers[l][2], dx[b], dl[b], k, dy[b], ws, stream=stream)
+            ev_k[b].record(stream)
+            ds.wait_event(ev_k[b])
+            with torch.cuda.stream(ds):
+                hy[b].copy_(dy[b], non_blocking=True)
+                ev_out[b].record(ds)
+        stream.wait_stream(cs)
+        stream.wait_stream(ds)
+
+    def capture_e2e(n, first):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            e2e_steps(n, first)
+        return g
 
     with torch.cuda.stream(stream):
-        for l in range(3):
-            e2e_step(l % LAYERS)
+        e2e_steps(3, 0)
     stream.synchronize()
-    g_e2e = run_steps(e2e_step, K, W)
+    Ge = min(K, args.graph_steps)
+    g_e2e = []
+    if K // Ge:
+        g_e2e.append((capture_e2e(Ge, W), K // Ge))
+    if K % Ge:
+        g_e2e.append((capture_e2e(K % Ge, W + (K // Ge) * Ge), 1))
     replay(g_e2e)
     torch.cuda.synchronize()
     dist_barrier()
@@ -390,8 +496,9 @@ def run_gpu(args, log):
                      "kernel": f"moe::decode_kernel<{'nvfp4' if fmt == 'nvfp4' else 'int4'}, fused>",
                      "peak_kind": peak_kind, "alg_bytes_per_launch": alg_bytes,
                      "avg_launch_us": dur_ms * 1e3, "isolated_launch_us": isolated_ms * 1e3},
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2 + T * E * 4,
-                "d2h_bytes_per_step": T * H * 2},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": xl_bytes,
+                "d2h_bytes_per_step": T * H * 2,
+                "overlap": "each step's copies run on copy streams beside the neighbouring steps' kernels"},
         "gpu_launches": K,
         "clocks": clk.summary(),
     }
@@ -439,7 +546,7 @@ def run_gpu_prefill(args, log):
     y = torch.empty((T, H), dtype=torch.int16, device=dev)
     stream = torch.cuda.Stream(device=dev)
 
-    def step(l, ev=None, xin=None, lin=None):
+    def step(l, ev=None, xin=None, lin=None, yout=None):
         moe.moe_route(ls[l] if lin is None else lin, k, idx, w, stream=stream)
         moe.moe_permute(idx, E, counts, offsets, sorted_rows, inv, pws, x=xs[l] if xin is None else xin,
                         x_perm=x_perm, stream=stream)
@@ -448,7 +555,7 @@ def run_gpu_prefill(args, log):
         moe.moe_ffn_grouped_prefill(layers[l][2], x_perm, offsets, y_perm, fws, stream=stream)
         if ev is not None:
             ev[1].record(stream)
-        moe.moe_unpermute_combine(y_perm, w, y, inv=inv, stream=stream)
+        moe.moe_unpermute_combine(y_perm, w, y if yout is None else yout, inv=inv, stream=stream)
 
     K, W = args.steps, args.warmup
     with torch.cuda.stream(stream):
@@ -488,32 +595,15 @@ def run_gpu_prefill(args, log):
     except Exception:
         peak, peak_kind = 1400.0, "fallback (sustained bf16)"
 
-    # end to end: H2D of x and logits from pinned memory, D2H of y, every step
+    # end to end: each step copies x and the logits (one pinned buffer) in and
+    # y out, on copy streams beside the neighbouring steps' kernels
     import synth as _s
-    hx = [torch.from_numpy(_s.activations_bf16(seed, l, T, H).view(np.int16)).pin_memory() for l in range(nl)]
-    hl = [torch.from_numpy((_s.router_logits(seed, l, T, E) + bias[None, :]).astype(np.float32)).pin_memory()
-          for l in range(nl)]
-    hy = torch.empty((T, H), dtype=torch.int16).pin_memory()
-    dx = torch.empty((T, H), dtype=torch.int16, device=dev)
-    dl = torch.empty((T, E), dtype=torch.float32, device=dev)
-    with torch.cuda.stream(stream):
-        for i in range(2):
-            dx.copy_(hx[i % nl], non_blocking=True)
-            dl.copy_(hl[i % nl], non_blocking=True)
-            step(i % nl, xin=dx, lin=dl)
-            hy.copy_(y, non_blocking=True)
-    torch.cuda.synchronize()
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        a0.record(stream)
-        for i in range(K):
-            dx.copy_(hx[(W + i) % nl], non_blocking=True)
-            dl.copy_(hl[(W + i) % nl], non_blocking=True)
-            step((W + i) % nl, xin=dx, lin=dl)
-            hy.copy_(y, non_blocking=True)
-        a1.record(stream)
-    a1.synchronize()
-    e2e_ms = dist_max(a0.elapsed_time(a1))
+    host_in = pinned_inputs(torch, [_s.activations_bf16(seed, l, T, H) for l in range(nl)],
+                            [_s.router_logits(seed, l, T, E) + bias[None, :] for l in range(nl)])
+    e2e_ms, h2d_bytes = pipelined_e2e(torch, dev, stream,
+                                      lambda l, xin, lin, yout: step(l, xin=xin, lin=lin, yout=yout),
+                                      host_in, T, H, E, K, W, nl)
+    e2e_ms = dist_max(e2e_ms)
 
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
@@ -529,8 +619,9 @@ def run_gpu_prefill(args, log):
                                        "profiles/prefill_kernel_grouped_2048tok.md",
                      "kernel": "moe::prefill_kernel (gate/up + down launches)", "peak_kind": peak_kind,
                      "alg_flop_per_launch_pair": flops, "avg_pair_us": dur_ms * 1e3},
-        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2 + T * E * 4,
-                "d2h_bytes_per_step": T * H * 2},
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d_bytes,
+                "d2h_bytes_per_step": T * H * 2,
+                "overlap": "each step's copies run on copy streams beside the neighbouring steps' kernels"},
         "gpu_launches": 8 * K,  # route, histogram, scan, scatter, gather, gate/up, down, combine
         "clocks": clk.summary(),
     }
@@ -583,7 +674,7 @@ def run_gpu_prefill_nvfp4(args, log):
     y = torch.empty((T, H), dtype=torch.int16, device=dev)
     stream = torch.cuda.Stream(device=dev)
 
-    def step(l, ev=None, xin=None, lin=None):
+    def step(l, ev=None, xin=None, lin=None, yout=None):
         moe.moe_route(ls[l] if lin is None else lin, k, idx, w, stream=stream)
         moe.moe_permute(idx, E, counts, offsets, sorted_rows, inv, pws, stream=stream)
         moe.moe_quantize_nvfp4_rows(xs[l] if xin is None else xin, xc, xsf, xg, src_rows=sorted_rows, src_div=k,
@@ -593,7 +684,7 @@ def run_gpu_prefill_nvfp4(args, log):
         moe.moe_ffn_grouped_prefill_nvfp4(layers[l][2], xc, xsf, xg, offsets, y_perm, fws, stream=stream)
         if ev is not None:
             ev[1].record(stream)
-        moe.moe_unpermute_combine(y_perm, w, y, inv=inv, stream=stream)
+        moe.moe_unpermute_combine(y_perm, w, y if yout is None else yout, inv=inv, stream=stream)
 
     K, W = args.steps, args.warmup
     with torch.cuda.stream(stream):
@@ -635,31 +726,15 @@ def run_gpu_prefill_nvfp4(args, log):
     achieved = alg_bytes / (dur_ms / 1e3) / 1e9
     flops = R * 6.0 * H * F
 
+    # end to end: each step copies x and the logits (one pinned buffer) in and
+    # y out, on copy streams beside the neighbouring steps' kernels
     import synth as _s
-    hx = [torch.from_numpy(_s.activations_bf16(seed, l, T, H).view(np.int16)).pin_memory() for l in range(nl)]
-    hl = [torch.from_numpy((_s.router_logits(seed, l, T, E) + bias[None, :]).astype(np.float32)).pin_memory()
-          for l in range(nl)]
-    hy = torch.empty((T, H), dtype=torch.int16).pin_memory()
-    dx = torch.empty((T, H), dtype=torch.int16, device=dev)
-    dl = torch.empty((T, E), dtype=torch.float32, device=dev)
-    with torch.cuda.stream(stream):
-        for i in range(2):
-            dx.copy_(hx[i % nl], non_blocking=True)
-            dl.copy_(hl[i % nl], non_blocking=True)
-            step(i % nl, xin=dx, lin=dl)
-            hy.copy_(y, non_blocking=True)
-    torch.cuda.synchronize()
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        a0.record(stream)
-        for i in range(K):
-            dx.copy_(hx[(W + i) % nl], non_blocking=True)
-            dl.copy_(hl[(W + i) % nl], non_blocking=True)
-            step((W + i) % nl, xin=dx, lin=dl)
-            hy.copy_(y, non_blocking=True)
-        a1.record(stream)
-    a1.synchronize()
-    e2e_ms = dist_max(a0.elapsed_time(a1))
+    host_in = pinned_inputs(torch, [_s.activations_bf16(seed, l, T, H) for l in range(nl)],
+                            [_s.router_logits(seed, l, T, E) + bias[None, :] for l in range(nl)])
+    e2e_ms, h2d_bytes = pipelined_e2e(torch, dev, stream,
+                                      lambda l, xin, lin, yout: step(l, xin=xin, lin=lin, yout=yout),
+                                      host_in, T, H, E, K, W, nl)
+    e2e_ms = dist_max(e2e_ms)
 
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
@@ -677,8 +752,9 @@ def run_gpu_prefill_nvfp4(args, log):
                      "kernel": "moe::prefill_nvfp4_kernel (gate/up + h quantise + down launches)",
                      "peak_kind": peak_kind, "alg_bytes_per_call": alg_bytes, "avg_call_us": dur_ms * 1e3,
                      "tflops": flops / (dur_ms / 1e3) / 1e12},
-        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2 + T * E * 4,
-                "d2h_bytes_per_step": T * H * 2},
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d_bytes,
+                "d2h_bytes_per_step": T * H * 2,
+                "overlap": "each step's copies run on copy streams beside the neighbouring steps' kernels"},
         "gpu_launches": 9 * K,
         "clocks": clk.summary(),
     }
