@@ -338,7 +338,13 @@ __device__ __forceinline__ void mma_f16_16816(float d[4], const uint32_t a[4], u
 template <int SH>
 __device__ __forceinline__ uint32_t e2m1x2_f16(uint32_t w) {
   static_assert(SH == 0 || SH == 4, "nibble offset");
-  return ((w << (9 - SH)) & 0x0E000E00u) | ((w << (12 - SH)) & 0x80008000u);
+  // the two moves as one multiply-add (the fields are disjoint, so + is |),
+  // which runs on the FMA pipe beside the integer pipe's masks
+  uint32_t r;
+  asm("mad.lo.u32 %0, %1, %2, %3;"
+      : "=r"(r)
+      : "r"(w & (0x00080008u << SH)), "n"(1u << (12 - SH)), "r"((w << (9 - SH)) & 0x0E000E00u));
+  return r;
 }
 
 __device__ __forceinline__ void e4m3x4_to_f32(uint32_t w, float f[4]) {
