@@ -3,26 +3,30 @@
 // Prefill groups the rows of a batch by routed expert ("drama-rs", sections
 // "Apple Silicon (MLX)" and "Layout": prefill runs a grouped MoE); every
 // expert's rows then form a dense contraction with that expert's weights.
-// Two launches of one kernel template, each tile two 128-row MMA blocks that
-// share the activation tile:
-//   gate/up:  D_gate, D_up [128 features][BN rows] = W [128][H] . X[BN][H]^T,
-//             epilogue h = SiLU(D_gate) * D_up -> bf16 workspace [rows][F]
-//   down:     D_0, D_1 [2 x 128 outputs][BN rows] = W_down [256][F] . h[BN][F]^T
-//             epilogue -> y_perm bf16 [rows][H]
-// The weights are the MMA's A operand (M = 128 rows per block), the rows of
-// an expert its B operand (N = BN tokens), so a few-row expert wastes N, not
-// M.
+// Two launches of one kernel template.  A tile is a chunk of up to BN = 256
+// rows of one expert and two 128-row weight blocks that share its activation
+// tile (gate and up of 128 features, or 256 consecutive down outputs):
+//   gate/up:  h = SiLU(D_gate) * D_up -> bf16 workspace [rows][F]
+//   down:     -> y_perm bf16 [rows][H]
+// A chunk of more than 128 rows puts the weights on the MMA's M (128 rows
+// per block, one accumulator each) and the rows on N (trimmed to the valid
+// rows).  A chunk of at most 128 rows is issued transposed: rows on M, the
+// two contiguous weight blocks as one N = 256 operand, one MMA per k16 step.
+// An MMA of M = 128, K = 16 costs about the same for any N up to ~200, so
+// this halves the tensor time of few-row tiles.  Chunks of more than 128
+// rows are scheduled first, in passes over the CTAs that alternate direction.
 //
 // Per 64-channel k block (one quantisation group):
-//   producer warp:   one TMA box per matrix of packed int4 blocks (8 strips),
-//                    TMA (128-byte swizzle) of the activation tile
-//   dequant warps:   int4 -> bf16 (fp32 q*s+m with one rounding, then nearest
-//                    even) into the 128-byte-swizzled K-major smem layout the
-//                    MMA reads
+//   int4 producer:   one TMA box per matrix of packed int4 blocks (8 strips)
+//   act. producer:   TMA (128-byte swizzle) of the 64-row boxes holding rows
+//   dequant warps:   int4 -> bf16, one FMA per code (q s + m in fp32, then
+//                    nearest even) into the 128-byte-swizzled K-major smem
+//                    layout the MMA reads
 //   MMA thread:      tcgen05.mma kind::f16 (bf16 x bf16 -> fp32 in tensor
-//                    memory), four k16 steps per block, commit -> stage free
-// then the dequant warps run the epilogue from tensor memory (tcgen05.ld),
-// turning 32 outputs x 16 rows around in shared memory for 16-byte stores.
+//                    memory), commit -> stages free
+// then the dequant warps run the epilogue from tensor memory (tcgen05.ld):
+// rows on N turn 32 outputs x 16 rows around in shared memory for 16-byte
+// stores; rows on M write stretches of their own row.
 // Every wait is bounded; a timeout raises the device error word.
 #include "common.cuh"
 #include "tcgen05.cuh"
