@@ -13,7 +13,9 @@ pytestmark = pytest.mark.gpu
 
 
 def _prefill(layer, x, logits, k):
-    """Device pipeline; returns idx, inv, y_perm (bf16 bits), y (bf16 bits)."""
+    """Device pipeline; returns idx, inv, y_perm (bf16 bits), y (bf16 bits),
+    offsets, sorted_rows and the bf16 h rows the gate/up launch left at the
+    start of the workspace (permuted row order)."""
     T, H = x.shape
     E = logits.shape[1]
     idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
@@ -33,7 +35,9 @@ def _prefill(layer, x, logits, k):
     moe.moe_unpermute_combine(y_perm, w, y, inv=inv)
     torch.cuda.synchronize()
     assert moe.moe_device_error() == 0
-    return idx.cpu().numpy(), inv.cpu().numpy(), to_u16(y_perm), to_u16(y), offsets.cpu().numpy()
+    h = pws[:T * k * layer.F * 2].view(torch.int16).view(T * k, layer.F)
+    return (idx.cpu().numpy(), inv.cpu().numpy(), to_u16(y_perm), to_u16(y), offsets.cpu().numpy(),
+            sorted_rows.cpu().numpy(), to_u16(h))
 
 
 def _check(seed, E, H, F, T, k, bias=None, logits=None):
@@ -44,12 +48,23 @@ def _check(seed, E, H, F, T, k, bias=None, logits=None):
             logits = (logits + bias[None, :]).astype(np.float32)
     oidx, _ = oracle.route(logits, k)
     layer = Layer(seed, 0, E, H, F, oidx.ravel())
-    idx, inv, y_perm, y, offsets = _prefill(layer, x, logits, k)
+    idx, inv, y_perm, y, offsets, sorted_rows, h = _prefill(layer, x, logits, k)
     assert np.array_equal(idx, oidx)
     _, _, oy_rows, oy = oracle.moe_forward_w4(x, logits, k, layer.canon)
     got_rows = synth.bf16_bits_to_f32(y_perm[inv])  # back to row order r = t*k + j
     ffn_close(got_rows, oy_rows, "y_perm")
     ffn_close(synth.bf16_bits_to_f32(y), synth.bf16_bits_to_f32(oy), "y")
+    # stage-wise: the gate/up launch's h of sampled rows against the oracle's h
+    rng = np.random.default_rng(seed)
+    ps = rng.choice(T * k, min(16, T * k), replace=False)
+    got_h, want_h = [], []
+    for p in ps:
+        r = int(sorted_rows[p])
+        e = int(oidx[r // k, r % k])
+        _, h_o = oracle.expert_ffn_w4(x[r // k], *layer.canon[e], return_h=True)
+        got_h.append(synth.bf16_bits_to_f32(h[p]))
+        want_h.append(h_o)
+    ffn_close(np.array(got_h), np.array(want_h), "h (gate/up stage)")
     return offsets
 
 
@@ -120,7 +135,7 @@ def test_prefill_full_shape_sampled_tokens():
     layer = L()
     layer.F = F
     layer.desc = moe.make_layer(E, H, F, gu, dn)
-    idx, inv, y_perm, y, offsets = _prefill(layer, x, logits, k)
+    idx, inv, y_perm, y, offsets, sorted_rows, h = _prefill(layer, x, logits, k)
     assert np.array_equal(idx, oidx)
     counts = np.bincount(oidx.ravel(), minlength=E)
     assert np.array_equal(np.diff(offsets), counts)
@@ -129,13 +144,17 @@ def test_prefill_full_shape_sampled_tokens():
     need = sorted(set(oidx[toks].ravel().tolist()))
     experts = {e: (oracle.quantize_w4(synth.expert_weights(seed, 0, e, 0, 2 * F, H)),
                    oracle.quantize_w4(synth.expert_weights(seed, 0, e, 1, H, F))) for e in need}
-    got_rows, want_rows, got_y, want_y = [], [], [], []
+    got_rows, want_rows, got_y, want_y, got_h, want_h = [], [], [], [], [], []
     for t in toks:
-        Yt = [oracle.expert_ffn_w4(x[t], *experts[int(e)]) for e in oidx[t]]
+        Yh = [oracle.expert_ffn_w4(x[t], *experts[int(e)], return_h=True) for e in oidx[t]]
+        Yt = [yh[0] for yh in Yh]
+        want_h.append(np.stack([yh[1] for yh in Yh]))
+        got_h.append(synth.bf16_bits_to_f32(h[inv[t * k:(t + 1) * k]]))
         want_rows.append(np.stack(Yt))
         got_rows.append(synth.bf16_bits_to_f32(y_perm[inv[t * k:(t + 1) * k]]))
         want_y.append(synth.bf16_bits_to_f32(oracle.combine(np.stack(Yt), ow[t:t + 1])[0]))
         got_y.append(synth.bf16_bits_to_f32(y[t]))
+    ffn_close(np.stack(got_h), np.stack(want_h), "sampled h rows (gate/up stage)")
     ffn_close(np.stack(got_rows), np.stack(want_rows), "sampled y_perm rows")
     ffn_close(np.stack(got_y), np.stack(want_y), "sampled y")
 
