@@ -93,15 +93,6 @@ struct PrefillArgs {
 struct TileInfo {
   int e, row0, nvalid, sub;
 };
-__device__ __forceinline__ int last_at_or_below(const int *start, int E, int c) {
-  int lo = 0, hi = E - 1;  // last expert with start[e] <= c
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (start[mid] <= c) lo = mid;
-    else hi = mid - 1;
-  }
-  return lo;
-}
 __device__ __forceinline__ TileInfo tile_info(int t, int n_sub, const int *heavy_start,
                                               const int *light_start, int E, const int32_t *offsets) {
   const int chunk = t / n_sub, nheavy = heavy_start[E];
@@ -117,10 +108,6 @@ __device__ __forceinline__ TileInfo tile_info(int t, int n_sub, const int *heavy
   ti.sub = t % n_sub;
   return ti;
 }
-// The i-th tile of CTA b: passes of G tiles, alternately in and against CTA
-// order, so the heavy tiles at the front spread evenly over the CTAs.
-__device__ __forceinline__ int cta_tile(int i, int b, int G) { return i * G + ((i & 1) ? G - 1 - b : b); }
-
 template <bool kGU>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_kernel(PrefillArgs a, const __grid_constant__ CUtensorMap act_map,

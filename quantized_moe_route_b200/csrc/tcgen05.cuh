@@ -112,6 +112,21 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, i
       : "memory");
 }
 
+// Grouped-GEMM tile scheduling shared by the prefill kernels.
+// Last expert e with start[e] <= c (start: exclusive scan of per-expert chunk counts).
+__device__ __forceinline__ int last_at_or_below(const int *start, int E, int c) {
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (start[mid] <= c) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+// The i-th tile of CTA b: passes of G tiles, alternately in and against CTA
+// order, so the heavy tiles numbered first spread evenly over the CTAs.
+__device__ __forceinline__ int cta_tile(int i, int b, int G) { return i * G + ((i & 1) ? G - 1 - b : b); }
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
