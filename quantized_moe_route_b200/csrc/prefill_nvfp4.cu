@@ -6,7 +6,7 @@
 // routed experts", section "Quantization") both operands of every expert's
 // contraction are E2M1 codes with one E4M3 scale per 16 input channels, which
 // the sm_100 tensor cores consume as they are: no dequantisation anywhere.
-//   gate/up:  D_gate, D_up [128 features][N <= 64 rows] = W [128][H] . X[N][H]^T,
+//   gate/up:  D_gate, D_up [128 features][N <= 80 rows] = W [128][H] . X[N][H]^T,
 //             epilogue g, u = D * G_x * G_w; h = SiLU(g) * u -> fp32 [rows][F]
 //   (h is re-quantised per row to NVFP4 between the two launches)
 //   down:     D [128 outputs][N <= 128 rows] = W_down [128][F] . h[N][F]^T,
@@ -23,7 +23,7 @@
 //               block-scaled MMAs per matrix (K = 64 each), commit -> stage free
 //   warps 4..11 epilogue from tensor memory (tcgen05.ld), two warps per lane
 //               quarter; both launches keep two accumulator sets (gate/up
-//               tiles of 64 rows, down tiles of 128) so the epilogue of one
+//               tiles of 80 rows, down tiles of 128) so the epilogue of one
 //               tile overlaps the next tile's MMAs
 // Every wait is bounded; a timeout raises the device error word.
 #include "common.cuh"
@@ -43,17 +43,19 @@ template <bool kGU>
 struct NpCfg {
   static constexpr int kMats = kGU ? 2 : 1;
   // rows per tile; the MMA's N is trimmed to the valid rows.  Gate/up tiles
-  // take 64 rows so that two accumulator sets fit in tensor memory beside
-  // the per-stage scales, and the epilogue of one tile overlaps the next
-  // tile's MMAs.
-  static constexpr int kBN = kGU ? 64 : 128;
-  static constexpr int kStages = kGU ? 4 : 5;
+  // take 80 rows so that two accumulator sets fit in tensor memory beside
+  // the per-stage scales (the epilogue of one tile overlaps the next tile's
+  // MMAs) with few enough tiles that no CTA takes more than three at 512
+  // tokens.
+  static constexpr int kBN = kGU ? 80 : 128;
+  static constexpr int kBRows = (kBN + 31) / 32 * 32;  // rows of the activation buffers: whole 32-row boxes
+  static constexpr int kStages = kGU ? 3 : 5;
   static constexpr uint32_t kACodes = kNpBM * 128;  // 16 KB per matrix
-  static constexpr uint32_t kBCodes = kBN * 128;    // 8 or 16 KB
+  static constexpr uint32_t kBCodes = kBRows * 128;  // 12 or 16 KB
   static constexpr uint32_t kARaw = 8 * 256;        // 8 strips x (4 x 64 scale bytes)
   // [rows][16 scale bytes]; the rearrangement reads 128 rows, past the end
-  // of a 64-row buffer into the stage's own atom area (rows it never uses)
-  static constexpr uint32_t kBRaw = kBN * 16;
+  // of a shorter buffer into the stage's own atom area (rows it never uses)
+  static constexpr uint32_t kBRaw = kBRows * 16;
   static constexpr uint32_t kAtom = 512;            // 128 rows x 4 scales, tensor-memory order
   static constexpr uint32_t kOffA = 0;
   static constexpr uint32_t kOffB = kOffA + kMats * kACodes;
@@ -354,9 +356,9 @@ __global__ void __launch_bounds__(kNpThreads, 1)
       // the tile's activation globals times the expert's weight global,
       // loaded while the MMAs run: lane l holds rows l, l + 32, ...
       const float wG = a.w_G[ti.e];
-      float gl[C::kBN / 32];
+      float gl[C::kBRows / 32];
 #pragma unroll
-      for (int i = 0; i < C::kBN / 32; ++i) {
+      for (int i = 0; i < C::kBRows / 32; ++i) {
         const int r = 32 * i + lane;
         gl[i] = r < ti.nvalid ? __fmul_rn(a.act_G[ti.row0 + r], wG) : 0.f;
       }
@@ -368,7 +370,7 @@ __global__ void __launch_bounds__(kNpThreads, 1)
       const int wrow = ti.sub * kNpBM + q * 32 + lane;  // feature (gate/up) or output channel (down)
       const uint32_t trow = tmem_base + ab * C::kAccCols + ((uint32_t)(q * 32) << 16);
 #pragma unroll
-      for (int i = 0; i < C::kBN / 32; ++i) {
+      for (int i = 0; i < C::kBRows / 32; ++i) {
         const int c0 = 32 * i + 16 * half;  // rows c0 .. c0 + 15
         if (c0 >= ti.nvalid) break;
         uint32_t v0[16], v1[16];

@@ -105,9 +105,9 @@ def test_nvfp4_prefill_ragged_rows():
 
 
 def test_nvfp4_prefill_tile_boundaries():
-    """Experts whose row counts sit on either side of the 64-row gate/up and
-    128-row down tile sizes, in one batch."""
-    counts = [0, 1, 63, 64, 65, 127, 128, 129, 200, 3]
+    """Experts whose row counts sit on either side of the 80-row gate/up and
+    128-row down tile sizes (and of the 32-row activation boxes), in one batch."""
+    counts = [0, 1, 31, 33, 79, 80, 81, 127, 128, 129, 159, 160, 161, 200, 3]
     E, k = len(counts), 1
     owner = np.repeat(np.arange(E), counts)
     owner = owner[np.random.default_rng(6).permutation(owner.size)]
