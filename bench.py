@@ -49,7 +49,7 @@ DECODE_TRAFFIC = {"w4": 14242560, "nvfp4": 14289152}
 DTYPE_NV = "nvfp4 weights and activations (e2m1 + e4m3/16 + fp32 global), fp32 accumulate"
 # the same for the prefill FFN kernels: both launches of one layer at the bench's
 # token count (the bench's first layer), from profiles/prefill_*.md
-PREFILL_TRAFFIC = {"w4": 316057344, "nvfp4": 139742976}
+PREFILL_TRAFFIC = {"w4": 316057344, "nvfp4": 136497408}
 
 
 # ---------------------------------------------------------------------------- helpers
