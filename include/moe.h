@@ -344,8 +344,10 @@ MOE_API moe_status moe_ffn_w4a16_decode_static(const moe_w4_layer *layer, const 
  * accumulation in tensor memory, h rounded to bf16).
  * Source: "drama-rs", "Layout" (prefill: grouped MoE) and "Apple Silicon
  * (MLX)" (prefill groups rows by routed expert).
- * Workspace: moe_prefill_workspace_bytes(rows, F) bytes (h, bf16 [rows][F]),
- * 16-byte aligned.  Requirements: H % 256 == 0, F % 128 == 0, E <= 960,
+ * Workspace: moe_prefill_workspace_bytes(rows, F) bytes, 16-byte aligned.
+ * After the call its first rows * F * 2 bytes hold h (bf16 [rows][F], the
+ * gate/up stage, in the same grouped row order), for stage-wise checks.
+ * Requirements: H % 256 == 0, F % 128 == 0, E <= 960,
  * offsets non-decreasing with offsets[0] == 0 and offsets[E] == rows.
  * rows == 0 is a no-op.
  */
