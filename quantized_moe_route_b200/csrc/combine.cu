@@ -7,7 +7,9 @@
 
 namespace moe {
 
-template <bool kBf16In>
+// KC > 0 (bf16 rows only): k == KC is known at compile time, so the KC row
+// indices, then the KC rows, are all requested before the in-order sum.
+template <bool kBf16In, int KC = 0>
 __global__ void combine_kernel(const void *__restrict__ Y, const int32_t *__restrict__ inv,
                                const float *__restrict__ w, int T, int k, int H,
                                uint16_t *__restrict__ y) {
@@ -18,7 +20,29 @@ __global__ void combine_kernel(const void *__restrict__ Y, const int32_t *__rest
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  for (int j = 0; j < k; ++j) {
+  if (KC > 0) {
+    size_t pr[KC > 0 ? KC : 1];
+    float wr[KC > 0 ? KC : 1];
+    uint4 q[KC > 0 ? KC : 1];
+#pragma unroll
+    for (int j = 0; j < KC; ++j) {
+      const int r = t * KC + j;
+      pr[j] = inv ? (size_t)inv[r] : (size_t)r;
+      wr[j] = w[r];
+    }
+#pragma unroll
+    for (int j = 0; j < KC; ++j) q[j] = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(Y) + pr[j] * H + c0);
+#pragma unroll
+    for (int j = 0; j < KC; ++j) {
+      const uint32_t u[4] = {q[j].x, q[j].y, q[j].z, q[j].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] = __fadd_rn(acc[2 * i], __fmul_rn(wr[j], __uint_as_float(u[i] << 16)));
+        acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], __fmul_rn(wr[j], __uint_as_float(u[i] & 0xFFFF0000u)));
+      }
+    }
+  }
+  for (int j = 0; KC == 0 && j < k; ++j) {
     const int r = t * k + j;
     const size_t p = inv ? (size_t)inv[r] : (size_t)r;
     const float wj = w[r];
@@ -65,6 +89,6 @@ extern "C" MOE_API moe_status moe_unpermute_combine(const void *Y, int y_dtype, 
   if (T > 65535) return MOE_ERR_UNSUPPORTED_SHAPE;
   const int threads = 128;
   dim3 grid((H / 8 + threads - 1) / threads, T);
-  return launch_pdl(y_dtype == 1 ? combine_kernel<true> : combine_kernel<false>, grid, dim3(threads), 0,
-                    as_stream(stream), Y, inv, w, T, k, H, y);
+  auto kern = y_dtype == 1 ? (k == 8 ? combine_kernel<true, 8> : combine_kernel<true>) : combine_kernel<false>;
+  return launch_pdl(kern, grid, dim3(threads), 0, as_stream(stream), Y, inv, w, T, k, H, y);
 }
