@@ -69,3 +69,60 @@ def test_fma_form_error_bound_on_adversarial_groups(K):
     bound = 2.0 ** -24 * (2.0 ** (K + 1) * s + np.abs(m)) + 2.0 ** -23 * np.abs(q * s + m)
     assert np.all(err <= bound)
     assert np.all(err <= 2.0 ** -9 * s + 2.0 ** -23 * (np.abs(q * s + m) + np.abs(m)))
+
+
+# --------------------------------------------------------------- bit tricks
+def _f32_from_bits(u):
+    return np.asarray(u, np.uint32).view(np.float32).astype(np.float64)
+
+
+def test_prefill_nibble_to_magic_float():
+    """The prefill's per-word code extraction: for a packed word w, with
+    wl = w << 8 and wr = w >> 12, pair i = 0..3 takes nibble i (channel k) and
+    nibble i + 4 (channel k + 1) from (source, bit) = (wl, 8), (w, 16) for i = 0;
+    (wl, 12), (wr, 8); (w, 8), (wr, 12); (w, 12), (wr, 16); OR-ed into the
+    exponent pattern (150 - p) << 23 each is the fp32 value 2^(23 - p) + q."""
+    rng = np.random.default_rng(0)
+    w = rng.integers(0, 2 ** 32, 20000, dtype=np.uint64).astype(np.uint32)
+    wl = (w.astype(np.uint64) << 8).astype(np.uint32)
+    wr = w >> 12
+    src = {"w": w, "wl": wl, "wr": wr}
+    plan = [(("wl", 8), ("w", 16)), (("wl", 12), ("wr", 8)), (("w", 8), ("wr", 12)), (("w", 12), ("wr", 16))]
+    for i, pair in enumerate(plan):
+        for odd, (name, p) in enumerate(pair):
+            n = i + 4 * odd
+            q = (w >> (4 * n)) & 15
+            v = _f32_from_bits((src[name] & np.uint32(0xF << p)) | np.uint32((150 - p) << 23))
+            assert np.array_equal(v, 2.0 ** (23 - p) + q), (i, odd)
+
+
+def test_decode_int4_fragment_is_bf16_128_plus_q():
+    """The int4 decode's A fragment: ((w >> 4 i) & 0x000F000F) | 0x43004300 holds,
+    in each 16-bit half, the bf16 value 128 + q of nibble i (low half) and
+    nibble i + 4 (high half)."""
+    rng = np.random.default_rng(1)
+    w = rng.integers(0, 2 ** 32, 5000, dtype=np.uint64).astype(np.uint32)
+    for i in range(4):
+        a = ((w >> (4 * i)) & np.uint32(0x000F000F)) | np.uint32(0x43004300)
+        lo = _f32_from_bits((a & np.uint32(0xFFFF)) << 16)
+        hi = _f32_from_bits(a & np.uint32(0xFFFF0000))
+        assert np.array_equal(lo, 128.0 + ((w >> (4 * i)) & 15))
+        assert np.array_equal(hi, 128.0 + ((w >> (4 * i + 16)) & 15))
+
+
+@pytest.mark.parametrize("SH", [0, 4])
+def test_decode_e2m1_pair_to_f16(SH):
+    """The NVFP4 decode's fragment half: for the E2M1 codes at bits [SH, SH+4)
+    and [SH+16, SH+20) of w, (sign * 2^(12 - SH)) + ((w << (9 - SH)) & 0x0E000E00)
+    with sign = w & (0x00080008 << SH) is, per 16-bit half, the f16 encoding of
+    the code's value times 2^-14 (E2M1 magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6)."""
+    e2m1 = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float64)
+    codes = np.arange(256, dtype=np.uint32)
+    w = ((codes & 15) << SH) | ((codes >> 4) << (SH + 16))
+    sgn = w & np.uint32(0x00080008 << SH)
+    r = (sgn.astype(np.uint64) * (1 << (12 - SH)) + ((w.astype(np.uint64) << (9 - SH)) & 0x0E000E00)).astype(np.uint32)
+    for half, c in ((r & np.uint32(0xFFFF), codes & 15), (r >> 16, codes >> 4)):
+        val = half.astype(np.uint16).view(np.float16).astype(np.float64)
+        want = np.where(c & 8, -1.0, 1.0) * e2m1[c & 7] * 2.0 ** -14
+        assert np.array_equal(np.abs(val), np.abs(want))
+        assert np.array_equal(np.signbit(val), (c & 8) != 0)
