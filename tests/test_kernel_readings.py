@@ -126,3 +126,27 @@ def test_decode_e2m1_pair_to_f16(SH):
         want = np.where(c & 8, -1.0, 1.0) * e2m1[c & 7] * 2.0 ** -14
         assert np.array_equal(np.abs(val), np.abs(want))
         assert np.array_equal(np.signbit(val), (c & 8) != 0)
+
+
+# --------------------------------------------------------------- tile schedule
+def _cta_tile(i, b, G):
+    """The prefill kernels' i-th tile of CTA b: passes of G tiles, alternately
+    in and against CTA order."""
+    return i * G + (G - 1 - b if i & 1 else b)
+
+
+@pytest.mark.parametrize("G", [1, 2, 7, 148, 160])
+def test_alternating_passes_cover_every_tile_once(G):
+    """Each role of a CTA walks its tiles while cta_tile(i) < ntiles and stops at
+    the first one past the end; over all CTAs that must visit every tile exactly
+    once (no later pass may bring a CTA back below ntiles)."""
+    for ntiles in list(range(0, 3 * G + 3)) + [560, 1120, 4321]:
+        seen = []
+        for b in range(G):
+            i = 0
+            while _cta_tile(i, b, G) < ntiles:
+                seen.append(_cta_tile(i, b, G))
+                i += 1
+            # nothing below ntiles after the stop
+            assert all(_cta_tile(j, b, G) >= ntiles for j in range(i, i + 4))
+        assert sorted(seen) == list(range(ntiles))
