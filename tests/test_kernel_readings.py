@@ -150,3 +150,40 @@ def test_alternating_passes_cover_every_tile_once(G):
             # nothing below ntiles after the stop
             assert all(_cta_tile(j, b, G) >= ntiles for j in range(i, i + 4))
         assert sorted(seen) == list(range(ntiles))
+
+
+def _chunks_int4_prefill(counts, BN=256, BM=128):
+    """The int4 prefill's chunk numbering: per expert n // BN full chunks plus a
+    partial one; chunks of more than BM rows ("heavy") first, then those of at
+    most BM rows, each group in expert order.  Returns (e, row0, nvalid) per
+    chunk index."""
+    offsets = np.concatenate([[0], np.cumsum(counts)])
+    hc = [n // BN + (1 if n % BN > BM else 0) for n in counts]
+    lc = [1 if 0 < n % BN <= BM else 0 for n in counts]
+    hs = np.concatenate([[0], np.cumsum(hc)])
+    ls = np.concatenate([[0], np.cumsum(lc)])
+    out = []
+    for c in range(hs[-1] + ls[-1]):
+        if c < hs[-1]:
+            e = int(np.searchsorted(hs, c, side="right") - 1)
+            row0 = offsets[e] + (c - hs[e]) * BN
+        else:
+            e = int(np.searchsorted(ls, c - hs[-1], side="right") - 1)
+            row0 = offsets[e] + counts[e] // BN * BN
+        out.append((e, int(row0), int(min(BN, offsets[e + 1] - row0))))
+    return out, int(hs[-1])
+
+
+def test_heavy_first_chunks_partition_the_rows():
+    rng = np.random.default_rng(7)
+    cases = [[0, 1, 127, 128, 129, 255, 256, 257, 384, 385, 513, 16], [0] * 5, [2048]]
+    cases += [list(rng.integers(0, 700, rng.integers(1, 40))) for _ in range(50)]
+    for counts in cases:
+        chunks, nheavy = _chunks_int4_prefill(counts)
+        offsets = np.concatenate([[0], np.cumsum(counts)])
+        covered = np.zeros(int(offsets[-1]), np.int32)
+        for c, (e, row0, nv) in enumerate(chunks):
+            assert nv > 0 and offsets[e] <= row0 and row0 + nv <= offsets[e + 1]
+            assert (nv > 128) == (c < nheavy)  # heavy chunks are exactly the first nheavy
+            covered[row0:row0 + nv] += 1
+        assert np.all(covered == 1)
