@@ -34,9 +34,11 @@ def build(force: bool = False) -> str:
 
 
 def lib():
+    """The oracle library.  ORACLE_LIB names another build of moe_oracle.c to
+    load instead (the mutation tests load deliberately broken copies)."""
     global _lib
     if _lib is None:
-        _lib = ctypes.CDLL(build())
+        _lib = ctypes.CDLL(os.environ.get("ORACLE_LIB") or build())
         _declare(_lib)
     return _lib
 

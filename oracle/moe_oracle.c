@@ -416,8 +416,12 @@ ORC_API void orc_moe_forward_w4(const uint16_t *x, const float *logits, int T, i
 /* ("Drama 3 - NVFP4 routed experts", section "Quantization": round-to-      */
 /* nearest, one E4M3 scale per 16 input weights, FP32 global per matrix,     */
 /* dynamic per-token FP32 activation scales with E4M3 block scales.)         */
-/* Parity: decode tables pinned exhaustively; quantiser pinned by round trip */
-/* and error bound.                                                          */
+/* Parity: pinned.  Decode tables exhaustively; the global by hand values;  */
+/* the quantiser by round trip, per-(row, block) scales and error bound; the */
+/* GEMV by a constant-code closed form, one-hot rows with a distinct scale   */
+/* per (row, block), and a float64 matmul of the decoded operands within the */
+/* fp32 summation bound; the FFN by a constant-code closed form and a        */
+/* stage-wise composition of the pinned pieces.                              */
 /* ------------------------------------------------------------------------ */
 
 ORC_API float orc_nvfp4_global(const float *v, size_t n) {
