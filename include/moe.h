@@ -260,6 +260,13 @@ MOE_API moe_status moe_permute(const int32_t *idx, int T, int k, int E, const ui
  * experts of a token distinct.  Errors: INVALID_ARG, UNSUPPORTED_SHAPE,
  * WORKSPACE, CUDA.  A device-side wait that times out (it cannot under the
  * requirements above) raises the device error word: see moe_device_error().
+ * Co-residency: the kernel's thread blocks (one per SM, at most the SM count)
+ * wait on one another's results, so all of them must run at the same time.
+ * The launch is cooperative: while other work (another stream, another
+ * process under MPS) holds SMs, the GPU starts the grid only once every block
+ * can run, instead of starting part of it.  The same holds for
+ * moe_decode_layer_w4a16, moe_decode_layer_nvfp4 and
+ * moe_ffn_w4a16_decode_static.
  */
 MOE_API size_t moe_decode_workspace_bytes(int T, int k, int F);
 MOE_API moe_status moe_ffn_w4a16_decode(const moe_w4_layer *layer, const uint16_t *x,
@@ -327,7 +334,10 @@ MOE_API moe_status moe_decode_layer_nvfp4(const moe_nvfp4_layer *layer, const ui
  *     CTA counter word with a cudaMemsetAsync on `stream`, then launches the
  *     kernel; the call-number word keeps counting across calls.
  *   - The first call on a device looks up the array's device address on that
- *     (current) device; make that first call before any stream capture.
+ *     (current) device; make that first call before any stream capture.  The
+ *     address is cached per device for the life of the process: after a
+ *     cudaDeviceReset it is stale, so do not call this function again on
+ *     that device.
  *   - Every call on a device shares the one array and leaves its contents
  *     behind: two calls whose executions overlap on the GPU (different
  *     streams, no ordering between them) race and give wrong results.
@@ -402,6 +412,35 @@ MOE_API moe_status moe_unpermute_combine(const void *Y, int y_dtype, const int32
  * the device error word: 0 = none, otherwise a code naming the kernel and
  * wait that timed out.  The word is cleared on read. */
 MOE_API moe_status moe_device_error(int *out, moe_stream_t stream);
+
+/* Codes of the device error word. */
+#define MOE_DEVERR_DECODE_H_WAIT 0x101 /* decode: a wait for h or a row output gave up */
+#define MOE_DEVERR_PREFILL_WAIT 0x201  /* prefill: a pipeline barrier wait gave up */
+
+/*
+ * Test hooks for failure detection (no counterpart on the pages).  Each one
+ * makes a bounded device-side wait run out on purpose, without any fault, so
+ * that a test can check that the kernel gives up, returns, raises the device
+ * error word and leaves the GPU usable:
+ *   - moe_debug_starve_decode: moe_ffn_w4a16_decode whose gate/up work items
+ *     consume their weights but publish no h, with the down items' wait for
+ *     h bounded by `polls` polls (each >= 100 ns).  Raises
+ *     MOE_DEVERR_DECODE_H_WAIT.  y_rows is left unspecified; zero-fill the
+ *     workspace before its next use.
+ *   - moe_debug_starve_prefill: the gate/up launch of moe_ffn_grouped_prefill
+ *     whose weight producer issues no loads, every pipeline wait bounded by
+ *     `polls` sleeping polls (each at most ~10 us).  Raises
+ *     MOE_DEVERR_PREFILL_WAIT; the workspace (h) is left unspecified.
+ * Arguments and errors as for the calls they derive from; polls >= 1.
+ */
+MOE_API moe_status moe_debug_starve_decode(const moe_w4_layer *layer, const uint16_t *x,
+                                           const int32_t *idx, int T, int k, float *y_rows,
+                                           void *ws, size_t ws_bytes, unsigned int polls,
+                                           moe_stream_t stream);
+MOE_API moe_status moe_debug_starve_prefill(const moe_w4_layer *layer, const uint16_t *x_perm,
+                                            const int32_t *offsets, int rows, void *ws,
+                                            size_t ws_bytes, unsigned int polls,
+                                            moe_stream_t stream);
 
 #ifdef __cplusplus
 }

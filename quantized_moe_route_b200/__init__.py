@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(HERE, "libmoe.so")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE = 0, 1, 2
 MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = 3, 4, 5
+MOE_DEVERR_DECODE_H_WAIT, MOE_DEVERR_PREFILL_WAIT = 0x101, 0x201
 MOE_W4_PLAIN, MOE_W4_GATE_UP = 0, 1
 
 _lib = None
@@ -79,6 +80,9 @@ SIGNATURES = {
                                            _vp]),
     "moe_unpermute_combine": (_i, [_vp, _i, _vp, _vp, _i, _i, _i, _vp, _vp]),
     "moe_device_error": (_i, [ctypes.POINTER(ctypes.c_int), _vp]),
+    "moe_debug_starve_decode": (_i, [ctypes.POINTER(moe_w4_layer), _vp, _vp, _i, _i, _vp, _vp, _sz, ctypes.c_uint,
+                                     _vp]),
+    "moe_debug_starve_prefill": (_i, [ctypes.POINTER(moe_w4_layer), _vp, _vp, _i, _vp, _sz, ctypes.c_uint, _vp]),
 }
 
 
@@ -278,3 +282,17 @@ def moe_device_error(stream=None) -> int:
     out = ctypes.c_int(0)
     _check(lib().moe_device_error(ctypes.byref(out), _stream(stream)), "moe_device_error")
     return out.value
+
+
+def moe_debug_starve_decode(layer: moe_w4_layer, x, idx, y_rows, ws, polls, stream=None):
+    T, k = idx.shape
+    _check(lib().moe_debug_starve_decode(ctypes.byref(layer), _p(x), _p(idx), T, k, _p(y_rows), _p(ws),
+                                         ws.numel() * ws.element_size(), polls, _stream(stream)),
+           "moe_debug_starve_decode")
+
+
+def moe_debug_starve_prefill(layer: moe_w4_layer, x_perm, offsets, ws, polls, stream=None):
+    rows = x_perm.shape[0]
+    _check(lib().moe_debug_starve_prefill(ctypes.byref(layer), _p(x_perm), _p(offsets), rows, _p(ws),
+                                          ws.numel() * ws.element_size(), polls, _stream(stream)),
+           "moe_debug_starve_prefill")

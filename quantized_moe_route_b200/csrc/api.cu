@@ -1,4 +1,5 @@
 // api.cu -- status strings, CUDA error bookkeeping and the device error word.
+#include <atomic>
 #include <cstdio>
 #include <cstring>
 
@@ -27,16 +28,19 @@ __device__ int g_device_error;
 
 // The symbol's device address, looked up once per device (the lookup is not
 // a stream operation, so it is also safe while a stream is being captured).
+// Host threads may race on the first lookup; both find the same address.
 int *device_error_word() {
-  static int *cached[64] = {nullptr};
+  static std::atomic<int *> cached[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!cached[dev]) {
+  int *w = cached[dev].load(std::memory_order_acquire);
+  if (!w) {
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
-    cached[dev] = static_cast<int *>(p);
+    w = static_cast<int *>(p);
+    cached[dev].store(w, std::memory_order_release);
   }
-  return cached[dev];
+  return w;
 }
 
 }  // namespace moe

@@ -38,6 +38,8 @@
 // 2^-15); the tensor core sums one 16-channel block per m16n8k16 step, the
 // weight block scale is applied to that step's result in fp32, and 2^14 and
 // the two globals are applied once per output.
+#include <atomic>
+
 #include "common.cuh"
 #include "nvfp4.cuh"
 #include "route.cuh"
@@ -75,6 +77,8 @@ struct DecodeArgs {
   int nstages;               // even: team t owns the stages s = t (mod 2)
   uint32_t stage_bytes;
   uint32_t h_off;            // offset of a B item's h tile inside its stage
+  uint32_t h_polls;          // bound of a B item's wait for h (polls of >= 100 ns)
+  int starve_gate_up;        // test hook: A items write no h, so B items time out
 };
 
 struct DecodeSmem {
@@ -746,6 +750,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
 
   // ---- team `team` runs the CTA's items q = team, team + 2, ...
   bool aborted = false;
+  int q_abort = 0;  // the item a team gave up on
   for (int q = team; q < myCount; q += 2) {
     const int item = blockIdx.x + q * G;
     const int stage = q % a.nstages;
@@ -794,12 +799,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
           else if (!kFp4) h_s[(size_t)n * F + (f & ~63) + w4_kpos(f & 63)] = (uint16_t)(w >> 32);
         }
         ready = !team_or(bar_id, !mine);
-        if (ready || ++spins > (1u << 20)) break;
+        if (ready || ++spins > a.h_polls) break;
         __nanosleep(100);
       }
       if (!ready) {
         if (ttid == 0) atomicExch(a.err, DEVERR_DECODE_H_WAIT);
         aborted = true;
+        q_abort = q;
         break;
       }
       if (!kFp4) {
@@ -827,11 +833,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
     if (team_or(bar_id, !landed)) {  // only a copy stalled for seconds gets here
       if (ttid == 0) atomicExch(a.err, DEVERR_DECODE_H_WAIT);
       aborted = true;
+      q_abort = q;
       break;
     }
     const int nbmax = ntok > 8 ? 2 : 1;
     float *red = reinterpret_cast<float *>(st);  // reused once the weights are consumed
-    if (isA) {
+    if (isA && a.starve_gate_up) {
+      // test hook: the weights landed, but no h is computed or published
+    } else if (isA) {
       float acc[2][2][4] = {};
       const uint8_t *base[2] = {st, st + stripA};
       if (kFp4) {
@@ -947,14 +956,23 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
     fence_proxy_async_smem();
     if (team_or(bar_id, aborted)) {
       aborted = true;
+      q_abort = q;
       break;
     }
     if (ttid == 0 && q + a.nstages < myCount) issue(blockIdx.x + (q + a.nstages) * G, nA, stage, pol);
   }
 
-  // ---- aborted: let this team's in-flight copies land before leaving
+  // ---- aborted: let this team's in-flight copies land before leaving.  The
+  // team has issued the copies of its items up to q_abort + nstages - 2 (the
+  // first nstages at setup, then item q + nstages after finishing item q);
+  // a stage's last issued copy is the one to wait for (phases complete in
+  // order).
   if (aborted && ttid == 0) {
-    for (int s = team; s < a.nstages; s += 2) mbar_wait_bounded(&bars[s], 0, 1u << 20);
+    const int hi = min(myCount - 1, q_abort + a.nstages - 2);
+    for (int s = team; s < a.nstages && s <= hi; s += 2) {
+      const int ql = s + (hi - s) / a.nstages * a.nstages;
+      mbar_wait_bounded(&bars[s], (uint32_t)(ql / a.nstages) & 1u, 1u << 20);
+    }
   }
   __syncthreads();
   // ---- last CTA out records this call's epoch for the next call
@@ -968,8 +986,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
   }
 }
 
-// One or two CTAs per SM (all resident: B items wait on A items of other
-// CTAs); as many weight stages as fit.
+// One CTA per SM, as many weight stages as fit.  B items wait on A items of
+// other CTAs, so every CTA must be resident at once: the launch is
+// cooperative (the driver starts the grid only when all of its CTAs can run
+// together, and refuses a grid that can never fit), and the grid is sized
+// from the occupancy the kernel really gets.
 template <int kFmt, bool kFused, int PER>
 static moe_status decode_launch(DecodeArgs &a, bool pdl, cudaStream_t stream) {
   const int H = a.H, F = a.F, T = a.T, k = a.k;
@@ -984,30 +1005,41 @@ static moe_status decode_launch(DecodeArgs &a, bool pdl, cudaStream_t stream) {
   const DecodeSmem L = decode_smem_layout(kFmt, T, H, F, nst, a.stage_bytes);
   if (L.total > cap) return MOE_ERR_UNSUPPORTED_SHAPE;
   a.nstages = nst;
-  static bool attr_done[64] = {false};
-  if (dev < 64 && !attr_done[dev]) {
+  // per device: the shared-memory opt-in and the CTAs per SM it allows
+  // (host threads may race here; both values are idempotent)
+  static std::atomic<int> per_sm[64];
+  if (dev < 0 || dev >= 64) {
+    set_cuda_error(cudaErrorInvalidDevice);
+    return MOE_ERR_CUDA;
+  }
+  if (per_sm[dev].load(std::memory_order_acquire) == 0) {
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<kFmt, kFused, PER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)cap);
+    int occ = 0;
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<kFmt, kFused, PER>, kDecThreads, cap);
     if (e != cudaSuccess) {
       set_cuda_error(e);
       return MOE_ERR_CUDA;
     }
-    attr_done[dev] = true;
+    if (occ < 1) return MOE_ERR_UNSUPPORTED_SHAPE;
+    per_sm[dev].store(occ, std::memory_order_release);
   }
-  // one CTA per SM, all resident (B items wait on A items of other CTAs)
   const int maxItems = T * k * (F / 16 + H / kDecOutRows);
-  const int grid = max(1, min(sms, (maxItems + 1) / 2));
+  const int grid = max(1, min(sms * per_sm[dev].load(std::memory_order_acquire), (maxItems + 1) / 2));
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kDecThreads);
   cfg.dynamicSmemBytes = L.total;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = pdl ? 2 : 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<kFmt, kFused, PER>, a);
   if (e != cudaSuccess) {
     set_cuda_error(e);
@@ -1054,6 +1086,8 @@ static void decode_fill(DecodeArgs &a, const moe_w4_layer *layer, const uint16_t
   a.F = layer->F;
   a.ctrl = reinterpret_cast<unsigned int *>(scratch);
   a.hbuf = reinterpret_cast<unsigned long long *>(scratch + kDecCtrlBytes);
+  a.h_polls = 1u << 20;
+  a.starve_gate_up = 0;
 }
 
 }  // namespace moe
@@ -1075,6 +1109,23 @@ extern "C" MOE_API moe_status moe_ffn_w4a16_decode(const moe_w4_layer *layer, co
   if (reinterpret_cast<uintptr_t>(ws) % 16) return MOE_ERR_INVALID_ARG;
   DecodeArgs a;
   decode_fill(a, layer, x, idx, T, k, y_rows, static_cast<uint8_t *>(ws));
+  a.err = device_error_word();
+  if (!a.err) return MOE_ERR_CUDA;
+  return decode_launch<kFmtW4, false, 8>(a, true, as_stream(stream));
+}
+
+extern "C" MOE_API moe_status moe_debug_starve_decode(const moe_w4_layer *layer, const uint16_t *x,
+                                                      const int32_t *idx, int T, int k, float *y_rows,
+                                                      void *ws, size_t ws_bytes, unsigned int polls,
+                                                      moe_stream_t stream) {
+  moe_status st = decode_check(layer, x, idx, T, k, y_rows);
+  if (st != MOE_OK || T == 0) return st;
+  if (!ws || ws_bytes < moe_decode_workspace_bytes(T, k, layer->F)) return MOE_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) % 16 || polls == 0) return MOE_ERR_INVALID_ARG;
+  DecodeArgs a;
+  decode_fill(a, layer, x, idx, T, k, y_rows, static_cast<uint8_t *>(ws));
+  a.h_polls = polls;
+  a.starve_gate_up = 1;
   a.err = device_error_word();
   if (!a.err) return MOE_ERR_CUDA;
   return decode_launch<kFmtW4, false, 8>(a, true, as_stream(stream));
@@ -1175,9 +1226,11 @@ constexpr size_t kStaticScratchBytes = kDecCtrlBytes + kStaticHBytes;
 static __device__ __align__(256) uint8_t g_decode_scratch[kStaticScratchBytes];
 
 // Device address of g_decode_scratch on the current device, looked up once per
-// device (the lookup needs that device to be current).
+// device (the lookup needs that device to be current).  Host threads may race
+// on the first lookup; both find the same address.  A device reset
+// (cudaDeviceReset) invalidates the cached address.
 static uint8_t *static_scratch_address(moe_status *st) {
-  static uint8_t *addr[64] = {nullptr};
+  static std::atomic<uint8_t *> addr[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess || dev < 0 || dev >= 64) {
@@ -1185,7 +1238,8 @@ static uint8_t *static_scratch_address(moe_status *st) {
     *st = MOE_ERR_CUDA;
     return nullptr;
   }
-  if (!addr[dev]) {
+  uint8_t *a = addr[dev].load(std::memory_order_acquire);
+  if (!a) {
     void *p = nullptr;
     e = cudaGetSymbolAddress(&p, g_decode_scratch);
     if (e != cudaSuccess || !p) {
@@ -1193,10 +1247,11 @@ static uint8_t *static_scratch_address(moe_status *st) {
       *st = MOE_ERR_CUDA;
       return nullptr;
     }
-    addr[dev] = static_cast<uint8_t *>(p);
+    a = static_cast<uint8_t *>(p);
+    addr[dev].store(a, std::memory_order_release);
   }
   *st = MOE_OK;
-  return addr[dev];
+  return a;
 }
 
 }  // namespace moe

@@ -28,6 +28,8 @@
 // rows on N turn 32 outputs x 16 rows around in shared memory for 16-byte
 // stores; rows on M write stretches of their own row.
 // Every wait is bounded; a timeout raises the device error word.
+#include <atomic>
+
 #include "common.cuh"
 #include "tcgen05.cuh"
 
@@ -81,6 +83,8 @@ struct PrefillArgs {
   int ld_out;              // F (gate/up) or H (down)
   int F;                   // gate/up: features per matrix (strip index of the up half)
   int spe;                 // strip pairs (gate/up) or strips (down) per expert
+  uint32_t wait_polls;     // bound of every pipeline wait (sleeping polls)
+  int starve_weights;      // test hook: the int4 producer issues no loads
 };
 
 // ---------------------------------------------------------------- tiles
@@ -94,17 +98,21 @@ struct TileInfo {
   int e, row0, nvalid, sub;
 };
 __device__ __forceinline__ TileInfo tile_info(int t, int n_sub, const int *heavy_start,
-                                              const int *light_start, int E, const int32_t *offsets) {
+                                              const int *light_start, int E, const int32_t *offsets,
+                                              int rows) {
   const int chunk = t / n_sub, nheavy = heavy_start[E];
   TileInfo ti;
+  int o0, o1;
   if (chunk < nheavy) {
     ti.e = last_at_or_below(heavy_start, E, chunk);
-    ti.row0 = offsets[ti.e] + (chunk - heavy_start[ti.e]) * kPfBN;
+    o0 = clamped_offset(offsets, ti.e, rows), o1 = clamped_offset(offsets, ti.e + 1, rows);
+    ti.row0 = o0 + (chunk - heavy_start[ti.e]) * kPfBN;
   } else {
     ti.e = last_at_or_below(light_start, E, chunk - nheavy);
-    ti.row0 = offsets[ti.e] + (offsets[ti.e + 1] - offsets[ti.e]) / kPfBN * kPfBN;  // the partial chunk
+    o0 = clamped_offset(offsets, ti.e, rows), o1 = clamped_offset(offsets, ti.e + 1, rows);
+    ti.row0 = o0 + (o1 - o0) / kPfBN * kPfBN;  // the partial chunk
   }
-  ti.nvalid = min(kPfBN, offsets[ti.e + 1] - ti.row0);
+  ti.nvalid = min(kPfBN, o1 - ti.row0);
   ti.sub = t % n_sub;
   return ti;
 }
@@ -158,7 +166,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     int hcarry = 0, lcarry = 0;
     for (int e0 = 0; e0 < a.E; e0 += 32) {
       const int e = e0 + lane;
-      const int n = e < a.E ? max(a.offsets[e + 1] - a.offsets[e], 0) : 0;
+      const int n = e < a.E ? max(clamped_offset(a.offsets, e + 1, a.rows) - clamped_offset(a.offsets, e, a.rows), 0)
+                            : 0;
       const int rem = n % kPfBN;
       const int hc = n / kPfBN + (rem > kPfBM ? 1 : 0), lc = (rem > 0 && rem <= kPfBM) ? 1 : 0;
       int hi = hc, li = lc;
@@ -196,14 +205,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ int4 producer
-    if (lane == 0) {
+    if (lane == 0 && !a.starve_weights) {
       uint32_t it = 0;
       for (int i = 0, t = cta_tile(0, blockIdx.x, G); t < ntiles && !*abort_s; t = cta_tile(++i, blockIdx.x, G)) {
-        const TileInfo ti = tile_info(t, a.n_sub, heavy_start, light_start, a.E, a.offsets);
+        const TileInfo ti = tile_info(t, a.n_sub, heavy_start, light_start, a.E, a.offsets, a.rows);
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % C::kRawStages;
           const uint32_t ph = (it / C::kRawStages) & 1u;
-          if (!mbar_wait_sleep(&raw_empty[s], ph ^ 1u, kPfWaitPolls)) {
+          if (!mbar_wait_sleep(&raw_empty[s], ph ^ 1u, a.wait_polls)) {
             fail();
             break;
           }
@@ -221,18 +230,23 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
         }
       }
+      // aborted: the last load issued into each stage lands before the CTA
+      // leaves (iterations [0, it) were issued)
+      if (*abort_s)
+        for (uint32_t j = it > (uint32_t)C::kRawStages ? it - C::kRawStages : 0u; j < it; ++j)
+          mbar_wait_sleep(&raw_full[j % C::kRawStages], (j / C::kRawStages) & 1u, a.wait_polls);
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ activation producer
     if (lane == 0) {
       uint32_t it = 0;
       for (int i = 0, t = cta_tile(0, blockIdx.x, G); t < ntiles && !*abort_s; t = cta_tile(++i, blockIdx.x, G)) {
-        const TileInfo ti = tile_info(t, a.n_sub, heavy_start, light_start, a.E, a.offsets);
+        const TileInfo ti = tile_info(t, a.n_sub, heavy_start, light_start, a.E, a.offsets, a.rows);
         const int nbox = (ti.nvalid + 63) / 64;  // whole 64-row boxes covering the valid rows
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % C::kBStages;
           const uint32_t ph = (it / C::kBStages) & 1u;
-          if (!mbar_wait_sleep(&b_empty[s], ph ^ 1u, kPfWaitPolls)) {
+          if (!mbar_wait_sleep(&b_empty[s], ph ^ 1u, a.wait_polls)) {
             fail();
             break;
           }
@@ -242,6 +256,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             tma_load_2d(btile + r * 128, &act_map, kb * kPfBK, ti.row0 + r, &b_full[s]);
         }
       }
+      if (*abort_s)  // as for the int4 producer
+        for (uint32_t j = it > (uint32_t)C::kBStages ? it - C::kBStages : 0u; j < it; ++j)
+          mbar_wait_sleep(&b_full[j % C::kBStages], (j / C::kBStages) & 1u, a.wait_polls);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -251,14 +268,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       uint32_t it = 0, tcount = 0;
       for (int i = 0, t = cta_tile(0, blockIdx.x, G); t < ntiles && !*abort_s;
            t = cta_tile(++i, blockIdx.x, G), ++tcount) {
-        const TileInfo ti = tile_info(t, a.n_sub, heavy_start, light_start, a.E, a.offsets);
+        const TileInfo ti = tile_info(t, a.n_sub, heavy_start, light_start, a.E, a.offsets, a.rows);
         // A tile of at most 128 rows is issued transposed (rows on M, the 256
         // weight rows on N): one MMA per k16 step instead of two.  An MMA
         // costs about as much at N = 16 as at N = 200, so this halves the
         // tensor time of the many few-row tiles.
         const bool swapped = ti.nvalid <= kPfBM;
         const uint32_t idesc = idesc_bf16_f32(swapped ? C::kMats * kPfBM : (ti.nvalid + 15) & ~15);
-        if (!mbar_wait_sleep(tmem_empty, (tcount & 1u) ^ 1u, kPfWaitPolls)) {
+        if (!mbar_wait_sleep(tmem_empty, (tcount & 1u) ^ 1u, a.wait_polls)) {
           fail();
           break;
         }
@@ -267,8 +284,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int sa = it % C::kAStages, sb = it % C::kBStages;
           const uint32_t pa = (it / C::kAStages) & 1u, pb = (it / C::kBStages) & 1u;
-          if (!mbar_wait_sleep(&b_full[sb], pb, kPfWaitPolls) ||
-              !mbar_wait_sleep(&a_full[sa], pa, kPfWaitPolls)) {
+          if (!mbar_wait_sleep(&b_full[sb], pb, a.wait_polls) ||
+              !mbar_wait_sleep(&a_full[sa], pa, a.wait_polls)) {
             fail();
             ok = false;
             break;
@@ -325,13 +342,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const uint32_t scale_off = (uint32_t)(rbk * kBlkBytes + kBlkCodeBytes + 4 * gi);
     uint32_t it = 0, tcount = 0;
     for (int i = 0, t = cta_tile(0, blockIdx.x, G); t < ntiles; t = cta_tile(++i, blockIdx.x, G), ++tcount) {
-      const TileInfo ti = tile_info(t, a.n_sub, heavy_start, light_start, a.E, a.offsets);
+      const TileInfo ti = tile_info(t, a.n_sub, heavy_start, light_start, a.E, a.offsets, a.rows);
       bool ok = true;
       for (int kb = 0; kb < KB; ++kb, ++it) {
         const int sr = it % C::kRawStages, sa = it % C::kAStages;
         const uint32_t pr = (it / C::kRawStages) & 1u, pa = (it / C::kAStages) & 1u;
-        const bool landed = mbar_wait_sleep(&raw_full[sr], pr, kPfWaitPolls) &&
-                            mbar_wait_sleep(&a_empty[sa], pa ^ 1u, kPfWaitPolls);
+        const bool landed = mbar_wait_sleep(&raw_full[sr], pr, a.wait_polls) &&
+                            mbar_wait_sleep(&a_empty[sa], pa ^ 1u, a.wait_polls);
         if (!landed || *abort_s) {
           if (!landed) fail();
           ok = false;
@@ -394,7 +411,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (!ok) break;
       // ---- epilogue: accumulators of this tile; the four warps of a lane
       // quarter split the columns
-      if (!mbar_wait_sleep(tmem_full, tcount & 1u, kPfWaitPolls)) {
+      if (!mbar_wait_sleep(tmem_full, tcount & 1u, a.wait_polls)) {
         fail();
         break;
       }
@@ -534,15 +551,19 @@ static moe_status prefill_launch(const PrefillArgs &a, const CUtensorMap &map, c
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  static bool attr_done[64] = {false};
-  if (dev < 64 && !attr_done[dev]) {
+  static std::atomic<bool> attr_done[64];  // per device; the attribute call is idempotent
+  if (dev < 0 || dev >= 64) {
+    set_cuda_error(cudaErrorInvalidDevice);
+    return MOE_ERR_CUDA;
+  }
+  if (!attr_done[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(prefill_kernel<kGU>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmemBytes);
     if (e != cudaSuccess) {
       set_cuda_error(e);
       return MOE_ERR_CUDA;
     }
-    attr_done[dev] = true;
+    attr_done[dev].store(true, std::memory_order_release);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(sms);
@@ -611,6 +632,8 @@ extern "C" MOE_API moe_status moe_ffn_grouped_prefill(const moe_w4_layer *layer,
   gu.ld_out = F;
   gu.F = F;
   gu.spe = F / 16;  // strip pairs per expert
+  gu.wait_polls = kPfWaitPolls;
+  gu.starve_weights = 0;
   moe_status st = prefill_launch<true>(gu, xmap, gumap, s);
   if (st != MOE_OK) return st;
   PrefillArgs dn = gu;
@@ -622,4 +645,42 @@ extern "C" MOE_API moe_status moe_ffn_grouped_prefill(const moe_w4_layer *layer,
   dn.ld_out = H;
   dn.spe = H / 16;  // strips per expert
   return prefill_launch<false>(dn, hmap, dnmap, s);
+}
+
+extern "C" MOE_API moe_status moe_debug_starve_prefill(const moe_w4_layer *layer, const uint16_t *x_perm,
+                                                       const int32_t *offsets, int rows, void *ws,
+                                                       size_t ws_bytes, unsigned int polls,
+                                                       moe_stream_t stream) {
+  if (!layer || rows <= 0 || polls == 0) return MOE_ERR_INVALID_ARG;
+  const int E = layer->E, H = layer->H, F = layer->F;
+  if (E <= 0 || H <= 0 || F <= 0) return MOE_ERR_INVALID_ARG;
+  if (H % (2 * kPfBM) || F % kPfBM || E > 960) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!layer->gate_up || !x_perm || !offsets) return MOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < moe_prefill_workspace_bytes(rows, F)) return MOE_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(x_perm) % 16 || reinterpret_cast<uintptr_t>(ws) % 16 ||
+      reinterpret_cast<uintptr_t>(layer->gate_up) % 16)
+    return MOE_ERR_INVALID_ARG;
+  int *err = device_error_word();
+  if (!err) return MOE_ERR_CUDA;
+  CUtensorMap xmap, gumap;
+  if (!make_act_map(&xmap, x_perm, rows, H) || !make_w4_map(&gumap, layer->gate_up, E, 2 * F, H, true)) {
+    set_cuda_error(cudaErrorInvalidValue);
+    return MOE_ERR_CUDA;
+  }
+  PrefillArgs gu;
+  gu.w = static_cast<const uint8_t *>(layer->gate_up);
+  gu.w_stride = w4_packed_bytes(2 * F, H);
+  gu.offsets = offsets;
+  gu.out = static_cast<uint16_t *>(ws);
+  gu.err = err;
+  gu.E = E;
+  gu.K = H;
+  gu.rows = rows;
+  gu.n_sub = F / kPfBM;
+  gu.ld_out = F;
+  gu.F = F;
+  gu.spe = F / 16;
+  gu.wait_polls = polls;
+  gu.starve_weights = 1;
+  return prefill_launch<true>(gu, xmap, gumap, as_stream(stream));
 }

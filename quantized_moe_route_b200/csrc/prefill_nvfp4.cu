@@ -26,6 +26,8 @@
 //               tiles of 80 rows, down tiles of 128) so the epilogue of one
 //               tile overlaps the next tile's MMAs
 // Every wait is bounded; a timeout raises the device error word.
+#include <atomic>
+
 #include "common.cuh"
 #include "nvfp4.cuh"
 #include "tcgen05.cuh"
@@ -130,7 +132,7 @@ struct NpTile {
   int e, row0, nvalid, sub;
 };
 __device__ __forceinline__ NpTile np_tile(int t, int n_sub, const int *chunk_start, int E,
-                                          const int32_t *offsets, int bn) {
+                                          const int32_t *offsets, int rows, int bn) {
   const int chunk = t / n_sub;
   int lo = 0, hi = E - 1;  // last expert with chunk_start[e] <= chunk
   while (lo < hi) {
@@ -140,8 +142,8 @@ __device__ __forceinline__ NpTile np_tile(int t, int n_sub, const int *chunk_sta
   }
   NpTile ti;
   ti.e = lo;
-  ti.row0 = offsets[lo] + (chunk - chunk_start[lo]) * bn;
-  ti.nvalid = min(bn, offsets[lo + 1] - ti.row0);
+  ti.row0 = clamped_offset(offsets, lo, rows) + (chunk - chunk_start[lo]) * bn;
+  ti.nvalid = min(bn, clamped_offset(offsets, lo + 1, rows) - ti.row0);
   ti.sub = t % n_sub;
   return ti;
 }
@@ -189,7 +191,8 @@ __global__ void __launch_bounds__(kNpThreads, 1)
     int carry = 0;
     for (int e0 = 0; e0 < a.E; e0 += 32) {
       const int e = e0 + lane;
-      const int n = e < a.E ? a.offsets[e + 1] - a.offsets[e] : 0;
+      const int n = e < a.E ? max(clamped_offset(a.offsets, e + 1, a.rows) - clamped_offset(a.offsets, e, a.rows), 0)
+                            : 0;
       const int c = (max(n, 0) + C::kBN - 1) / C::kBN;
       int incl = c;
 #pragma unroll
@@ -221,7 +224,7 @@ __global__ void __launch_bounds__(kNpThreads, 1)
     if (lane == 0) {
       uint32_t it = 0;
       for (int t = blockIdx.x; t < ntiles && !*abort_s; t += G) {
-        const NpTile ti = np_tile(t, a.n_sub, chunk_start, a.E, a.offsets, C::kBN);
+        const NpTile ti = np_tile(t, a.n_sub, chunk_start, a.E, a.offsets, a.rows, C::kBN);
         const int strip0 = ti.e * a.spe + 8 * ti.sub;  // first strip (pair) of the weight tile
         for (int kt = 0; kt < KT; ++kt, ++it) {
           const int s = it % C::kStages;
@@ -301,7 +304,7 @@ __global__ void __launch_bounds__(kNpThreads, 1)
       const uint64_t dsw0 = smem_desc_sw128(smem_u32(smem)), dpl0 = smem_desc_plain(smem_u32(smem));
       uint32_t it = 0, tcount = 0;
       for (int t = blockIdx.x; t < ntiles && !*abort_s; t += G, ++tcount) {
-        const NpTile ti = np_tile(t, a.n_sub, chunk_start, a.E, a.offsets, C::kBN);
+        const NpTile ti = np_tile(t, a.n_sub, chunk_start, a.E, a.offsets, a.rows, C::kBN);
         const uint32_t idesc = idesc_nvf4((ti.nvalid + 15) & ~15);
         const int ab = tcount % C::kAcc;
         const uint32_t acc0 = tmem_base + ab * C::kAccCols;
@@ -351,7 +354,7 @@ __global__ void __launch_bounds__(kNpThreads, 1)
     const int half = (warp - 4) >> 2;  // the two warps of a quarter take alternate 16-column chunks
     uint32_t tcount = 0;
     for (int t = blockIdx.x; t < ntiles; t += G, ++tcount) {
-      const NpTile ti = np_tile(t, a.n_sub, chunk_start, a.E, a.offsets, C::kBN);
+      const NpTile ti = np_tile(t, a.n_sub, chunk_start, a.E, a.offsets, a.rows, C::kBN);
       const int ab = tcount % C::kAcc;
       // the tile's activation globals times the expert's weight global,
       // loaded while the MMAs run: lane l holds rows l, l + 32, ...
@@ -468,15 +471,19 @@ static moe_status np_launch(const NpArgs &a, const CUtensorMap &wm, const CUtens
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  static bool attr_done[64] = {false};
-  if (dev < 64 && !attr_done[dev]) {
+  static std::atomic<bool> attr_done[64];  // per device; the attribute call is idempotent
+  if (dev < 0 || dev >= 64) {
+    set_cuda_error(cudaErrorInvalidDevice);
+    return MOE_ERR_CUDA;
+  }
+  if (!attr_done[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(prefill_nvfp4_kernel<kGU>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmemBytes);
     if (e != cudaSuccess) {
       set_cuda_error(e);
       return MOE_ERR_CUDA;
     }
-    attr_done[dev] = true;
+    attr_done[dev].store(true, std::memory_order_release);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(sms);

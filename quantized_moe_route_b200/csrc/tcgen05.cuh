@@ -112,6 +112,14 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, i
       : "memory");
 }
 
+// offsets[i] clamped to [0, rows].  A group table that breaks its contract
+// (offsets[E] > rows, a negative or decreasing entry) then selects no row
+// outside [0, rows): nothing is read or written out of bounds, and a
+// decreasing pair simply gives its expert no rows.
+__device__ __forceinline__ int clamped_offset(const int32_t *offsets, int i, int rows) {
+  return min(max(offsets[i], 0), rows);
+}
+
 // Grouped-GEMM tile scheduling shared by the prefill kernels.
 // Last expert e with start[e] <= c (start: exclusive scan of per-expert chunk counts).
 __device__ __forceinline__ int last_at_or_below(const int *start, int E, int c) {

@@ -1,4 +1,6 @@
 """GPU parity of the decode path (route -> weight-streaming FFN -> combine)."""
+import time
+
 import numpy as np
 import pytest
 import torch
@@ -145,3 +147,64 @@ def test_fused_layer_one_expert_for_all_tokens_and_reuse():
     assert np.array_equal(y1, y2)
     _, _, _, oy = oracle.moe_forward_w4(x, logits, k, layer.canon)
     ffn_close(synth.bf16_bits_to_f32(y1), synth.bf16_bits_to_f32(oy), "fused y")
+
+
+def test_fused_decode_waits_while_another_stream_holds_an_sm():
+    """The decode kernel's down items wait on gate/up items of other CTAs of
+    the same grid, so every CTA must run at once.  The launch is cooperative:
+    while a kernel on another stream holds one SM (and all its shared memory)
+    for about a second, the decode grid does not start on the other SMs and
+    then time out waiting for the missing CTA; it waits for the SM, runs
+    whole, and gives the oracle's result with no device error."""
+    import gpu_hold
+    E, H, F, T, k, seed = 256, 2048, 512, 1, 8, 91
+    x = synth.activations_bf16(seed, 0, T, H)
+    logits = synth.router_logits(seed, 0, T, E)
+    oidx, _ = oracle.route(logits, k)
+    layer = Layer(seed, 0, E, H, F, oidx.ravel())
+    xd, ld = u16(x), torch.from_numpy(logits).cuda()
+    y = torch.empty((T, H), dtype=torch.int16, device="cuda")
+    ws = torch.zeros(moe.moe_decode_layer_workspace_bytes(T, k, H, F), dtype=torch.uint8, device="cuda")
+    done = torch.zeros(1, dtype=torch.int32, device="cuda")
+    smem = torch.cuda.get_device_properties(0).shared_memory_per_block_optin
+    side, main = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    gpu_hold.hold_sm(2_000_000_000, smem, done, side)  # about one second at 1.9 GHz
+    time.sleep(0.05)  # the holding CTA is resident before the decode is launched
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(main):
+        e0.record(main)
+        moe.moe_decode_layer_w4a16(layer.desc, xd, ld, k, y, ws, stream=main)
+        e1.record(main)
+    torch.cuda.synchronize()
+    assert done.item() == 1
+    assert moe.moe_device_error() == 0
+    _, _, _, oy = oracle.moe_forward_w4(x, logits, k, layer.canon)
+    ffn_close(synth.bf16_bits_to_f32(to_u16(y)), synth.bf16_bits_to_f32(oy), "y")
+    # the grid did wait for the held SM (it needs every SM)
+    assert e0.elapsed_time(e1) > 300.0
+
+
+@pytest.mark.parametrize("T", [1, 16])
+def test_fused_decode_chain_of_two_full_size_layers(T):
+    """The 40-layer stream's launch configuration: full-size layers (256
+    experts, hidden 2048, width 512, top-8), one fused launch per layer, the
+    second layer reading the first one's y; each layer's rows are checked
+    against the oracle on that layer's own input."""
+    E, H, F, k, seed = 256, 2048, 512, 8, 92
+    x = synth.activations_bf16(seed, 0, T, H)
+    ws = torch.zeros(moe.moe_decode_layer_workspace_bytes(T, k, H, F), dtype=torch.uint8, device="cuda")
+    xin = x
+    d_in = u16(x)
+    for l in range(2):
+        logits = synth.router_logits(seed, l, T, E)
+        oidx, _ = oracle.route(logits, k)
+        layer = Layer(seed, l, E, H, F, oidx.ravel())
+        y = torch.empty((T, H), dtype=torch.int16, device="cuda")
+        moe.moe_decode_layer_w4a16(layer.desc, d_in, torch.from_numpy(logits).cuda(), k, y, ws)
+        torch.cuda.synchronize()
+        assert moe.moe_device_error() == 0
+        _, _, _, oy = oracle.moe_forward_w4(xin, logits, k, layer.canon)
+        got = to_u16(y)
+        ffn_close(synth.bf16_bits_to_f32(got), synth.bf16_bits_to_f32(oy), f"layer {l} y")
+        xin, d_in = got, y  # the next layer reads this layer's output

@@ -1,6 +1,7 @@
 """Edge cases at the documented limits: the fused decode at its row limit
 (T*k = 256) and expert limit (E = 1024), the prefill at E = 960, the
-no-op T = 0 / rows = 0 calls, and the rejections just past each limit."""
+no-op T = 0 / rows = 0 calls, the rejections just past each limit, and a
+prefill group table that claims more rows than the call has."""
 import ctypes
 
 import numpy as np
@@ -105,3 +106,32 @@ def test_nvfp4_prefill_at_expert_limit():
     from test_gpu_prefill_nvfp4 import _check as nv_check
     g = nv_check(79, 960, 256, 256, 128, 4, stagewise_rows=4)
     assert (np.diff(g["offsets"]) == 0).sum() > 400
+
+
+def test_prefill_offsets_past_rows_write_nothing_past_rows():
+    """A group table that breaks its contract (offsets[E] = 160 > rows = 100)
+    is clamped to the rows the caller passed: the rows below 100 still get
+    their experts' outputs, and nothing at or past row 100 (of y_perm or of
+    the h workspace) is written."""
+    E, H, F, rows, pad, seed = 4, 256, 128, 100, 96, 81
+    offsets = np.array([0, 30, 60, 100, 160], np.int32)
+    layer = Layer(seed, 0, E, H, F, range(E))
+    xp = synth.activations_bf16(seed, 0, rows + pad, H)
+    x_perm = u16(xp)
+    sentinel = 0x5A5A
+    y_perm = torch.full((rows + pad, H), sentinel, dtype=torch.int16, device="cuda")
+    hbytes = moe.moe_prefill_workspace_bytes(rows, F)
+    ws = torch.full((hbytes + pad * F * 2,), 0x5A, dtype=torch.uint8, device="cuda")
+    d_off = torch.from_numpy(offsets).cuda()
+    L = moe.lib()
+    st = L.moe_ffn_grouped_prefill(ctypes.byref(layer.desc), moe._p(x_perm), moe._p(d_off), rows, moe._p(y_perm),
+                                   moe._p(ws), hbytes, None)
+    assert st == moe.MOE_OK
+    torch.cuda.synchronize()
+    assert moe.moe_device_error() == 0
+    y = to_u16(y_perm)
+    assert np.all(y[rows:] == sentinel)
+    assert np.all(ws[rows * F * 2:].cpu().numpy() == 0x5A)
+    want = np.stack([oracle.expert_ffn_w4(xp[p], *layer.canon[int(np.searchsorted(offsets, p, side="right") - 1)])
+                     for p in range(rows)])
+    ffn_close(synth.bf16_bits_to_f32(y[:rows]), want, "y_perm (valid rows)")

@@ -4,7 +4,8 @@ moe_ffn_w4a16_decode_static serves callers that cannot allocate device
 memory (plugins whose host owns all device memory, fixed memory plans): it
 keeps its scratch in a fixed library-owned array instead of a caller
 workspace.  Here it is called through the C ABI and compared with the
-workspace form, moe_ffn_w4a16_decode, on two calls in a row.  This file is
+workspace form, moe_ffn_w4a16_decode, on two calls in a row, and with the
+CPU oracle's per-row expert outputs.  This file is
 collected last so that a run stopping at the first failure has run every
 other test already.
 """
@@ -51,8 +52,10 @@ def test_static_scratch_decode_matches_workspace_decode(E, H, F, T, k):
     layer = Layer(31, 0, E, H, F, idx_np.ravel())
     idx = torch.from_numpy(idx_np).cuda()
     ref, outs = _decode_both(layer, u16(x), idx, k)
+    _, _, oracle_rows, _ = oracle.moe_forward_w4(x, logits, k, layer.canon)
     for y in outs:
         ffn_close(y, ref, "static-scratch decode vs workspace decode")
+        ffn_close(y, oracle_rows, "static-scratch decode vs oracle")
 
 
 def test_static_scratch_rejects_sizes_over_its_limit():
