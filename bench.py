@@ -1,24 +1,35 @@
 #!/usr/bin/env python
-"""Benchmark of the routed int4 MoE FFN hot path on B200.
+"""Benchmark of the routed int4 / NVFP4 MoE FFN hot path on B200.
 
-Default workload (one "step"): single-layer decode of 1 token through a MoE
-layer with 256 experts, top-8, hidden 2048, expert width 512 -- route, the
-weight-streaming expert FFN, combine.  Steps rotate over 40 resident layers
-(40 x 256 experts x 3 int4 matrices = 18.1 GB in HBM, each layer with its own
-activations and fresh router logits), so the 14.2 MB a step streams is never
-L2-resident from an earlier step (inputs larger than L2, no flush needed).
+One JSON line.  Its top level is single-layer decode: one token through one
+MoE layer (256 experts, top-8, hidden 2048, expert width 512) per step,
+route + weight-streaming expert FFN + combine in one launch, steps rotating
+over 40 resident int4 layers (18.1 GB, so the 14.2 MB a step streams never
+sits in L2 from an earlier step).  With the default --workload all, a `legs`
+object adds:
+  decode_stream_T1/T4/T16  40 chained layers per step (x of layer l+1 = y of
+                           layer l, fresh router logits per layer), 1/4/16 tokens
+  prefill_2048             2048 tokens (Zipf-skewed routing): route, permute,
+                           tcgen05 grouped FFN (two launches), combine
+  nvfp4_prefill_512        the NVFP4 experts on 512 Zipf-routed tokens
+  nvfp4_decode_T1          single-layer decode on 40 resident NVFP4 layers
+Each leg carries its own roofline (HBM GB/s or TFLOP/s against the measured
+peak), end-to-end throughput through the C ABI with host buffers, and the CPU
+oracle timed on a bounded sample of the same workload (one core and all
+cores).
 
-Prints one JSON line (see the design doc for every key).  Multi-GPU: one process
-per GPU (torchrun), each rank an independent replica of the workload (the
-path has no exchange step), barrier + max-over-ranks timing.
+Multi-GPU: one process per GPU (torchrun); each rank is an independent
+replica of the workload (the path has no exchange step): barrier + max over
+ranks of the device-timed region.
 
---impl reference times the CPU oracle (plain C, single thread) on the same
+--impl reference times the CPU oracle (plain C, one thread) on the top-level
 workload: each step is one token through one layer, rotating over a small
 pool of sampled token-layers.
 """
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -34,32 +45,86 @@ sys.path.insert(0, ROOT)
 
 E, TOPK, H, F = 256, 8, 2048, 512
 LAYERS = 40
-EXPERT_BYTES = 1769472  # packed int4 gate/up + down of one expert (36 B per 64 weights)
+EXPERT_BYTES = 1769472  # packed gate/up + down of one expert (36 B per 64 weights, int4 or NVFP4)
 METRIC = "routed-expert tokens/s + HBM GB/s (decode), TFLOP/s (prefill) vs roofline"
+DTYPE_W4 = "int4 weights (f16 scale/min), bf16 activations, fp32 accumulate"
+DTYPE_NV = "nvfp4 weights and activations (e2m1 + e4m3/16 + fp32 global), fp32 accumulate"
 WORKLOAD = ("single-layer decode: 256 experts, top-8, hidden 2048, expert width 512, 1 token per step; "
             "steps rotate over 40 resident int4 layers (18.1 GB) with fresh router logits per layer")
 NV_WORKLOAD = ("NVFP4 single-layer decode: 256 experts, top-8, hidden 2048, expert width 512, 1 token per step; "
                "E2M1 weights with E4M3 scales per 16 channels and fp32 per-matrix globals, x and h quantised "
                "per token/row in the kernel; steps rotate over 40 resident NVFP4 layers (18.1 GB)")
-DTYPE_W4 = "int4 weights (f16 scale/min), bf16 activations, fp32 accumulate"
-# dram__bytes_read.sum + dram__bytes_write.sum of one decode launch at 1 token,
-# from the ncu captures summarised in profiles/ (taken on the current kernels;
-# set to None whenever the kernel changes)
-DECODE_TRAFFIC = {"w4": 14242560, "nvfp4": 14289152}
-DTYPE_NV = "nvfp4 weights and activations (e2m1 + e4m3/16 + fp32 global), fp32 accumulate"
-# the same for the prefill FFN kernels: both launches of one layer at the bench's
-# token count (the bench's first layer), from profiles/prefill_*.md
-PREFILL_TRAFFIC = {"w4": 316057344, "nvfp4": 136497408}
+STREAM_WORKLOAD = ("40-layer decode stream: {T} token(s) per step through 40 chained int4 MoE layers (x of layer l+1 "
+                   "= y of layer l), 256 experts, top-8, hidden 2048, expert width 512, fresh router logits "
+                   "N(0,1) per layer; 18.1 GB resident")
+PREFILL_WORKLOAD = ("grouped prefill: 2048 tokens x top-8 = 16,384 routed rows over 256 experts "
+                    "(router logits N(0,1) + Zipf(1.1) expert bias), hidden 2048, expert width 512; "
+                    "route, permute, tcgen05 grouped FFN, combine; 4 resident layers rotated")
+NVP_WORKLOAD = ("NVFP4 grouped prefill: 512 tokens x top-8 = 4,096 routed rows over 256 experts (router logits "
+                "N(0,1) + Zipf(1.1) expert bias), hidden 2048, expert width 512; route, permute, per-row NVFP4 "
+                "quantisation of the grouped rows, block-scaled tcgen05 grouped FFN, combine; 8 resident layers "
+                "rotated")
+
+# Seeds of the synthetic inputs: weights of the int4 and NVFP4 layer sets,
+# and the activations / logits of each leg (offset by the rank).
+SEED_W4, SEED_NV = 1000, 4000
+SEED_DECODE, SEED_STREAM, SEED_PREFILL, SEED_NVP, SEED_NVD = 1000, 2000, 3000, 4000, 5000
+
+# dram__bytes_read.sum + dram__bytes_write.sum per launch of a kernel, from an
+# ncu capture, with the digest of the kernel's sources at capture time.  A
+# digest that no longer matches the sources makes the bench report null.
+KERNEL_SOURCES = {
+    "decode": ["decode.cu", "common.cuh", "route.cuh", "nvfp4.cuh"],
+    "prefill": ["prefill.cu", "tcgen05.cuh", "common.cuh"],
+    "prefill_nvfp4": ["prefill_nvfp4.cu", "tcgen05.cuh", "common.cuh", "nvfp4.cuh"],
+}
+TRAFFIC = {
+    # key: (kernel, workload) -> {"bytes": per launch (or per launch pair), "sha": digest, "how": ...}
+}
 
 
 # ---------------------------------------------------------------------------- helpers
-def peaks():
+def sources_sha(kernel: str) -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "quantized_moe_route_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_of(key: str, kernel: str):
+    """(bytes, source note): the captured figure if the kernel's sources still
+    have the digest they had at capture time, else (None, why)."""
+    rec = TRAFFIC.get(key)
+    sha = sources_sha(kernel)
+    if rec is None:
+        return None, f"not captured for the current sources (sha {sha})"
+    if rec["sha"] != sha:
+        return None, f"stale: captured on sources {rec['sha']}, current {sha}"
+    return rec["bytes"], f"ncu capture ({rec['how']}) on sources {sha}"
+
+
+def hbm_peak():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            p = json.load(f)
-        return float(p["hbm_gbs"]), "measured"
+            return float(json.load(f)["hbm_gbs"]), "measured"
     except Exception:
         return 6650.0, "fallback"
+
+
+def bf16_peak_sustained():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops_sustained"]), "measured (sustained bf16)"
+    except Exception:
+        return 1400.0, "fallback (sustained bf16)"
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
 
 
 class ClockSampler:
@@ -91,6 +156,7 @@ class ClockSampler:
 
     def __exit__(self, *a):
         if self.proc:
+            time.sleep(0.15)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -144,7 +210,7 @@ def dist_max(v: float) -> float:
     return float(t.item())
 
 
-def job_throughput(units_per_rank: int, world: int, max_ms: float) -> float:
+def job_throughput(units_per_rank: float, world: int, max_ms: float) -> float:
     """Whole-job throughput of independent replicas: every rank's units over
     the slowest rank's time (weak scaling; no data-path exchange)."""
     return units_per_rank * world / (max_ms / 1e3)
@@ -156,15 +222,16 @@ def dist_barrier():
         dist.barrier()
 
 
-# ---------------------------------------------------------------------------- workload
-def build_layers(L, seed, log, fmt="w4"):
-    """Resident layers of packed experts (int4, or NVFP4 with fmt="nvfp4"),
-    generated, quantised and packed on the GPU."""
+def unique_experts(logits: np.ndarray, k: int = TOPK) -> int:
+    return len(set(np.argsort(-logits, axis=1, kind="stable")[:, :k].ravel().tolist()))
+
+
+# ---------------------------------------------------------------------------- layers
+def build_layers(L, seed, log):
+    """Resident int4 layers, generated, quantised and packed on the GPU."""
     import torch
     import synth
     import quantized_moe_route_b200 as moe
-    if fmt == "nvfp4":
-        return build_layers_nvfp4(L, seed, log)
     gu_b, d_b = moe.moe_w4_packed_bytes(2 * F, H), moe.moe_w4_packed_bytes(H, F)
     chunk = 32
     tmp = torch.empty((chunk, 2 * F, H), dtype=torch.float32, device="cuda")
@@ -193,7 +260,7 @@ def build_layers(L, seed, log, fmt="w4"):
         layers.append((gu, dn, moe.make_layer(E, H, F, gu, dn)))
     torch.cuda.synchronize()
     del tmp, codes, sc, mn
-    log(f"built {L} layers in {time.time() - t0:.1f}s")
+    log(f"built {L} int4 layers in {time.time() - t0:.1f}s")
     return layers
 
 
@@ -239,300 +306,352 @@ def layer_inputs(seed, l, T):
     return x, logits
 
 
-def pipelined_e2e(torch, dev, stream, run_step, host_in, T, H, E, K, W, nl):
-    """End-to-end time (ms) of K stream-ordered steps through the C ABI
-    with host buffers.  Every step copies its inputs (x then the logits, one
-    pinned buffer per layer) host -> device and its result y device -> host.
-    The copies run on two copy streams beside the neighbouring steps' kernels;
-    device inputs and outputs are double-buffered, and the kernels stay in
-    order on `stream`.  Returns the H2D bytes per step too."""
-    xb = T * H * 2
-    nbytes = host_in[0].numel()
-    dxl = [torch.empty(nbytes, dtype=torch.uint8, device=dev) for _ in range(2)]
-    dx = [b[:xb].view(torch.int16).view(T, H) for b in dxl]
-    dl = [b[xb:].view(torch.float32).view(T, E) for b in dxl]
-    dy = [torch.empty((T, H), dtype=torch.int16, device=dev) for _ in range(2)]
-    hy = [torch.empty((T, H), dtype=torch.int16).pin_memory() for _ in range(2)]
-    cs, ds = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_k = [torch.cuda.Event() for _ in range(2)]
-    ev_out = [torch.cuda.Event() for _ in range(2)]
+# ---------------------------------------------------------------------------- timing
+class Ctx:
+    """Per-process state shared by the legs: distributed setup, device,
+    stream, and the resident layer sets (built once)."""
 
-    def steps(n, first):
-        cs.wait_stream(stream)
-        ds.wait_stream(stream)
-        for i in range(n):
-            l, b = (first + i) % nl, i % 2
-            if i >= 2:
-                cs.wait_event(ev_k[b])  # the step that read this input buffer is done
-            with torch.cuda.stream(cs):
-                dxl[b].copy_(host_in[l], non_blocking=True)
-                ev_in[b].record(cs)
-            stream.wait_event(ev_in[b])
-            if i >= 2:
-                stream.wait_event(ev_out[b])  # this output buffer's last result has been read
-            with torch.cuda.stream(stream):
-                run_step(l, dx[b], dl[b], dy[b])
-            ev_k[b].record(stream)
-            ds.wait_event(ev_k[b])
-            with torch.cuda.stream(ds):
-                hy[b].copy_(dy[b], non_blocking=True)
-                ev_out[b].record(ds)
-        stream.wait_stream(cs)
-        stream.wait_stream(ds)
+    def __init__(self, args, log):
+        import torch
+        self.args, self.log = args, log
+        self.world, self.rank, self.local = dist_setup()
+        torch.cuda.set_device(self.local)
+        self.dev = torch.device("cuda", self.local)
+        self.stream = torch.cuda.Stream(device=self.dev)
+        self._w4, self._nv = None, None
 
-    steps(2, 0)
-    torch.cuda.synchronize()
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a0.record(stream)
-    steps(K, W)
-    a1.record(stream)
-    a1.synchronize()
-    return a0.elapsed_time(a1), nbytes
+    def w4_layers(self):
+        if self._w4 is None:
+            self._w4 = build_layers(self.args.layers, SEED_W4 + self.rank, self.log)
+        return self._w4
+
+    def nv_layers(self):
+        if self._nv is None:
+            self._nv = build_layers_nvfp4(self.args.layers, SEED_NV + self.rank, self.log)
+        return self._nv
+
+    def capture(self, fn, first, n, events=None):
+        """One CUDA graph of steps first .. first + n - 1 (fn(i) enqueues step i)."""
+        import torch
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.stream):
+            for i in range(n):
+                if events is None:
+                    fn(first + i)
+                else:
+                    fn(first + i, events[i])
+        return g
+
+    def graphs(self, fn, first, K):
+        """Exactly K steps as graphs of at most --graph-steps steps."""
+        G = max(1, min(K, self.args.graph_steps))
+        out, i = [], 0
+        while i < K:
+            n = min(G, K - i)
+            out.append(self.capture(fn, first + i, n))
+            i += n
+        return out
+
+    def replay(self, graphs):
+        import torch
+        with torch.cuda.stream(self.stream):
+            for g in graphs:
+                g.replay()
+
+    def timed(self, fn, K, W, n_resident, eager_touch=True):
+        """Device time (ms, max over ranks) of exactly K steps W .. W + K - 1,
+        after every resident layer has been touched (untimed) and W warm-up
+        steps.  Returns (ms, clock summary)."""
+        import torch
+        if eager_touch:
+            with torch.cuda.stream(self.stream):
+                for i in range(n_resident):
+                    fn(i)
+        g_warm = self.graphs(fn, 0, max(W, n_resident))
+        g_main = self.graphs(fn, W, K)
+        self.replay(g_warm)
+        torch.cuda.synchronize()
+        dist_barrier()
+        with ClockSampler(self.local) as clk:
+            torch.cuda.synchronize()
+            dist_barrier()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(self.stream)
+            self.replay(g_main)
+            e1.record(self.stream)
+            e1.synchronize()
+            torch.cuda.synchronize()
+            dist_barrier()
+        ms = dist_max(e0.elapsed_time(e1))
+        del g_warm, g_main
+        return ms, clk.summary()
+
+    def e2e(self, run_step, host_in, out_shape, K, W, nl):
+        """End-to-end time (ms, max over ranks) of K stream-ordered steps through
+        the C ABI with host buffers: every step copies its inputs (one pinned
+        buffer) host -> device and its result device -> host.  The copies run
+        on two copy streams beside the neighbouring steps' kernels; device
+        inputs and outputs are double-buffered and the kernels stay in order
+        on the compute stream.  run_step(i, d_in, d_out) enqueues step i.
+        Returns (ms, h2d bytes per step, d2h bytes per step)."""
+        import torch
+        dev, stream = self.dev, self.stream
+        nbytes = host_in[0].numel()
+        din = [torch.empty(nbytes, dtype=torch.uint8, device=dev) for _ in range(2)]
+        dout = [torch.empty(out_shape, dtype=torch.int16, device=dev) for _ in range(2)]
+        hout = [torch.empty(out_shape, dtype=torch.int16).pin_memory() for _ in range(2)]
+        cs, ds = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_k = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+
+        def steps(n, first):
+            cs.wait_stream(stream)
+            ds.wait_stream(stream)
+            for i in range(n):
+                l, b = (first + i) % nl, i % 2
+                if i >= 2:
+                    cs.wait_event(ev_k[b])  # the step that read this input buffer is done
+                with torch.cuda.stream(cs):
+                    din[b].copy_(host_in[l], non_blocking=True)
+                    ev_in[b].record(cs)
+                stream.wait_event(ev_in[b])
+                if i >= 2:
+                    stream.wait_event(ev_out[b])  # this output buffer's last result has been read
+                with torch.cuda.stream(stream):
+                    run_step(first + i, din[b], dout[b])
+                ev_k[b].record(stream)
+                ds.wait_event(ev_k[b])
+                with torch.cuda.stream(ds):
+                    hout[b].copy_(dout[b], non_blocking=True)
+                    ev_out[b].record(ds)
+            stream.wait_stream(cs)
+            stream.wait_stream(ds)
+
+        def capture(n, first):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                steps(n, first)
+            return g
+
+        with torch.cuda.stream(stream):
+            steps(3, 0)
+        stream.synchronize()
+        G = max(1, min(K, self.args.graph_steps))
+        gs, i = [], 0
+        while i < K:
+            n = min(G, K - i)
+            gs.append(capture(n, W + i))
+            i += n
+        self.replay(gs)
+        torch.cuda.synchronize()
+        dist_barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        self.replay(gs)
+        a1.record(stream)
+        a1.synchronize()
+        ms = dist_max(a0.elapsed_time(a1))
+        del gs
+        d2h = int(np.prod(out_shape)) * 2
+        return ms, nbytes, d2h
 
 
-def pinned_inputs(torch, x_list, lg_list):
-    """One pinned host buffer per layer: the bf16 activations, then the fp32 logits."""
-    out = []
-    for x, lg in zip(x_list, lg_list):
-        xb = np.ascontiguousarray(x).view(np.uint8).reshape(-1)
-        lb = np.ascontiguousarray(lg, dtype=np.float32).view(np.uint8).reshape(-1)
-        buf = torch.empty(xb.size + lb.size, dtype=torch.uint8).pin_memory()
-        buf[:xb.size].copy_(torch.from_numpy(xb))
-        buf[xb.size:].copy_(torch.from_numpy(lb))
-        out.append(buf)
+def pinned(torch, arrays):
+    """One pinned host buffer holding the raw bytes of the arrays, in order."""
+    parts = [np.ascontiguousarray(a).view(np.uint8).reshape(-1) for a in arrays]
+    n = sum(p.size for p in parts)
+    buf = torch.empty(n, dtype=torch.uint8).pin_memory()
+    o = 0
+    for p in parts:
+        buf[o:o + p.size].copy_(torch.from_numpy(p))
+        o += p.size
+    return buf
+
+
+def views(buf, specs):
+    """Typed views of a device byte buffer: specs = [(torch dtype, shape), ...]."""
+    out, o = [], 0
+    for dt, shape in specs:
+        n = int(np.prod(shape)) * dt.itemsize
+        out.append(buf[o:o + n].view(dt).view(*shape))
+        o += n
     return out
 
 
-def run_gpu(args, log):
-    global LAYERS
-    LAYERS = args.layers
+def hbm_roofline(alg_bytes, dur_ms, kernel, traffic_key, src_kernel, extra=None):
+    peak, peak_kind = hbm_peak()
+    achieved = alg_bytes / (dur_ms / 1e3) / 1e9
+    traffic, tsrc = traffic_of(traffic_key, src_kernel)
+    r = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+         "traffic": traffic, "traffic_source": tsrc, "kernel": kernel, "peak_kind": peak_kind,
+         "alg_bytes_per_launch": alg_bytes, "avg_launch_us": dur_ms * 1e3}
+    if extra:
+        r.update(extra)
+    return r
+
+
+# ---------------------------------------------------------------------------- legs
+def leg_decode(ctx, fmt, T):
+    """Single-layer decode, T tokens per step, one fused launch per step."""
     import torch
     import quantized_moe_route_b200 as moe
-    world, rank, local = dist_setup()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    T = args.tokens
-    seed = 1000 + rank
-    fmt = "nvfp4" if args.workload == "nvfp4-decode" else "w4"
-    layers = build_layers(LAYERS, seed, log, fmt)
-    decode_layer = moe.moe_decode_layer_nvfp4 if fmt == "nvfp4" else moe.moe_decode_layer_w4a16
-    k = TOPK
-    # per-layer device inputs (activations and router logits of every layer)
-    xs, ls, uniq = [], [], []
-    for l in range(LAYERS):
+    args, k = ctx.args, TOPK
+    layers = ctx.nv_layers() if fmt == "nvfp4" else ctx.w4_layers()
+    nl = len(layers)
+    call = moe.moe_decode_layer_nvfp4 if fmt == "nvfp4" else moe.moe_decode_layer_w4a16
+    seed = (SEED_NVD if fmt == "nvfp4" else SEED_DECODE) + ctx.rank
+    xs, ls, uniq, host = [], [], [], []
+    for l in range(nl):
         x, lg = layer_inputs(seed, l, T)
-        xs.append(torch.from_numpy(x.view(np.int16)).to(dev))
-        ls.append(torch.from_numpy(lg).to(dev))
-        uniq.append(len(set(np.argsort(-lg, axis=1, kind="stable")[:, :k].ravel().tolist())))
-    y = torch.empty((T, H), dtype=torch.int16, device=dev)
-    ws = torch.zeros(moe.moe_decode_layer_workspace_bytes(T, k, H, F), dtype=torch.uint8, device=dev)
-    stream = torch.cuda.Stream(device=dev)
+        xs.append(torch.from_numpy(x.view(np.int16)).to(ctx.dev))
+        ls.append(torch.from_numpy(lg).to(ctx.dev))
+        uniq.append(unique_experts(lg))
+        host.append(pinned(torch, [x, lg]))
+    y = torch.empty((T, H), dtype=torch.int16, device=ctx.dev)
+    ws = torch.zeros(moe.moe_decode_layer_workspace_bytes(T, k, H, F), dtype=torch.uint8, device=ctx.dev)
+    stream = ctx.stream
 
-    def step(l, ev=None):
-        # one launch: route + weight-streaming expert FFN + combine
+    def step(i, ev=None):
+        l = i % nl
         if ev is not None:
             ev[0].record(stream)
-        decode_layer(layers[l][2], xs[l], ls[l], k, y, ws, stream=stream)
+        call(layers[l][2], xs[l], ls[l], k, y, ws, stream=stream)
         if ev is not None:
             ev[1].record(stream)
 
-    def capture(fn, steps, first, events=None):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for i in range(steps):
-                if events is None:
-                    fn((first + i) % LAYERS)
-                else:
-                    fn((first + i) % LAYERS, events[i])
-        return g
-
-    def run_steps(fn, K, first):
-        """Exactly K steps: full graphs of G steps plus one remainder graph."""
-        G = min(K, args.graph_steps)
-        graphs = []
-        if K // G:
-            graphs.append((capture(fn, G, first), K // G))
-        if K % G:
-            graphs.append((capture(fn, K % G, first + (K // G) * G), 1))
-        return graphs
-
-    def replay(graphs):
-        with torch.cuda.stream(stream):  # a graph replays on the current stream
-            for g, n in graphs:
-                for _ in range(n):
-                    g.replay()
-
     K, W = args.steps, args.warmup
-    for l in range(min(W, LAYERS)):  # eager first touches, untimed
-        step(l)
-    torch.cuda.synchronize()
-    g_warm = run_steps(step, W, 0)
-    g_main = run_steps(step, K, W)
-    replay(g_warm)
-    torch.cuda.synchronize()
-
-    dist_barrier()
-    with ClockSampler(local) as clk:
-        torch.cuda.synchronize()
-        dist_barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        replay(g_main)
-        e1.record(stream)
-        e1.synchronize()
-        torch.cuda.synchronize()
-        dist_barrier()
-    ms = dist_max(e0.elapsed_time(e1))
-    tokens = K * T * world
-    value = job_throughput(K * T, world, ms)
-
-    # Each step is exactly one launch of the decode kernel, so the timed
-    # region over K is that kernel's average launch duration (back to back,
-    # PDL overlap included).  For reference, a second pass brackets every
-    # launch with its own events (which serialises the launches).
+    ms, clocks = ctx.timed(step, K, W, nl)
+    value = job_throughput(K * T, ctx.world, ms)
+    # each step is one launch, so the timed region over K is the kernel's
+    # average launch duration (back to back, PDL overlap included); a second
+    # pass brackets every launch with its own events (serialising them)
     P = min(K, args.graph_steps)
     evs = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
            for _ in range(P)]
-    g_prof = capture(step, P, W, evs)
-    with torch.cuda.stream(stream):
-        g_prof.replay()
+    g = ctx.capture(step, W, P, evs)
+    ctx.replay([g])
     torch.cuda.synchronize()
     isolated_ms = sum(a.elapsed_time(b) for a, b in evs) / P
+    del g
     dur_ms = ms / K
-    # streamed expert bytes + activations + logits in, y out (timed steps)
-    alg_bytes = sum(uniq[(W + i) % LAYERS] * EXPERT_BYTES + T * H * 2 + T * E * 4 + T * H * 2
-                    for i in range(K)) / K
-    peak, peak_kind = peaks()
-    achieved = alg_bytes / (dur_ms / 1e3) / 1e9
+    alg = sum(uniq[(W + i) % nl] * EXPERT_BYTES + T * H * 2 + T * E * 4 + T * H * 2 for i in range(K)) / K
+    kname = f"moe::decode_kernel<{'nvfp4' if fmt == 'nvfp4' else 'int4'}, fused>"
+    roof = hbm_roofline(alg, dur_ms, kname, f"decode_{fmt}_T{T}", "decode",
+                        {"isolated_launch_us": isolated_ms * 1e3})
 
-    # end to end through the C ABI with host buffers: every step copies its
-    # inputs (x and the logits, one pinned buffer) host -> device and its
-    # result y device -> host.  The copies run on two copy streams and
-    # overlap the neighbouring steps' kernels (double-buffered device inputs
-    # and outputs); the kernels stay in order on the decode stream.
-    xl_bytes = T * H * 2 + T * E * 4
-    hxl = []
-    for l in range(LAYERS):
-        x, lg = layer_inputs(seed, l, T)
-        buf = torch.empty(xl_bytes, dtype=torch.uint8).pin_memory()
-        buf[:T * H * 2].copy_(torch.from_numpy(x.view(np.uint8).reshape(-1)))
-        buf[T * H * 2:].copy_(torch.from_numpy(lg.view(np.uint8).reshape(-1)))
-        hxl.append(buf)
-    hy = [torch.empty((T, H), dtype=torch.int16).pin_memory() for _ in range(2)]
-    dxl = [torch.empty(xl_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
-    dx = [b[:T * H * 2].view(torch.int16).view(T, H) for b in dxl]
-    dl = [b[T * H * 2:].view(torch.float32).view(T, E) for b in dxl]
-    dy = [torch.empty((T, H), dtype=torch.int16, device=dev) for _ in range(2)]
-    cs, ds = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_k = [torch.cuda.Event() for _ in range(2)]
-    ev_out = [torch.cuda.Event() for _ in range(2)]
+    xb = T * H * 2
 
-    def e2e_steps(n, first):
-        cs.wait_stream(stream)
-        ds.wait_stream(stream)
-        for i in range(n):
-            l, b = (first + i) % LAYERS, i % 2
-            if i >= 2:
-                cs.wait_event(ev_k[b])  # the kernel that read this input buffer is done
-            with torch.cuda.stream(cs):
-                dxl[b].copy_(hxl[l], non_blocking=True)
-                ev_in[b].record(cs)
-            stream.wait_event(ev_in[b])
-            if i >= 2:
-                stream.wait_event(ev_out[b])  # this output buffer's last result has been read
-            decode_layer(layers[l][2], dx[b], dl[b], k, dy[b], ws, stream=stream)
-            ev_k[b].record(stream)
-            ds.wait_event(ev_k[b])
-            with torch.cuda.stream(ds):
-                hy[b].copy_(dy[b], non_blocking=True)
-                ev_out[b].record(ds)
-        stream.wait_stream(cs)
-        stream.wait_stream(ds)
+    def e2e_step(i, din, dout):
+        l = i % nl
+        x_d, l_d = views(din, [(torch.int16, (T, H)), (torch.float32, (T, E))])
+        call(layers[l][2], x_d, l_d, k, dout, ws, stream=stream)
 
-    def capture_e2e(n, first):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            e2e_steps(n, first)
-        return g
-
-    with torch.cuda.stream(stream):
-        e2e_steps(3, 0)
-    stream.synchronize()
-    Ge = min(K, args.graph_steps)
-    g_e2e = []
-    if K // Ge:
-        g_e2e.append((capture_e2e(Ge, W), K // Ge))
-    if K % Ge:
-        g_e2e.append((capture_e2e(K % Ge, W + (K // Ge) * Ge), 1))
-    replay(g_e2e)
-    torch.cuda.synchronize()
-    dist_barrier()
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a0.record(stream)
-    replay(g_e2e)
-    a1.record(stream)
-    a1.synchronize()
-    e2e_ms = dist_max(a0.elapsed_time(a1))
-    e2e_value = tokens / (e2e_ms / 1e3)
-
+    e2e_ms, h2d, d2h = ctx.e2e(e2e_step, host, (T, H), K, W, nl)
+    assert h2d == xb + T * E * 4
     out = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ctx.world, "steps": K, "warmup": W,
         "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": DTYPE_NV if fmt == "nvfp4" else DTYPE_W4, "data": "synthetic",
         "config": {"workload": NV_WORKLOAD if fmt == "nvfp4" else WORKLOAD, "experts": E, "top_k": k, "hidden": H,
-                   "expert_width": F, "tokens_per_step": T, "resident_layers": LAYERS, "seed": 1000,
-                   "l2": f"inputs larger than L2 ({LAYERS}-layer rotation, {LAYERS * E * EXPERT_BYTES / 1e9:.1f} GB)",
-                   "parallelism": f"replicas x{world}",
+                   "expert_width": F, "tokens_per_step": T, "resident_layers": nl, "seed": seed - ctx.rank,
+                   "l2": f"inputs larger than L2 ({nl}-layer rotation, {nl * E * EXPERT_BYTES / 1e9:.1f} GB); "
+                         f"every resident layer touched before timing",
+                   "parallelism": f"replicas x{ctx.world}",
                    "launch": f"one kernel per step (route + FFN + combine), CUDA graphs of "
                              f"{min(K, args.graph_steps)} steps, programmatic dependent launch"},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak,
-                     "traffic": DECODE_TRAFFIC.get(fmt) if T == 1 else None,
-                     "traffic_source": ("ncu capture, one launch at 1 token: profiles/decode_kernel_"
-                                        + ("nvfp4_" if fmt == "nvfp4" else "") + "single_layer_T1.md")
-                     if T == 1 else "not captured at this batch size",
-                     "kernel": f"moe::decode_kernel<{'nvfp4' if fmt == 'nvfp4' else 'int4'}, fused>",
-                     "peak_kind": peak_kind, "alg_bytes_per_launch": alg_bytes,
-                     "avg_launch_us": dur_ms * 1e3, "isolated_launch_us": isolated_ms * 1e3},
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": xl_bytes,
-                "d2h_bytes_per_step": T * H * 2,
+        "roofline": roof,
+        "e2e": {"value": job_throughput(K * T, ctx.world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
                 "overlap": "each step's copies run on copy streams beside the neighbouring steps' kernels"},
         "gpu_launches": K,
-        "clocks": clk.summary(),
+        "clocks": clocks,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(seed, T, budget_s=args.cpu_seconds, log=log, fmt=fmt)
-    del g_main, g_warm, g_prof, g_e2e
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-        dist.destroy_process_group()
-    return out if rank == 0 else None
+    return out
 
 
-PREFILL_WORKLOAD = ("grouped prefill: 2048 tokens x top-8 = 16,384 routed rows over 256 experts "
-                    "(router logits N(0,1) + Zipf(1.1) expert bias), hidden 2048, expert width 512; "
-                    "route, permute, tcgen05 grouped FFN, combine; 4 resident layers rotated")
-
-
-def run_gpu_prefill(args, log):
+def leg_stream(ctx, T):
+    """40 chained layers per step: layer l reads the previous layer's y."""
     import torch
     import synth
     import quantized_moe_route_b200 as moe
-    world, rank, local = dist_setup()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    T, k, nl = args.tokens, TOPK, args.layers
-    seed = 3000 + rank
-    layers = build_layers(nl, seed, log)
+    args, k = ctx.args, TOPK
+    layers = ctx.w4_layers()
+    nl = len(layers)
+    seed = SEED_STREAM + ctx.rank
+    x0 = synth.activations_bf16(seed, 0, T, H)
+    lgs = np.stack([synth.router_logits(seed, l, T, E) for l in range(nl)])  # [nl][T][E]
+    uniq = [unique_experts(lgs[l]) for l in range(nl)]
+    d_x0 = torch.from_numpy(x0.view(np.int16)).to(ctx.dev)
+    d_lg = torch.from_numpy(lgs).to(ctx.dev)
+    ys = [torch.empty((T, H), dtype=torch.int16, device=ctx.dev) for _ in range(nl)]
+    ws = torch.zeros(moe.moe_decode_layer_workspace_bytes(T, k, H, F), dtype=torch.uint8, device=ctx.dev)
+    stream = ctx.stream
+
+    def chain(x_in, lg, y_out):
+        for l in range(nl):
+            moe.moe_decode_layer_w4a16(layers[l][2], x_in if l == 0 else ys[l - 1], lg[l], k,
+                                       y_out if l == nl - 1 else ys[l], ws, stream=stream)
+
+    def step(i):
+        chain(d_x0, d_lg, ys[-1])
+
+    K, W = args.steps, args.warmup
+    ms, clocks = ctx.timed(step, K, W, 1)
+    value = job_throughput(K * T, ctx.world, ms)
+    step_ms = ms / K
+    bytes_step = sum(u * EXPERT_BYTES for u in uniq) + nl * (T * H * 2 + T * E * 4 + T * H * 2)
+    roof = hbm_roofline(bytes_step / nl, step_ms / nl, "moe::decode_kernel<int4, fused>", f"decode_w4_T{T}",
+                        "decode", {"alg_bytes_per_step": bytes_step, "unique_expert_bytes_per_step":
+                                   sum(u * EXPERT_BYTES for u in uniq), "launches_per_step": nl})
+    host = [pinned(torch, [x0, lgs])]
+
+    def e2e_step(i, din, dout):
+        x_d, l_d = views(din, [(torch.int16, (T, H)), (torch.float32, (nl, T, E))])
+        chain(x_d, l_d, dout)
+
+    e2e_ms, h2d, d2h = ctx.e2e(e2e_step, host, (T, H), K, W, 1)
+    return {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "ms_per_step": step_ms, "steps": K, "warmup": W,
+        "dtype": DTYPE_W4,
+        "unique_expert_gbs": sum(u * EXPERT_BYTES for u in uniq) / (step_ms / 1e3) / 1e9,
+        "config": {"workload": STREAM_WORKLOAD.format(T=T), "tokens_per_step": T, "layers_per_step": nl,
+                   "unique_experts_per_layer_mean": float(np.mean(uniq)), "seed": SEED_STREAM,
+                   "l2": f"inputs larger than L2 ({bytes_step / 1e6:.0f} MB of experts per step)",
+                   "launch": f"{nl} kernels per step (one per layer), CUDA graphs, programmatic dependent launch"},
+        "roofline": roof,
+        "e2e": {"value": job_throughput(K * T, ctx.world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "overlap": "each step's copies run on copy streams beside the neighbouring steps' kernels"},
+        "gpu_launches": nl * K,
+        "clocks": clocks,
+    }
+
+
+def _prefill_inputs(seed, T, nl, ctx):
+    import torch
+    import synth
     bias = synth.zipf_bias(seed, E)
-    xs, ls = [], []
+    xs, ls, host, uniq = [], [], [], []
     for l in range(nl):
-        xs.append(torch.from_numpy(synth.activations_bf16(seed, l, T, H).view(np.int16)).to(dev))
-        ls.append(torch.from_numpy((synth.router_logits(seed, l, T, E) + bias[None, :]).astype(np.float32)).to(dev))
+        x = synth.activations_bf16(seed, l, T, H)
+        lg = (synth.router_logits(seed, l, T, E) + bias[None, :]).astype(np.float32)
+        xs.append(torch.from_numpy(x.view(np.int16)).to(ctx.dev))
+        ls.append(torch.from_numpy(lg).to(ctx.dev))
+        host.append(pinned(torch, [x, lg]))
+        uniq.append(unique_experts(lg))
+    return xs, ls, host, uniq
+
+
+def leg_prefill(ctx, T=2048, nl=4):
+    import torch
+    import quantized_moe_route_b200 as moe
+    args, k = ctx.args, TOPK
+    layers = ctx.w4_layers()[:nl]
+    seed = SEED_PREFILL + ctx.rank
+    xs, ls, host, _ = _prefill_inputs(seed, T, nl, ctx)
     R = T * k
+    dev = ctx.dev
     idx = torch.empty((T, k), dtype=torch.int32, device=dev)
     w = torch.empty((T, k), dtype=torch.float32, device=dev)
     counts = torch.empty(E, dtype=torch.int32, device=dev)
@@ -544,121 +663,73 @@ def run_gpu_prefill(args, log):
     y_perm = torch.empty((R, H), dtype=torch.int16, device=dev)
     fws = torch.empty(moe.moe_prefill_workspace_bytes(R, F), dtype=torch.uint8, device=dev)
     y = torch.empty((T, H), dtype=torch.int16, device=dev)
-    stream = torch.cuda.Stream(device=dev)
+    stream = ctx.stream
 
-    def step(l, ev=None, xin=None, lin=None, yout=None):
-        moe.moe_route(ls[l] if lin is None else lin, k, idx, w, stream=stream)
-        moe.moe_permute(idx, E, counts, offsets, sorted_rows, inv, pws, x=xs[l] if xin is None else xin,
-                        x_perm=x_perm, stream=stream)
+    def run(l, x, lg, yout, ev=None):
+        moe.moe_route(lg, k, idx, w, stream=stream)
+        moe.moe_permute(idx, E, counts, offsets, sorted_rows, inv, pws, x=x, x_perm=x_perm, stream=stream)
         if ev is not None:
             ev[0].record(stream)
         moe.moe_ffn_grouped_prefill(layers[l][2], x_perm, offsets, y_perm, fws, stream=stream)
         if ev is not None:
             ev[1].record(stream)
-        moe.moe_unpermute_combine(y_perm, w, y if yout is None else yout, inv=inv, stream=stream)
+        moe.moe_unpermute_combine(y_perm, w, yout, inv=inv, stream=stream)
+
+    def step(i, ev=None):
+        l = i % nl
+        run(l, xs[l], ls[l], y, ev)
 
     K, W = args.steps, args.warmup
-    with torch.cuda.stream(stream):
-        for i in range(W):
-            step(i % nl)
-    torch.cuda.synchronize()
-    dist_barrier()
-    with ClockSampler(local) as clk:
-        torch.cuda.synchronize()
-        dist_barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for i in range(K):
-                step((W + i) % nl)
-            e1.record(stream)
-        e1.synchronize()
-        torch.cuda.synchronize()
-        dist_barrier()
-    ms = dist_max(e0.elapsed_time(e1))
-    tokens = K * T * world
-    value = job_throughput(K * T, world, ms)
-
-    # kernel-duration pass: events around the two grouped-GEMM launches
+    ms, clocks = ctx.timed(step, K, W, nl)
+    value = job_throughput(K * T, ctx.world, ms)
     P = min(K, 50)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(P)]
-    with torch.cuda.stream(stream):
-        for i in range(P):
-            step((W + i) % nl, evs[i])
+    evs = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+           for _ in range(P)]
+    g = ctx.capture(step, W, P, evs)
+    ctx.replay([g])
     torch.cuda.synchronize()
     dur_ms = sum(a.elapsed_time(b) for a, b in evs) / P
+    del g
     flops = R * 6.0 * H * F
     achieved = flops / (dur_ms / 1e3) / 1e12
-    try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            peak, peak_kind = float(json.load(f)["bf16_tflops_sustained"]), "measured (sustained bf16)"
-    except Exception:
-        peak, peak_kind = 1400.0, "fallback (sustained bf16)"
+    peak, peak_kind = bf16_peak_sustained()
+    traffic, tsrc = traffic_of("prefill_w4_2048", "prefill")
 
-    # end to end: each step copies x and the logits (one pinned buffer) in and
-    # y out, on copy streams beside the neighbouring steps' kernels
-    import synth as _s
-    host_in = pinned_inputs(torch, [_s.activations_bf16(seed, l, T, H) for l in range(nl)],
-                            [_s.router_logits(seed, l, T, E) + bias[None, :] for l in range(nl)])
-    e2e_ms, h2d_bytes = pipelined_e2e(torch, dev, stream,
-                                      lambda l, xin, lin, yout: step(l, xin=xin, lin=lin, yout=yout),
-                                      host_in, T, H, E, K, W, nl)
-    e2e_ms = dist_max(e2e_ms)
+    def e2e_step(i, din, dout):
+        x_d, l_d = views(din, [(torch.int16, (T, H)), (torch.float32, (T, E))])
+        run(i % nl, x_d, l_d, dout)
 
-    out = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
-        "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "int4 weights (f16 scale/min), bf16 activations, fp32 accumulate", "data": "synthetic",
-        "config": {"workload": PREFILL_WORKLOAD, "experts": E, "top_k": k, "hidden": H, "expert_width": F,
-                   "tokens_per_step": T, "routed_rows": R, "resident_layers": nl,
-                   "l2": "inputs larger than L2 (453 MB of experts per layer, 67 MB permuted rows)",
-                   "parallelism": f"replicas x{world}", "launch": "stream-ordered, PDL into the FFN kernels"},
+    e2e_ms, h2d, d2h = ctx.e2e(e2e_step, host, (T, H), K, W, nl)
+    return {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "ms_per_step": ms / K, "steps": K, "warmup": W,
+        "dtype": DTYPE_W4,
+        "config": {"workload": PREFILL_WORKLOAD, "tokens_per_step": T, "routed_rows": R, "resident_layers": nl,
+                   "seed": SEED_PREFILL,
+                   "l2": "inputs larger than L2 (up to 453 MB of experts per layer, 67 MB permuted rows)",
+                   "launch": "stream-ordered, programmatic dependent launch through the chain, CUDA graphs"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": PREFILL_TRAFFIC["w4"],
-                     "traffic_source": "ncu capture of the gate/up and down launches of one layer (2048 tokens): "
-                                       "profiles/prefill_kernel_grouped_2048tok.md",
+                     "frac": achieved / peak, "traffic": traffic, "traffic_source": tsrc,
                      "kernel": "moe::prefill_kernel (gate/up + down launches)", "peak_kind": peak_kind,
                      "alg_flop_per_launch_pair": flops, "avg_pair_us": dur_ms * 1e3},
-        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d_bytes,
-                "d2h_bytes_per_step": T * H * 2,
+        "e2e": {"value": job_throughput(K * T, ctx.world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
                 "overlap": "each step's copies run on copy streams beside the neighbouring steps' kernels"},
         "gpu_launches": 8 * K,  # route, histogram, scan, scatter, gather, gate/up, down, combine
-        "clocks": clk.summary(),
+        "clocks": clocks,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline_prefill(seed, bias, budget_s=args.cpu_seconds, log=log)
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-        dist.destroy_process_group()
-    return out if rank == 0 else None
 
 
-NVP_WORKLOAD = ("NVFP4 grouped prefill: 512 tokens x top-8 = 4,096 routed rows over 256 experts (router logits "
-                "N(0,1) + Zipf(1.1) expert bias), hidden 2048, expert width 512; route, permute, per-row NVFP4 "
-                "quantisation of the grouped rows, block-scaled tcgen05 grouped FFN, combine; 8 resident layers rotated")
-
-
-def run_gpu_prefill_nvfp4(args, log):
+def leg_prefill_nvfp4(ctx, T=512, nl=8):
     """Config 5's prefill leg: HBM-bound (the touched experts' 4.5-bit weights
     dominate the bytes; the FP4 tensor cores need a few microseconds)."""
     import torch
-    import synth
     import quantized_moe_route_b200 as moe
-    world, rank, local = dist_setup()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    T, k, nl = args.tokens, TOPK, args.layers
-    seed = 4000 + rank
-    layers = build_layers(nl, seed, log, "nvfp4")
-    bias = synth.zipf_bias(seed, E)
-    xs, ls, uniq = [], [], []
-    for l in range(nl):
-        xs.append(torch.from_numpy(synth.activations_bf16(seed, l, T, H).view(np.int16)).to(dev))
-        lg = (synth.router_logits(seed, l, T, E) + bias[None, :]).astype(np.float32)
-        ls.append(torch.from_numpy(lg).to(dev))
-        uniq.append(len(set(np.argsort(-lg, axis=1, kind="stable")[:, :k].ravel().tolist())))
+    args, k = ctx.args, TOPK
+    layers = ctx.nv_layers()[:nl]
+    seed = SEED_NVP + ctx.rank
+    xs, ls, host, uniq = _prefill_inputs(seed, T, nl, ctx)
     R = T * k
+    dev = ctx.dev
     idx = torch.empty((T, k), dtype=torch.int32, device=dev)
     w = torch.empty((T, k), dtype=torch.float32, device=dev)
     counts = torch.empty(E, dtype=torch.int32, device=dev)
@@ -672,161 +743,62 @@ def run_gpu_prefill_nvfp4(args, log):
     y_perm = torch.empty((R, H), dtype=torch.int16, device=dev)
     fws = torch.empty(moe.moe_prefill_nvfp4_workspace_bytes(R, F), dtype=torch.uint8, device=dev)
     y = torch.empty((T, H), dtype=torch.int16, device=dev)
-    stream = torch.cuda.Stream(device=dev)
+    stream = ctx.stream
 
-    def step(l, ev=None, xin=None, lin=None, yout=None):
-        moe.moe_route(ls[l] if lin is None else lin, k, idx, w, stream=stream)
+    def run(l, x, lg, yout, ev=None):
+        moe.moe_route(lg, k, idx, w, stream=stream)
         moe.moe_permute(idx, E, counts, offsets, sorted_rows, inv, pws, stream=stream)
-        moe.moe_quantize_nvfp4_rows(xs[l] if xin is None else xin, xc, xsf, xg, src_rows=sorted_rows, src_div=k,
-                                    rows=R, stream=stream)
+        moe.moe_quantize_nvfp4_rows(x, xc, xsf, xg, src_rows=sorted_rows, src_div=k, rows=R, stream=stream)
         if ev is not None:
             ev[0].record(stream)
         moe.moe_ffn_grouped_prefill_nvfp4(layers[l][2], xc, xsf, xg, offsets, y_perm, fws, stream=stream)
         if ev is not None:
             ev[1].record(stream)
-        moe.moe_unpermute_combine(y_perm, w, y if yout is None else yout, inv=inv, stream=stream)
+        moe.moe_unpermute_combine(y_perm, w, yout, inv=inv, stream=stream)
+
+    def step(i, ev=None):
+        l = i % nl
+        run(l, xs[l], ls[l], y, ev)
 
     K, W = args.steps, args.warmup
-    with torch.cuda.stream(stream):
-        for i in range(W):
-            step(i % nl)
-    torch.cuda.synchronize()
-    dist_barrier()
-    with ClockSampler(local) as clk:
-        torch.cuda.synchronize()
-        dist_barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for i in range(K):
-                step((W + i) % nl)
-            e1.record(stream)
-        e1.synchronize()
-        torch.cuda.synchronize()
-        dist_barrier()
-    ms = dist_max(e0.elapsed_time(e1))
-    tokens = K * T * world
-    value = job_throughput(K * T, world, ms)
-
-    # kernel-duration pass: events around the grouped FFN call (gate/up, h
-    # quantisation, down: three launches)
+    ms, clocks = ctx.timed(step, K, W, nl)
+    value = job_throughput(K * T, ctx.world, ms)
     P = min(K, 50)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(P)]
-    with torch.cuda.stream(stream):
-        for i in range(P):
-            step((W + i) % nl, evs[i])
+    evs = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+           for _ in range(P)]
+    g = ctx.capture(step, W, P, evs)
+    ctx.replay([g])
     torch.cuda.synchronize()
     dur_ms = sum(a.elapsed_time(b) for a, b in evs) / P
-    # algorithmic bytes of the call: touched experts' packed weights, the
+    del g
+    # algorithmic bytes of the FFN call: touched experts' packed weights, the
     # quantised rows in, h out (fp32) and back in, its codes out and in, y_perm out
     act = R * (H // 2 + H // 16 + 4)
     hq = R * (F // 2 + F // 16 + 4)
-    alg_bytes = sum(uniq[(W + i) % nl] * EXPERT_BYTES for i in range(P)) / P + act + 2 * R * F * 4 + 2 * hq + R * H * 2
-    peak, peak_kind = peaks()
-    achieved = alg_bytes / (dur_ms / 1e3) / 1e9
+    alg = sum(uniq[(W + i) % nl] * EXPERT_BYTES for i in range(P)) / P + act + 2 * R * F * 4 + 2 * hq + R * H * 2
     flops = R * 6.0 * H * F
+    roof = hbm_roofline(alg, dur_ms, "moe::prefill_nvfp4_kernel (gate/up + h quantise + down launches)",
+                        "prefill_nvfp4_512", "prefill_nvfp4",
+                        {"tflops": flops / (dur_ms / 1e3) / 1e12, "alg_bytes_per_call": alg})
 
-    # end to end: each step copies x and the logits (one pinned buffer) in and
-    # y out, on copy streams beside the neighbouring steps' kernels
-    import synth as _s
-    host_in = pinned_inputs(torch, [_s.activations_bf16(seed, l, T, H) for l in range(nl)],
-                            [_s.router_logits(seed, l, T, E) + bias[None, :] for l in range(nl)])
-    e2e_ms, h2d_bytes = pipelined_e2e(torch, dev, stream,
-                                      lambda l, xin, lin, yout: step(l, xin=xin, lin=lin, yout=yout),
-                                      host_in, T, H, E, K, W, nl)
-    e2e_ms = dist_max(e2e_ms)
+    def e2e_step(i, din, dout):
+        x_d, l_d = views(din, [(torch.int16, (T, H)), (torch.float32, (T, E))])
+        run(i % nl, x_d, l_d, dout)
 
-    out = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
-        "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": DTYPE_NV, "data": "synthetic",
-        "config": {"workload": NVP_WORKLOAD, "experts": E, "top_k": k, "hidden": H, "expert_width": F,
-                   "tokens_per_step": T, "routed_rows": R, "resident_layers": nl,
-                   "l2": f"inputs larger than L2 ({nl} layers x 453 MB of experts rotated)",
-                   "parallelism": f"replicas x{world}", "launch": "stream-ordered, PDL into the FFN kernels"},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": PREFILL_TRAFFIC["nvfp4"],
-                     "traffic_source": "ncu capture of the gate/up and down launches of one layer (512 tokens; "
-                                       "the h quantise launch between them is not included): "
-                                       "profiles/prefill_nvfp4_kernel_grouped_512tok.md",
-                     "kernel": "moe::prefill_nvfp4_kernel (gate/up + h quantise + down launches)",
-                     "peak_kind": peak_kind, "alg_bytes_per_call": alg_bytes, "avg_call_us": dur_ms * 1e3,
-                     "tflops": flops / (dur_ms / 1e3) / 1e12},
-        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d_bytes,
-                "d2h_bytes_per_step": T * H * 2,
+    e2e_ms, h2d, d2h = ctx.e2e(e2e_step, host, (T, H), K, W, nl)
+    return {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "ms_per_step": ms / K, "steps": K, "warmup": W,
+        "dtype": DTYPE_NV,
+        "config": {"workload": NVP_WORKLOAD, "tokens_per_step": T, "routed_rows": R, "resident_layers": nl,
+                   "seed": SEED_NVP, "l2": f"inputs larger than L2 ({nl} layers x up to 453 MB of experts rotated)",
+                   "launch": "stream-ordered, programmatic dependent launch through the chain, CUDA graphs"},
+        "roofline": roof,
+        "e2e": {"value": job_throughput(K * T, ctx.world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
                 "overlap": "each step's copies run on copy streams beside the neighbouring steps' kernels"},
         "gpu_launches": 9 * K,
-        "clocks": clk.summary(),
+        "clocks": clocks,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline_prefill_nvfp4(seed, bias, T, budget_s=args.cpu_seconds, log=log)
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-        dist.destroy_process_group()
-    return out if rank == 0 else None
-
-
-def cpu_baseline_prefill_nvfp4(seed, bias, T, budget_s, log):
-    """The oracle on sampled tokens of the NVFP4 prefill batch (tokens/s)."""
-    import oracle
-    import synth
-    import torch
-    x = synth.activations_bf16(seed, 0, T, H)
-    lg = (synth.router_logits(seed, 0, T, E) + bias[None, :]).astype(np.float32)
-    idx, _ = oracle.route(lg, TOPK)
-    toks = list(range(0, T, 61))[:6]
-    experts = {}
-    for e in sorted(set(idx[toks].ravel().tolist())):
-        wg = torch.empty((1, 2 * F, H), device="cuda")
-        wd = torch.empty((1, H, F), device="cuda")
-        synth.cuda_expert_weights(wg, seed, 0, e, synth.PROJ_GATE_UP)
-        synth.cuda_expert_weights(wd, seed, 0, e, synth.PROJ_DOWN)
-        experts[e] = (oracle_quantize(wg[0].cpu().numpy(), "nvfp4"), oracle_quantize(wd[0].cpu().numpy(), "nvfp4"))
-    t0 = time.time()
-    n = 0
-    while True:
-        t = toks[n % len(toks)]
-        oracle_forward(x[t:t + 1], lg[t:t + 1], experts, "nvfp4")
-        n += 1
-        if time.time() - t0 >= budget_s:
-            break
-    dt = time.time() - t0
-    return {"value": n / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} tokens of the {T}-token NVFP4 prefill batch ({len(toks)} distinct, all 8 experts each), "
-                      f"{dt:.1f}s"}
-
-
-def cpu_baseline_prefill(seed, bias, budget_s, log):
-    """The oracle on sampled tokens of the prefill workload (rows per second
-    scaled to tokens/s); weights of the sampled tokens' experts only."""
-    import oracle
-    import synth
-    T = 2048
-    x = synth.activations_bf16(seed, 0, T, H)
-    lg = (synth.router_logits(seed, 0, T, E) + bias[None, :]).astype(np.float32)
-    idx, _ = oracle.route(lg, TOPK)
-    toks = list(range(0, T, 97))[:8]
-    need = sorted(set(idx[toks].ravel().tolist()))
-    import torch
-    experts = {}
-    for e in need:
-        wg = torch.empty((1, 2 * F, H), device="cuda")
-        wd = torch.empty((1, H, F), device="cuda")
-        synth.cuda_expert_weights(wg, seed, 0, e, synth.PROJ_GATE_UP)
-        synth.cuda_expert_weights(wd, seed, 0, e, synth.PROJ_DOWN)
-        experts[e] = (oracle.quantize_w4(wg[0].cpu().numpy()), oracle.quantize_w4(wd[0].cpu().numpy()))
-    t0 = time.time()
-    n = 0
-    while True:
-        t = toks[n % len(toks)]
-        oracle.moe_forward_w4(x[t:t + 1], lg[t:t + 1], TOPK, experts)
-        n += 1
-        if time.time() - t0 >= budget_s:
-            break
-    dt = time.time() - t0
-    return {"value": n / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} tokens of the 2048-token prefill batch (8 distinct, all 8 experts each), {dt:.1f}s"}
 
 
 # ---------------------------------------------------------------------------- CPU oracle
@@ -851,49 +823,94 @@ def oracle_forward(x, lg, experts, fmt):
     return np.stack(ys)
 
 
-def oracle_pool(seed, T, n, log, use_gpu_generator, fmt="w4"):
-    """n sampled token-layers: canonical weights of their routed experts, built
-    with the seeded generator and the oracle's own quantiser."""
+def oracle_experts(w_seed, layer, experts, fmt):
+    """Canonical weights of the given experts of one layer, drawn with the
+    CPU twin of the seeded generator and quantised by the oracle."""
+    import synth
+    out = {}
+    for e in sorted(set(int(v) for v in experts)):
+        a = synth.expert_weights(w_seed, layer, e, synth.PROJ_GATE_UP, 2 * F, H)
+        b = synth.expert_weights(w_seed, layer, e, synth.PROJ_DOWN, H, F)
+        out[e] = (oracle_quantize(a, fmt), oracle_quantize(b, fmt))
+    return out
+
+
+def oracle_sample(job):
+    """The sample one oracle worker evaluates: a list of (x, logits, experts)
+    token-layers, and the tokens of the leg's unit each evaluation counts for.
+    job = (kind, fmt, w_seed, in_seed, T, worker)."""
     import oracle
     import synth
-    pool = []
-    t0 = time.time()
-    for l in range(n):
-        x, lg = layer_inputs(seed, l, T)
-        idx, _ = oracle.route(lg, TOPK)
-        experts = {}
-        for e in sorted(set(idx.ravel().tolist())):
-            if use_gpu_generator:
-                import torch
-                wg = torch.empty((1, 2 * F, H), device="cuda")
-                wd = torch.empty((1, H, F), device="cuda")
-                synth.cuda_expert_weights(wg, seed, l, e, synth.PROJ_GATE_UP)
-                synth.cuda_expert_weights(wd, seed, l, e, synth.PROJ_DOWN)
-                a, b = wg[0].cpu().numpy(), wd[0].cpu().numpy()
+    kind, fmt, w_seed, in_seed, T, wi = job
+    items = []
+    if kind in ("decode", "stream"):
+        for j in range(2):
+            l = (2 * wi + j) % LAYERS
+            if kind == "stream":
+                x = synth.activations_bf16(in_seed, 0, T, H)  # a layer's input in the chain has this shape
+                lg = synth.router_logits(in_seed, l, T, E)
             else:
-                a = synth.expert_weights(seed, l, e, synth.PROJ_GATE_UP, 2 * F, H)
-                b = synth.expert_weights(seed, l, e, synth.PROJ_DOWN, H, F)
-            experts[e] = (oracle_quantize(a, fmt), oracle_quantize(b, fmt))
-        pool.append((x, lg, experts))
-    log(f"oracle pool of {n} token-layers built in {time.time() - t0:.1f}s")
-    return pool
+                x, lg = layer_inputs(in_seed, l, T)
+            idx, _ = oracle.route(lg, TOPK)
+            items.append((x, lg, oracle_experts(w_seed, l, idx.ravel(), fmt)))
+        # a decode step is one layer of T tokens; a stream step is 40 layers
+        units = T if kind == "decode" else T / LAYERS
+    else:  # prefill: single tokens of the Zipf-routed batch, layer 0
+        bias = synth.zipf_bias(in_seed, E)
+        x = synth.activations_bf16(in_seed, 0, T, H)
+        lg = (synth.router_logits(in_seed, 0, T, E) + bias[None, :]).astype(np.float32)
+        idx, _ = oracle.route(lg, TOPK)
+        for j in range(2):
+            t = (97 * (2 * wi + j) + 13) % T
+            items.append((x[t:t + 1], lg[t:t + 1], oracle_experts(w_seed, 0, idx[t], fmt)))
+        units = 1
+    return items, units
 
 
-def cpu_baseline(seed, T, budget_s, log, fmt="w4"):
-    pool = oracle_pool(seed, T, 4, log, use_gpu_generator=True, fmt=fmt)
-    t0 = time.time()
-    n = 0
+def oracle_worker(job_budget):
+    """Evaluate one worker's sample repeatedly until the shared deadline;
+    returns (units, seconds).  Runs in a spawned process (or in-process for
+    the one-core figure); touches no GPU."""
+    job, deadline = job_budget
+    items, units = oracle_sample(job)
+    fmt = job[1]
+    n, t0 = 0, time.time()
     while True:
-        x, lg, experts = pool[n % len(pool)]
-        oracle_forward(x, lg, experts, fmt)
+        x, lg, ex = items[n % len(items)]
+        oracle_forward(x, lg, ex, fmt)
         n += 1
-        if time.time() - t0 >= budget_s:
+        if time.time() >= deadline and n >= 1:
             break
-    dt = time.time() - t0
-    return {"value": n * T / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} token-layer steps (T={T}) over a pool of {len(pool)} sampled layers, {dt:.1f}s"}
+    return n * units, time.time() - t0
 
 
+def cpu_baseline(kind, fmt, w_seed, in_seed, T, seconds, log, unit="tokens/s"):
+    """The oracle, as it stands, on bounded samples of a leg's workload: one
+    core, then one spawned process per host core (rows of the workload split
+    over processes, each its own sample).  The value is the all-core figure."""
+    import multiprocessing as mp
+    t0 = time.time()
+    u1, s1 = oracle_worker(((kind, fmt, w_seed, in_seed, T, 0), time.time() + seconds))
+    one = u1 / s1
+    n = host_cores()
+    ctxp = mp.get_context("spawn")
+    jobs = [((kind, fmt, w_seed, in_seed, T, i), time.time() + seconds + 6.0) for i in range(n)]
+    with ctxp.Pool(n) as pool:
+        res = pool.map(oracle_worker, jobs, chunksize=1)
+    allc = sum(u / s for u, s in res)
+    log(f"cpu baseline {kind}/{fmt}/T={T}: {one:.3g} (1 core) {allc:.3g} ({n} cores) {unit} "
+        f"in {time.time() - t0:.0f}s")
+    what = {"decode": f"token-layer evaluations (T={T}) over 2 sampled layers per process",
+            "stream": f"layer evaluations of the 40-layer chain (T={T}, a step = 40 of them) over 2 sampled layers "
+                      f"per process",
+            "prefill": f"single tokens of the {T}-token Zipf-routed batch (all 8 experts each), 2 per process"}[kind]
+    return {"value": allc, "unit": unit, "cores": n, "kind": "oracle",
+            "sample": f"{what}; about {seconds:.0f}s per process",
+            "single_core": {"value": one, "cores": 1, "sample": f"{what.split(' per process')[0]}, "
+                                                                 f"{s1:.1f}s on one core"}}
+
+
+# ---------------------------------------------------------------------------- reference arm
 def run_reference(args, log):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -901,7 +918,11 @@ def run_reference(args, log):
         return None
     import oracle
     T = args.tokens
-    pool = oracle_pool(1000, T, 4, log, use_gpu_generator=False)
+    pool = []
+    for l in range(4):
+        x, lg = layer_inputs(SEED_DECODE, l, T)
+        idx, _ = oracle.route(lg, TOPK)
+        pool.append((x, lg, oracle_experts(SEED_W4, l, idx.ravel(), "w4")))
     for i in range(args.warmup):
         x, lg, ex = pool[i % len(pool)]
         oracle.moe_forward_w4(x, lg, TOPK, ex)
@@ -916,7 +937,7 @@ def run_reference(args, log):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "int4 weights (f16 scale/min), bf16 activations, fp32 accumulate", "data": "synthetic",
+        "dtype": DTYPE_W4, "data": "synthetic",
         "config": {"workload": WORKLOAD, "experts": E, "top_k": TOPK, "hidden": H, "expert_width": F,
                    "tokens_per_step": T, "parallelism": "single CPU thread (oracle)"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
@@ -924,42 +945,84 @@ def run_reference(args, log):
     }
 
 
+# ---------------------------------------------------------------------------- main
+def run_native(args, log):
+    ctx = Ctx(args, log)
+    wl = args.workload
+    cpu = ctx.rank == 0 and ctx.world == 1 and not args.no_cpu_baseline
+    sec = args.cpu_seconds
+    legs, cpu_jobs = {}, {}
+    if wl in ("all", "decode"):
+        top = leg_decode(ctx, "w4", args.tokens or 1)
+        cpu_jobs["top"] = ("decode", "w4", SEED_W4, SEED_DECODE, args.tokens or 1)
+    elif wl == "nvfp4-decode":
+        top = leg_decode(ctx, "nvfp4", args.tokens or 1)
+        cpu_jobs["top"] = ("decode", "nvfp4", SEED_NV, SEED_NVD, args.tokens or 1)
+    elif wl == "stream":
+        top = leg_stream(ctx, args.tokens or 1)
+        cpu_jobs["top"] = ("stream", "w4", SEED_W4, SEED_STREAM, args.tokens or 1)
+    elif wl == "prefill":
+        top = leg_prefill(ctx, args.tokens or 2048)
+        cpu_jobs["top"] = ("prefill", "w4", SEED_W4, SEED_PREFILL, args.tokens or 2048)
+    elif wl == "nvfp4-prefill":
+        top = leg_prefill_nvfp4(ctx, args.tokens or 512)
+        cpu_jobs["top"] = ("prefill", "nvfp4", SEED_NV, SEED_NVP, args.tokens or 512)
+    else:
+        raise SystemExit(f"unknown workload {wl}")
+    if wl == "all":
+        for T in (1, 4, 16):
+            legs[f"decode_stream_T{T}"] = leg_stream(ctx, T)
+            cpu_jobs[f"decode_stream_T{T}"] = ("stream", "w4", SEED_W4, SEED_STREAM, T)
+        legs["prefill_2048"] = leg_prefill(ctx, 2048)
+        cpu_jobs["prefill_2048"] = ("prefill", "w4", SEED_W4, SEED_PREFILL, 2048)
+        legs["nvfp4_prefill_512"] = leg_prefill_nvfp4(ctx, 512)
+        cpu_jobs["nvfp4_prefill_512"] = ("prefill", "nvfp4", SEED_NV, SEED_NVP, 512)
+        legs["nvfp4_decode_T1"] = leg_decode(ctx, "nvfp4", 1)
+        cpu_jobs["nvfp4_decode_T1"] = ("decode", "nvfp4", SEED_NV, SEED_NVD, 1)
+    if cpu:
+        for name, (kind, fmt, ws, xs, T) in cpu_jobs.items():
+            cb = cpu_baseline(kind, fmt, ws, xs, T, sec, log)
+            (top if name == "top" else legs[name])["cpu_baseline"] = cb
+    if legs:
+        top["legs"] = legs
+        top["gpu_launches_all_legs"] = top["gpu_launches"] + sum(v["gpu_launches"] for v in legs.values())
+    if ctx.world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return top if ctx.rank == 0 else None
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100000, help="timed steps")
+    ap.add_argument("--steps", type=int, default=200, help="timed steps of every leg")
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "nvfp4-decode", "nvfp4-prefill"])
-    ap.add_argument("--tokens", type=int, default=None, help="tokens per step (decode 1, prefill 2048)")
+    ap.add_argument("--workload", default="all",
+                    choices=["all", "decode", "stream", "prefill", "nvfp4-decode", "nvfp4-prefill"])
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="tokens per step of a single workload (decode 1, prefill 2048, NVFP4 prefill 512)")
     ap.add_argument("--layers", type=int, default=LAYERS,
-                    help="resident layers the steps rotate over (40 = 18.1 GB, larger than L2)")
+                    help="resident layers of each format (40 = 18.1 GB, larger than L2)")
     ap.add_argument("--graph-steps", type=int, default=400, help="steps captured per CUDA graph")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds", type=float, default=5.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quiet", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.tokens is None:
-        args.tokens = {"prefill": 2048, "nvfp4-prefill": 512}.get(args.workload, 1)
-    if args.workload == "prefill" and args.layers == LAYERS:
-        args.layers = 4
-    if args.workload == "nvfp4-prefill" and args.layers == LAYERS:
-        args.layers = 8
 
     def log(msg):
         if not args.quiet:
             print(f"[bench] {msg}", file=sys.stderr, flush=True)
 
     if args.impl == "reference":
+        if args.tokens is None:
+            args.tokens = 1
         out = run_reference(args, log)
-    elif args.workload == "prefill":
-        out = run_gpu_prefill(args, log)
-    elif args.workload == "nvfp4-prefill":
-        out = run_gpu_prefill_nvfp4(args, log)
     else:
-        out = run_gpu(args, log)
+        out = run_native(args, log)
     if out is not None:
         print(json.dumps(out), flush=True)
 
