@@ -74,6 +74,10 @@ def _declare(L):
         "orc_combine": (None, [_f32p, _f32p, _c_int, _c_int, _c_int, _u16p]),
         "orc_moe_forward_w4": (None, [_u16p, _f32p, _c_int, _c_int, _c_int, _c_int, _c_int,
                                       _vp, _vp, _vp, _vp, _vp, _vp, _i32p, _f32p, _vp, _u16p]),
+        "orc_quantize_w4_clip": (None, [_f32p, _c_int, _c_int, _u8p, _u16p, _u16p]),
+        "orc_quantize_sym128": (None, [_f32p, _c_int, _c_int, _u8p, _u16p]),
+        "orc_dequant_sym128": (_c_f, [_c_u8, _c_u16]),
+        "orc_expert_ffn_sym128": (None, [_u16p, _c_int, _c_int, _u8p, _u16p, _u8p, _u16p, _f32p, _vp]),
         "orc_nvfp4_global": (_c_f, [_f32p, ctypes.c_size_t]),
         "orc_nvfp4_quantize": (None, [_f32p, _c_int, _c_int, _c_f, _u8p, _u8p]),
         "orc_nvfp4_gemv": (None, [_u8p, _u8p, _c_f, _u8p, _u8p, _c_f, _c_int, _c_int, _f32p]),
@@ -261,6 +265,50 @@ def moe_forward_w4(x_bf16, logits, k, experts):
     lib().orc_moe_forward_w4(x, logits, T, E, k, H, F, *[ctypes.cast(t, ctypes.c_void_p) for t in tabs],
                              idx, w, _ptr(y_rows), y)
     return idx, w, y_rows, y
+
+
+# ---------------------------------------------------------------- clip search, symmetric group 128
+def quantize_w4_clip(w):
+    """Asymmetric group-64 int4 with the MSE clip search -> (codes u8 [N][K], scale f16 bits, min f16 bits)."""
+    w = _c(w, np.float32)
+    N, K = w.shape
+    codes = np.empty((N, K), np.uint8)
+    scale = np.empty((N, K // 64), np.uint16)
+    minv = np.empty((N, K // 64), np.uint16)
+    lib().orc_quantize_w4_clip(w, N, K, codes, scale, minv)
+    return codes, scale, minv
+
+
+def quantize_sym128(w):
+    """Symmetric group-128 int4 (zero point 8) with the MSE clip search -> (codes u8 [N][K], scale f16 bits)."""
+    w = _c(w, np.float32)
+    N, K = w.shape
+    codes = np.empty((N, K), np.uint8)
+    scale = np.empty((N, K // 128), np.uint16)
+    lib().orc_quantize_sym128(w, N, K, codes, scale)
+    return codes, scale
+
+
+def dequant_sym128(codes, scale):
+    N, K = codes.shape
+    out = np.empty((N, K), np.float32)
+    L = lib()
+    for n in range(N):
+        for k in range(K):
+            out[n, k] = L.orc_dequant_sym128(int(codes[n, k]), int(scale[n, k // 128]))
+    return out
+
+
+def expert_ffn_sym128(x_bf16, gu, d, return_h=False):
+    """x_bf16: uint16 [H]; gu, d: (codes, scale) symmetric group-128 pairs."""
+    x = _c(x_bf16, np.uint16)
+    H = x.shape[0]
+    F = gu[0].shape[0] // 2
+    Y = np.empty(H, np.float32)
+    h = np.empty(F, np.float32) if return_h else None
+    lib().orc_expert_ffn_sym128(x, H, F, _c(gu[0], np.uint8), _c(gu[1], np.uint16), _c(d[0], np.uint8),
+                                _c(d[1], np.uint16), Y, _ptr(h))
+    return (Y, h) if return_h else Y
 
 
 # ---------------------------------------------------------------- NVFP4

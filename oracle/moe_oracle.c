@@ -408,6 +408,154 @@ ORC_API void orc_moe_forward_w4(const uint16_t *x, const float *logits, int T, i
 }
 
 /* ------------------------------------------------------------------------ */
+/* MSE clip search, and the symmetric group-128 int4 format.                 */
+/*                                                                           */
+/* "Drama 3 int4 (drama-rs format)", table "What's quantized": routed        */
+/* experts int4, asymmetric, group 64, f16 scale + min, MSE clip search.     */
+/* "drama-3-w4a16", section "How it was made": round-to-nearest int4, one    */
+/* scale per 128 input weights, each scale chosen from 20 clipping ratios    */
+/* (1.0 down to 0.81) by minimum squared error; table "At a glance": int4,   */
+/* symmetric, group 128, GPTQ packing.                                       */
+/* Readings (the pages give no formulas):                                    */
+/*   - ratio i = 0..19 is p_i = (100 - i) / 100 (one fp32 division); the     */
+/*     candidate range is the group's range scaled by p_i;                   */
+/*   - the squared error of a candidate is summed in fp32 over the group's   */
+/*     channels in ascending order, each term d * d with d the dequantised   */
+/*     value minus the weight; the smallest error wins, ties to the larger   */
+/*     ratio (smaller i);                                                    */
+/*   - asymmetric (group 64): m = f16(p mn) toward -inf, s = f16((p mx - m)  */
+/*     / 15) toward +inf, codes as in orc_quantize_w4; p = 1 is exactly      */
+/*     orc_quantize_w4's choice;                                             */
+/*   - symmetric (group 128), with GPTQ's zero point 8: w = (q - 8) s,       */
+/*     q in 0..15, s = f16(2 p amax / 15) nearest-even (fp32 p * amax, then  */
+/*     * 2, then / 15), q = clamp(rint(w / s) + 8, 0, 15); s = 0 gives q = 8.*/
+/* Parity: pinned (p = 1 equals the plain quantiser; the chosen candidate's  */
+/* error is the brute-force minimum over the 20; error bound of unclipped   */
+/* elements; the mean relative error on Gaussian weights the w4a16 page      */
+/* reports for int4 group 128).                                              */
+/* ------------------------------------------------------------------------ */
+
+static float clip_ratio(int i) { return (float)(100 - i) / 100.0f; }
+
+ORC_API void orc_quantize_w4_clip(const float *w, int N, int K, uint8_t *codes,
+                                  uint16_t *scale, uint16_t *minv) {
+  const int G = K / 64;
+  for (int n = 0; n < N; ++n) {
+    for (int g = 0; g < G; ++g) {
+      const float *wg = w + (size_t)n * K + (size_t)g * 64;
+      float mn = wg[0], mx = wg[0];
+      for (int i = 1; i < 64; ++i) {
+        if (wg[i] < mn) mn = wg[i];
+        if (wg[i] > mx) mx = wg[i];
+      }
+      float best = INFINITY;
+      for (int c = 0; c < 20; ++c) {
+        const float p = clip_ratio(c);
+        uint16_t mh = orc_f32_to_f16(p * mn, 1);
+        float m = orc_f16_to_f32(mh);
+        float span = p * mx - m;
+        uint16_t sh = orc_f32_to_f16(span / 15.0f, 2);
+        float s = orc_f16_to_f32(sh);
+        uint8_t q[64];
+        float err = 0.0f;
+        for (int i = 0; i < 64; ++i) {
+          float qi = 0.0f;
+          if (s > 0.0f) {
+            qi = nearbyintf((wg[i] - m) / s);
+            if (qi < 0.0f) qi = 0.0f;
+            if (qi > 15.0f) qi = 15.0f;
+          }
+          q[i] = (uint8_t)qi;
+          float d = fmaf(qi, s, m) - wg[i];
+          err += d * d;
+        }
+        if (err < best) {
+          best = err;
+          scale[(size_t)n * G + g] = sh;
+          minv[(size_t)n * G + g] = mh;
+          memcpy(codes + (size_t)n * K + (size_t)g * 64, q, 64);
+        }
+      }
+    }
+  }
+}
+
+ORC_API void orc_quantize_sym128(const float *w, int N, int K, uint8_t *codes, uint16_t *scale) {
+  const int G = K / 128;
+  for (int n = 0; n < N; ++n) {
+    for (int g = 0; g < G; ++g) {
+      const float *wg = w + (size_t)n * K + (size_t)g * 128;
+      float amax = 0.0f;
+      for (int i = 0; i < 128; ++i) {
+        float a = fabsf(wg[i]);
+        if (a > amax) amax = a;
+      }
+      float best = INFINITY;
+      for (int c = 0; c < 20; ++c) {
+        const float p = clip_ratio(c);
+        float t = p * amax;
+        t = 2.0f * t;
+        uint16_t sh = orc_f32_to_f16(t / 15.0f, 0);
+        float s = orc_f16_to_f32(sh);
+        uint8_t q[128];
+        float err = 0.0f;
+        for (int i = 0; i < 128; ++i) {
+          float qi = 8.0f;
+          if (s > 0.0f) {
+            qi = nearbyintf(wg[i] / s) + 8.0f;
+            if (qi < 0.0f) qi = 0.0f;
+            if (qi > 15.0f) qi = 15.0f;
+          }
+          q[i] = (uint8_t)qi;
+          float d = (qi - 8.0f) * s - wg[i];
+          err += d * d;
+        }
+        if (err < best) {
+          best = err;
+          scale[(size_t)n * G + g] = sh;
+          memcpy(codes + (size_t)n * K + (size_t)g * 128, q, 128);
+        }
+      }
+    }
+  }
+}
+
+/* w = (q - 8) * s, exact in fp32 (s has 11 significant bits, q - 8 four). */
+ORC_API float orc_dequant_sym128(uint8_t q, uint16_t s) {
+  return ((float)q - 8.0f) * orc_f16_to_f32(s);
+}
+
+/* One expert's SwiGLU FFN on one bf16 row with symmetric group-128 weights,
+ * each weight dequantised literally by orc_dequant_sym128; otherwise as
+ * orc_expert_ffn_w4 (fp32 sums in ascending order, h = SiLU(g) * u). */
+ORC_API void orc_expert_ffn_sym128(const uint16_t *x, int H, int F, const uint8_t *gu_codes,
+                                   const uint16_t *gu_scale, const uint8_t *d_codes,
+                                   const uint16_t *d_scale, float *Y, float *h_out) {
+  const int Gh = H / 128, Gf = F / 128;
+  float *xf = (float *)malloc(sizeof(float) * (size_t)H);
+  float *h = (float *)malloc(sizeof(float) * (size_t)F);
+  for (int i = 0; i < H; ++i) xf[i] = orc_bf16_to_f32(x[i]);
+  for (int n = 0; n < F; ++n) {
+    float g = 0.0f, u = 0.0f;
+    for (int i = 0; i < H; ++i) {
+      size_t rg = (size_t)n, ru = (size_t)(F + n);
+      g += orc_dequant_sym128(gu_codes[rg * H + i], gu_scale[rg * Gh + i / 128]) * xf[i];
+      u += orc_dequant_sym128(gu_codes[ru * H + i], gu_scale[ru * Gh + i / 128]) * xf[i];
+    }
+    h[n] = g / (1.0f + expf(-g)) * u;
+  }
+  for (int c = 0; c < H; ++c) {
+    float acc = 0.0f;
+    for (int n = 0; n < F; ++n)
+      acc += orc_dequant_sym128(d_codes[(size_t)c * F + n], d_scale[(size_t)c * Gf + n / 128]) * h[n];
+    Y[c] = acc;
+  }
+  if (h_out) memcpy(h_out, h, sizeof(float) * (size_t)F);
+  free(xf);
+  free(h);
+}
+
+/* ------------------------------------------------------------------------ */
 /* NVFP4 (E2M1 codes, E4M3 scale per 16 input channels, FP32 global scale).  */
 /* Global scale of a tensor (a weight matrix, gate and up taken together, or */
 /* one activation row): G = amax / (448 * 6); G = 1 when amax == 0.          */

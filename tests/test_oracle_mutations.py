@@ -19,6 +19,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "moe_oracle.c")
 NVFP4_PINS = "tests/test_oracle_nvfp4.py"
 METHOD_PINS = "tests/test_oracle_method.py"
+CLIP_PINS = "tests/test_oracle_clip.py"
 
 # (name, text in the oracle, replacement, pin file that must fail)
 MUTATIONS = [
@@ -60,6 +61,26 @@ MUTATIONS = [
     ("dequant: scale and min swapped",
      "fmaf((float)q, orc_f16_to_f32(s), orc_f16_to_f32(m))",
      "fmaf((float)q, orc_f16_to_f32(m), orc_f16_to_f32(s))", METHOD_PINS),
+    ("clip search: ratios 1.0 down to 0.62 instead of 0.81",
+     "return (float)(100 - i) / 100.0f;", "return (float)(100 - 2 * i) / 100.0f;", CLIP_PINS),
+    ("clip search: asymmetric min rounded to nearest",
+     "uint16_t mh = orc_f32_to_f16(p * mn, 1);", "uint16_t mh = orc_f32_to_f16(p * mn, 0);", CLIP_PINS),
+    ("clip search: absolute instead of squared error",
+     "float d = (qi - 8.0f) * s - wg[i];\n          err += d * d;",
+     "float d = (qi - 8.0f) * s - wg[i];\n          err += fabsf(d);", CLIP_PINS),
+    ("clip search: the largest error wins",
+     "          q[i] = (uint8_t)qi;\n          float d = fmaf(qi, s, m) - wg[i];\n          err += d * d;\n        }\n"
+     "        if (err < best) {",
+     "          q[i] = (uint8_t)qi;\n          float d = fmaf(qi, s, m) - wg[i];\n          err += d * d;\n        }\n"
+     "        if (-err < best) {", CLIP_PINS),
+    ("symmetric group 128: zero point 7",
+     "qi = nearbyintf(wg[i] / s) + 8.0f;", "qi = nearbyintf(wg[i] / s) + 7.0f;", CLIP_PINS),
+    ("symmetric group 128: scale amax / 7.5 dropped to amax / 8",
+     "uint16_t sh = orc_f32_to_f16(t / 15.0f, 0);", "uint16_t sh = orc_f32_to_f16(t / 16.0f, 0);", CLIP_PINS),
+    ("symmetric group 128: dequant with zero point 7",
+     "return ((float)q - 8.0f) * orc_f16_to_f32(s);", "return ((float)q - 7.0f) * orc_f16_to_f32(s);", CLIP_PINS),
+    ("symmetric group 128 FFN: down scales indexed by output row only",
+     "d_scale[(size_t)c * Gf + n / 128]", "d_scale[(size_t)c * Gf]", CLIP_PINS),
     ("combine: routing weight dropped",
      "acc += w[(size_t)t * k + j] * Yrows[((size_t)t * k + j) * H + c];",
      "acc += Yrows[((size_t)t * k + j) * H + c];", METHOD_PINS),
