@@ -360,8 +360,9 @@ class Ctx:
 
     def timed(self, fn, K, W, n_resident, eager_touch=True):
         """Device time (ms, max over ranks) of exactly K steps W .. W + K - 1,
-        after every resident layer has been touched (untimed) and W warm-up
-        steps.  Returns (ms, clock summary)."""
+        after every resident layer has been touched (untimed), W warm-up
+        steps and one untimed replay of the timed graphs.  Returns (ms, clock
+        summary)."""
         import torch
         if eager_touch:
             with torch.cuda.stream(self.stream):
@@ -370,6 +371,7 @@ class Ctx:
         g_warm = self.graphs(fn, 0, max(W, n_resident))
         g_main = self.graphs(fn, W, K)
         self.replay(g_warm)
+        self.replay(g_main)  # a graph's first replay uploads it: keep that out of the timed region
         torch.cuda.synchronize()
         dist_barrier()
         with ClockSampler(self.local) as clk:
@@ -531,6 +533,7 @@ def leg_decode(ctx, fmt, T):
            for _ in range(P)]
     g = ctx.capture(step, W, P, evs)
     ctx.replay([g])
+    ctx.replay([g])
     torch.cuda.synchronize()
     isolated_ms = sum(a.elapsed_time(b) for a, b in evs) / P
     del g
@@ -687,6 +690,7 @@ def leg_prefill(ctx, T=2048, nl=4):
            for _ in range(P)]
     g = ctx.capture(step, W, P, evs)
     ctx.replay([g])
+    ctx.replay([g])
     torch.cuda.synchronize()
     dur_ms = sum(a.elapsed_time(b) for a, b in evs) / P
     del g
@@ -767,6 +771,7 @@ def leg_prefill_nvfp4(ctx, T=512, nl=8):
     evs = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
            for _ in range(P)]
     g = ctx.capture(step, W, P, evs)
+    ctx.replay([g])
     ctx.replay([g])
     torch.cuda.synchronize()
     dur_ms = sum(a.elapsed_time(b) for a, b in evs) / P

@@ -96,6 +96,47 @@ MOE_API size_t moe_w4_packed_bytes(int N, int K);
 MOE_API moe_status moe_quantize_w4(const float *w, int N, int K, uint8_t *codes,
                                    uint16_t *scale, uint16_t *minv, moe_stream_t stream);
 
+/*
+ * The same format with the MSE clip search: for every group, 20 candidate
+ * ranges, the group's [min, max] scaled by p_i = (100 - i) / 100 (i = 0..19,
+ * 1.0 down to 0.81), each rounded as above (m toward -inf, s toward +inf from
+ * the rounded m) and coded by nearest rounding; the candidate with the
+ * smallest fp32 sum over the group, in channel order, of (q*s + m - w)^2 wins,
+ * ties to the larger ratio.  p = 1 is exactly moe_quantize_w4's choice, so
+ * no group gets a larger squared error.  Bit-exact with the reference.
+ * Source: "Drama 3 int4 (drama-rs format)", table "What's quantized" (MSE
+ * clip search); "drama-3-w4a16", section "How it was made" (20 clipping
+ * ratios 1.0 -> 0.81 by minimum squared error).  Errors as moe_quantize_w4.
+ */
+MOE_API moe_status moe_quantize_w4_clip(const float *w, int N, int K, uint8_t *codes,
+                                        uint16_t *scale, uint16_t *minv, moe_stream_t stream);
+
+/*
+ * Symmetric group-128 int4 ("drama-3-w4a16", table "At a glance": int4,
+ * symmetric, group 128, GPTQ packing; section "How it was made": one scale
+ * per 128 input weights, round-to-nearest, clip search as above):
+ *   w = (q - 8) * s,  q in 0..15 (GPTQ's zero point 8), s f16 per 128 inputs,
+ *   candidate s_i = f16(2 * (p_i * amax) / 15) nearest-even,
+ *   q = clamp(rint(w / s) + 8, 0, 15) (s == 0 gives q = 8).
+ * Outputs codes u8 [N][K] and scale f16 [N][K/128].  Errors: INVALID_ARG,
+ * UNSUPPORTED_SHAPE (K % 128).
+ */
+MOE_API moe_status moe_quantize_w4_sym128(const float *w, int N, int K, uint8_t *codes,
+                                          uint16_t *scale, moe_stream_t stream);
+
+/*
+ * Packs a symmetric group-128 matrix (codes [N][K], scale [N][K/128]) into the
+ * int4 device form above, so every int4 kernel runs it unchanged: each group
+ * of 128 becomes two groups of 64 with scale s and min -8 s, and q*s + (-8 s)
+ * equals (q - 8) * s exactly.  Requires |s| < 8192 (so that -8 s is an f16).
+ * ws: moe_pack_w4_sym128_workspace_bytes(N, K) bytes of scratch, 4-byte
+ * aligned.  Errors: as moe_pack_w4, UNSUPPORTED_SHAPE for K % 128, WORKSPACE.
+ */
+MOE_API size_t moe_pack_w4_sym128_workspace_bytes(int N, int K);
+MOE_API moe_status moe_pack_w4_sym128(const uint8_t *codes, const uint16_t *scale, int N, int K,
+                                      int kind, void *packed, size_t packed_bytes, void *ws,
+                                      size_t ws_bytes, moe_stream_t stream);
+
 /* Canonical -> packed.  packed_bytes must be >= moe_w4_packed_bytes(N, K).
  * Errors: INVALID_ARG, UNSUPPORTED_SHAPE (N % 16, K % 64, GATE_UP with N % 32),
  * WORKSPACE (packed_bytes too small). */

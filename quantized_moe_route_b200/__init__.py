@@ -56,6 +56,10 @@ SIGNATURES = {
     "moe_pack_w4": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
     "moe_unpack_w4": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp]),
     "moe_dequant_w4": (_i, [_vp, _i, _i, _i, _vp, _vp]),
+    "moe_quantize_w4_clip": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp]),
+    "moe_quantize_w4_sym128": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
+    "moe_pack_w4_sym128_workspace_bytes": (_sz, [_i, _i]),
+    "moe_pack_w4_sym128": (_i, [_vp, _vp, _i, _i, _i, _vp, _sz, _vp, _sz, _vp]),
     "moe_nvfp4_packed_bytes": (_sz, [_i, _i]),
     "moe_nvfp4_global": (_i, [_vp, _sz, _vp, _vp]),
     "moe_quantize_nvfp4": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp]),
@@ -133,6 +137,28 @@ def moe_pack_w4(codes, scale, minv, kind, packed, stream=None):
     nbytes = packed.numel() * packed.element_size()
     _check(lib().moe_pack_w4(_p(codes), _p(scale), _p(minv), N, K, kind, _p(packed), nbytes,
                              _stream(stream)), "moe_pack_w4")
+
+
+def moe_quantize_w4_clip(w, codes, scale, minv, stream=None):
+    N, K = w.shape
+    _check(lib().moe_quantize_w4_clip(_p(w), N, K, _p(codes), _p(scale), _p(minv), _stream(stream)),
+           "moe_quantize_w4_clip")
+
+
+def moe_quantize_w4_sym128(w, codes, scale, stream=None):
+    N, K = w.shape
+    _check(lib().moe_quantize_w4_sym128(_p(w), N, K, _p(codes), _p(scale), _stream(stream)),
+           "moe_quantize_w4_sym128")
+
+
+def moe_pack_w4_sym128(codes, scale, kind, packed, ws, stream=None):
+    N, K = codes.shape
+    _check(lib().moe_pack_w4_sym128(_p(codes), _p(scale), N, K, kind, _p(packed), packed.numel(), _p(ws),
+                                    ws.numel() * ws.element_size(), _stream(stream)), "moe_pack_w4_sym128")
+
+
+def moe_pack_w4_sym128_workspace_bytes(N, K) -> int:
+    return lib().moe_pack_w4_sym128_workspace_bytes(N, K)
 
 
 def moe_nvfp4_packed_bytes(N: int, K: int) -> int:
