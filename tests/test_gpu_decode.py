@@ -149,40 +149,51 @@ def test_fused_layer_one_expert_for_all_tokens_and_reuse():
     ffn_close(synth.bf16_bits_to_f32(y1), synth.bf16_bits_to_f32(oy), "fused y")
 
 
-def test_fused_decode_waits_while_another_stream_holds_an_sm():
-    """The decode kernel's down items wait on gate/up items of other CTAs of
-    the same grid, so every CTA must run at once.  The launch is cooperative:
-    while a kernel on another stream holds one SM (and all its shared memory)
-    for about a second, the decode grid does not start on the other SMs and
-    then time out waiting for the missing CTA; it waits for the SM, runs
-    whole, and gives the oracle's result with no device error."""
+def test_decode_with_an_sm_held_by_another_stream():
+    """The unfused decode kernel's down items wait on gate/up items of other
+    CTAs of the same grid, so every CTA must run at once: its launch is
+    cooperative, and while a kernel on another stream holds one SM (and all
+    its shared memory) for about a second, the grid waits for the SM, runs
+    whole, and gives the oracle's result with no device error.  The fused
+    layer kernel waits only inside its clusters, so it runs beside the held
+    SM and gives the oracle's result too."""
     import gpu_hold
     E, H, F, T, k, seed = 256, 2048, 512, 1, 8, 91
     x = synth.activations_bf16(seed, 0, T, H)
     logits = synth.router_logits(seed, 0, T, E)
     oidx, _ = oracle.route(logits, k)
     layer = Layer(seed, 0, E, H, F, oidx.ravel())
-    xd, ld = u16(x), torch.from_numpy(logits).cuda()
+    xd, ld, idx = u16(x), torch.from_numpy(logits).cuda(), torch.from_numpy(oidx).cuda()
+    y_rows = torch.empty((T * k, H), device="cuda")
+    ws = decode_workspace(T, k, F)
     y = torch.empty((T, H), dtype=torch.int16, device="cuda")
-    ws = torch.zeros(moe.moe_decode_layer_workspace_bytes(T, k, H, F), dtype=torch.uint8, device="cuda")
-    done = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lws = torch.zeros(moe.moe_decode_layer_workspace_bytes(T, k, H, F), dtype=torch.uint8, device="cuda")
+    done = torch.zeros(2, dtype=torch.int32, device="cuda")
     smem = torch.cuda.get_device_properties(0).shared_memory_per_block_optin
     side, main = torch.cuda.Stream(), torch.cuda.Stream()
+    _, _, oy_rows, oy = oracle.moe_forward_w4(x, logits, k, layer.canon)
     torch.cuda.synchronize()
-    gpu_hold.hold_sm(2_000_000_000, smem, done, side)  # about one second at 1.9 GHz
+    gpu_hold.hold_sm(2_000_000_000, smem, done[0:1], side)  # about one second at 1.9 GHz
     time.sleep(0.05)  # the holding CTA is resident before the decode is launched
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(main):
         e0.record(main)
-        moe.moe_decode_layer_w4a16(layer.desc, xd, ld, k, y, ws, stream=main)
+        moe.moe_ffn_w4a16_decode(layer.desc, xd, idx, y_rows, ws, stream=main)
         e1.record(main)
     torch.cuda.synchronize()
-    assert done.item() == 1
+    assert done[0].item() == 1
     assert moe.moe_device_error() == 0
-    _, _, _, oy = oracle.moe_forward_w4(x, logits, k, layer.canon)
-    ffn_close(synth.bf16_bits_to_f32(to_u16(y)), synth.bf16_bits_to_f32(oy), "y")
-    # the grid did wait for the held SM (it needs every SM)
-    assert e0.elapsed_time(e1) > 300.0
+    ffn_close(y_rows.cpu().numpy(), oy_rows, "y_rows")
+    assert e0.elapsed_time(e1) > 300.0  # the grid did wait for the held SM (it needs every SM)
+    gpu_hold.hold_sm(2_000_000_000, smem, done[1:2], side)
+    time.sleep(0.05)
+    with torch.cuda.stream(main):
+        moe.moe_decode_layer_w4a16(layer.desc, xd, ld, k, y, lws, stream=main)
+    main.synchronize()
+    assert moe.moe_device_error() == 0
+    ffn_close(synth.bf16_bits_to_f32(to_u16(y)), synth.bf16_bits_to_f32(oy), "fused y")
+    torch.cuda.synchronize()
+    assert done[1].item() == 1
 
 
 @pytest.mark.parametrize("T", [1, 16])
