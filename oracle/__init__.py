@@ -74,6 +74,7 @@ def _declare(L):
         "orc_combine": (None, [_f32p, _f32p, _c_int, _c_int, _c_int, _u16p]),
         "orc_moe_forward_w4": (None, [_u16p, _f32p, _c_int, _c_int, _c_int, _c_int, _c_int,
                                       _vp, _vp, _vp, _vp, _vp, _vp, _i32p, _f32p, _vp, _u16p]),
+        "orc_router_logits": (None, [_u16p, _u16p, _c_int, _c_int, _c_int, _f32p]),
         "orc_quantize_w4_clip": (None, [_f32p, _c_int, _c_int, _u8p, _u16p, _u16p]),
         "orc_quantize_sym128": (None, [_f32p, _c_int, _c_int, _u8p, _u16p]),
         "orc_dequant_sym128": (_c_f, [_c_u8, _c_u16]),
@@ -265,6 +266,18 @@ def moe_forward_w4(x_bf16, logits, k, experts):
     lib().orc_moe_forward_w4(x, logits, T, E, k, H, F, *[ctypes.cast(t, ctypes.c_void_p) for t in tabs],
                              idx, w, _ptr(y_rows), y)
     return idx, w, y_rows, y
+
+
+# ---------------------------------------------------------------- router linear
+def router_logits(x_bf16, wr_bf16):
+    """x bf16 bits [T][H], Wr bf16 bits [E][H] -> fp32 logits [T][E]."""
+    x = _c(x_bf16, np.uint16)
+    wr = _c(wr_bf16, np.uint16)
+    T, H = x.shape
+    E = wr.shape[0]
+    out = np.empty((T, E), np.float32)
+    lib().orc_router_logits(x, wr, T, E, H, out)
+    return out
 
 
 # ---------------------------------------------------------------- clip search, symmetric group 128

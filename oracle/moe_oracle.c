@@ -385,6 +385,28 @@ ORC_API void orc_combine(const float *Yrows, const float *w, int T, int k, int H
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* Router linear: logits[t][e] = sum_k x[t][k] * Wr[e][k], x and Wr bf16,    */
+/* each product and the running sum fp32, k ascending; no bias.  The router  */
+/* keeps bf16 weights ("Drama 3 int4 (drama-rs format)", table "What's       */
+/* quantized": embeddings, router, norms bf16 / f32; "DRAMA-3 MLX            */
+/* expert-only 4-bit", section "Quantization and provenance": routers retain */
+/* source BF16); fp32 accumulation and no bias are this build's reading.     */
+/* Parity: pinned (one-hot rows select a channel of x exactly; a float64     */
+/* matmul within the fp32 summation bound; linearity in x).                  */
+/* ------------------------------------------------------------------------ */
+
+ORC_API void orc_router_logits(const uint16_t *x, const uint16_t *wr, int T, int E, int H,
+                               float *logits) {
+  for (int t = 0; t < T; ++t)
+    for (int e = 0; e < E; ++e) {
+      float acc = 0.0f;
+      for (int i = 0; i < H; ++i)
+        acc += orc_bf16_to_f32(x[(size_t)t * H + i]) * orc_bf16_to_f32(wr[(size_t)e * H + i]);
+      logits[(size_t)t * E + e] = acc;
+    }
+}
+
 /* Whole routed MoE FFN for T tokens: route, then for every (t, j) the
  * expert FFN of expert idx[t][j] on x[t], then the combine.  Expert weights
  * come as per-expert pointer tables (an entry may be NULL when the expert is

@@ -20,6 +20,7 @@ SRC = os.path.join(ROOT, "oracle", "moe_oracle.c")
 NVFP4_PINS = "tests/test_oracle_nvfp4.py"
 METHOD_PINS = "tests/test_oracle_method.py"
 CLIP_PINS = "tests/test_oracle_clip.py"
+ROUTER_PINS = "tests/test_oracle_router.py"
 
 # (name, text in the oracle, replacement, pin file that must fail)
 MUTATIONS = [
@@ -81,6 +82,11 @@ MUTATIONS = [
      "return ((float)q - 8.0f) * orc_f16_to_f32(s);", "return ((float)q - 7.0f) * orc_f16_to_f32(s);", CLIP_PINS),
     ("symmetric group 128 FFN: down scales indexed by output row only",
      "d_scale[(size_t)c * Gf + n / 128]", "d_scale[(size_t)c * Gf]", CLIP_PINS),
+    ("router linear: weight matrix transposed",
+     "orc_bf16_to_f32(wr[(size_t)e * H + i])", "orc_bf16_to_f32(wr[(size_t)i * E + e])", ROUTER_PINS),
+    ("router linear: first channel skipped",
+     "      for (int i = 0; i < H; ++i)\n        acc += orc_bf16_to_f32(x[(size_t)t * H + i])",
+     "      for (int i = 1; i < H; ++i)\n        acc += orc_bf16_to_f32(x[(size_t)t * H + i])", ROUTER_PINS),
     ("combine: routing weight dropped",
      "acc += w[(size_t)t * k + j] * Yrows[((size_t)t * k + j) * H + c];",
      "acc += Yrows[((size_t)t * k + j) * H + c];", METHOD_PINS),
