@@ -261,6 +261,29 @@ MOE_API moe_status moe_route(const float *logits, int T, int E, int k, int32_t *
                              moe_stream_t stream);
 
 /*
+ * The router linear fused with routing, in one launch: logits[t][e] =
+ * sum_k x[t][k] * Wr[e][k] (x bf16 [T][H], Wr bf16 [E][H], fp32 products and
+ * sums, no bias), then the routing of moe_route on those logits (idx, w as
+ * there).  logits fp32 [T][E] is an optional output (NULL: kept in the
+ * workspace).  Source: the router stays bf16 ("Drama 3 int4 (drama-rs
+ * format)", table "What's quantized"; "DRAMA-3 MLX expert-only 4-bit",
+ * section "Quantization and provenance"); fp32 accumulation and no bias are
+ * this library's reading.  The tensor cores sum the products in their own
+ * order, so logits can differ from a sequential fp32 sum in the last bits; the
+ * selection is made on the logits this call computes.
+ * Workspace: moe_router_route_workspace_bytes(T, E) bytes, 16-byte aligned,
+ * zero-filled before its first use; every call leaves it ready for the next
+ * stream-ordered call.  Limits: E % 16 == 0 (E % 64 == 0 above 64), E <=
+ * 1024, H % 64 == 0, 1 <= k <= min(E, 32).  x, Wr 16-byte aligned, logits
+ * 8-byte aligned.  T == 0 is a no-op.  Errors: INVALID_ARG,
+ * UNSUPPORTED_SHAPE, WORKSPACE, CUDA.
+ */
+MOE_API size_t moe_router_route_workspace_bytes(int T, int E);
+MOE_API moe_status moe_router_route(const uint16_t *x, const uint16_t *wr, int T, int E, int H, int k,
+                                    float *logits, int32_t *idx, float *w, void *ws, size_t ws_bytes,
+                                    moe_stream_t stream);
+
+/*
  * Group the T*k rows r = t*k + j by expert idx[r] (stable: within an expert,
  * rows in increasing r).  Outputs counts [E], offsets [E+1] (exclusive scan,
  * offsets[E] = T*k), sorted_rows [T*k] (row ids in grouped order), inv [T*k]

@@ -67,6 +67,8 @@ SIGNATURES = {
     "moe_unpack_nvfp4": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
     "moe_quantize_nvfp4_rows": (_i, [_vp, _i, _i, _i, _vp, _i, _vp, _vp, _vp, _vp]),
     "moe_route": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
+    "moe_router_route_workspace_bytes": (_sz, [_i, _i]),
+    "moe_router_route": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_permute_workspace_bytes": (_sz, [_i, _i, _i]),
     "moe_permute": (_i, [_vp, _i, _i, _i, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_decode_workspace_bytes": (_sz, [_i, _i, _i]),
@@ -220,6 +222,18 @@ def make_nvfp4_layer(E, H, F, gate_up, down, g_gu, g_d) -> moe_nvfp4_layer:
 def moe_route(logits, k, idx, w, stream=None):
     T, E = logits.shape
     _check(lib().moe_route(_p(logits), T, E, k, _p(idx), _p(w), _stream(stream)), "moe_route")
+
+
+def moe_router_route_workspace_bytes(T, E) -> int:
+    return lib().moe_router_route_workspace_bytes(T, E)
+
+
+def moe_router_route(x, wr, k, idx, w, ws, logits=None, stream=None):
+    """Router linear (bf16 Wr [E][H] times x [T][H]) and routing in one launch."""
+    T, H = x.shape
+    E = wr.shape[0]
+    _check(lib().moe_router_route(_p(x), _p(wr), T, E, H, k, _p(logits), _p(idx), _p(w), _p(ws),
+                                  ws.numel() * ws.element_size(), _stream(stream)), "moe_router_route")
 
 
 def moe_permute_workspace_bytes(T, k, E) -> int:
