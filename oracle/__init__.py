@@ -75,6 +75,9 @@ def _declare(L):
         "orc_moe_forward_w4": (None, [_u16p, _f32p, _c_int, _c_int, _c_int, _c_int, _c_int,
                                       _vp, _vp, _vp, _vp, _vp, _vp, _i32p, _f32p, _vp, _u16p]),
         "orc_router_logits": (None, [_u16p, _u16p, _c_int, _c_int, _c_int, _f32p]),
+        "orc_moe_forward_w4_shared": (None, [_u16p, _f32p, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                             _vp, _vp, _vp, _vp, _vp, _vp, _u8p, _u16p, _u16p, _u8p, _u16p,
+                                             _u16p, _i32p, _f32p, _vp, _u16p]),
         "orc_quantize_w4_clip": (None, [_f32p, _c_int, _c_int, _u8p, _u16p, _u16p]),
         "orc_quantize_sym128": (None, [_f32p, _c_int, _c_int, _u8p, _u16p]),
         "orc_dequant_sym128": (_c_f, [_c_u8, _c_u16]),
@@ -265,6 +268,43 @@ def moe_forward_w4(x_bf16, logits, k, experts):
     y = np.empty((T, H), np.uint16)
     lib().orc_moe_forward_w4(x, logits, T, E, k, H, F, *[ctypes.cast(t, ctypes.c_void_p) for t in tabs],
                              idx, w, _ptr(y_rows), y)
+    return idx, w, y_rows, y
+
+
+def moe_forward_w4_shared(x_bf16, logits, k, experts, shared):
+    """The routed experts plus a shared expert (weight 1, after the routed
+    sum).  shared: (gu triple, d triple).  Returns (idx [T][k], w [T][k],
+    y_rows fp32 [T][k+1][H], y bf16 bits [T][H])."""
+    x = _c(x_bf16, np.uint16)
+    logits = _c(logits, np.float32)
+    T, H = x.shape
+    E = logits.shape[1]
+    idx, _ = route(logits, k)
+    need = sorted(set(int(e) for e in idx.ravel()))
+    missing = [e for e in need if e not in experts]
+    if missing:
+        raise KeyError(f"oracle needs weights of experts {missing}")
+    F = shared[0][0].shape[0] // 2
+    keep = []
+
+    def table(which, part, dt):
+        arr = (ctypes.c_void_p * E)()
+        for e in need:
+            a = _c(experts[e][which][part], dt)
+            keep.append(a)
+            arr[e] = a.ctypes.data
+        return arr
+
+    tabs = [table(0, 0, np.uint8), table(0, 1, np.uint16), table(0, 2, np.uint16),
+            table(1, 0, np.uint8), table(1, 1, np.uint16), table(1, 2, np.uint16)]
+    sh = [_c(shared[0][0], np.uint8), _c(shared[0][1], np.uint16), _c(shared[0][2], np.uint16),
+          _c(shared[1][0], np.uint8), _c(shared[1][1], np.uint16), _c(shared[1][2], np.uint16)]
+    idx = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float32)
+    y_rows = np.empty((T, k + 1, H), np.float32)
+    y = np.empty((T, H), np.uint16)
+    lib().orc_moe_forward_w4_shared(x, logits, T, E, k, H, F, *[ctypes.cast(t, ctypes.c_void_p) for t in tabs],
+                                    *sh, idx, w, _ptr(y_rows), y)
     return idx, w, y_rows, y
 
 

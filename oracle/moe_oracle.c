@@ -385,6 +385,49 @@ ORC_API void orc_combine(const float *Yrows, const float *w, int T, int k, int H
     }
 }
 
+/* Shared expert: one more SwiGLU expert applied to every token, added after
+ * the routed experts with weight 1:
+ *   y_t = bf16( (sum over j < k, in order, of w[t][j] Y_(t,j))  +  1 * Y_s(x_t) )
+ * -- the combine of k + 1 rows whose last row is the shared expert's, with
+ * weight 1.  The pages list a shared expert beside the routed ones ("Drama 3
+ * int4 (drama-rs format)", table "What's quantized"; "Drama 3 - NVFP4 routed
+ * experts", section "Quantization"); weight 1, its place after the routed
+ * sum, and its int4 storage (in the routed experts' format) are this build's
+ * reading.  idx/w receive the k routed choices; y_rows (optional) [T][k+1][H]
+ * the rows.  Parity: pinned (zero shared weights give the routed-only result;
+ * zero routed weights give the shared expert alone; the composition of the
+ * pinned FFN and combine). */
+ORC_API void orc_moe_forward_w4_shared(const uint16_t *x, const float *logits, int T, int E, int k,
+                                       int H, int F, const uint8_t *const *gu_codes,
+                                       const uint16_t *const *gu_scale,
+                                       const uint16_t *const *gu_min,
+                                       const uint8_t *const *d_codes,
+                                       const uint16_t *const *d_scale,
+                                       const uint16_t *const *d_min, const uint8_t *s_gu_codes,
+                                       const uint16_t *s_gu_scale, const uint16_t *s_gu_min,
+                                       const uint8_t *s_d_codes, const uint16_t *s_d_scale,
+                                       const uint16_t *s_d_min, int32_t *idx, float *w,
+                                       float *y_rows, uint16_t *y) {
+  const int k1 = k + 1;
+  orc_route(logits, T, E, k, idx, w);
+  float *rows = y_rows ? y_rows : (float *)malloc(sizeof(float) * (size_t)T * k1 * H);
+  float *w1 = (float *)malloc(sizeof(float) * (size_t)T * k1);
+  for (int t = 0; t < T; ++t) {
+    for (int j = 0; j < k; ++j) {
+      int e = idx[(size_t)t * k + j];
+      orc_expert_ffn_w4(x + (size_t)t * H, H, F, gu_codes[e], gu_scale[e], gu_min[e], d_codes[e],
+                        d_scale[e], d_min[e], rows + ((size_t)t * k1 + j) * H, NULL);
+      w1[(size_t)t * k1 + j] = w[(size_t)t * k + j];
+    }
+    orc_expert_ffn_w4(x + (size_t)t * H, H, F, s_gu_codes, s_gu_scale, s_gu_min, s_d_codes,
+                      s_d_scale, s_d_min, rows + ((size_t)t * k1 + k) * H, NULL);
+    w1[(size_t)t * k1 + k] = 1.0f;
+  }
+  orc_combine(rows, w1, T, k1, H, y);
+  free(w1);
+  if (!y_rows) free(rows);
+}
+
 /* ------------------------------------------------------------------------ */
 /* Router linear: logits[t][e] = sum_k x[t][k] * Wr[e][k], x and Wr bf16,    */
 /* each product and the running sum fp32, k ascending; no bias.  The router  */

@@ -21,6 +21,7 @@ NVFP4_PINS = "tests/test_oracle_nvfp4.py"
 METHOD_PINS = "tests/test_oracle_method.py"
 CLIP_PINS = "tests/test_oracle_clip.py"
 ROUTER_PINS = "tests/test_oracle_router.py"
+SHARED_PINS = "tests/test_oracle_shared.py"
 
 # (name, text in the oracle, replacement, pin file that must fail)
 MUTATIONS = [
@@ -87,6 +88,11 @@ MUTATIONS = [
     ("router linear: first channel skipped",
      "      for (int i = 0; i < H; ++i)\n        acc += orc_bf16_to_f32(x[(size_t)t * H + i])",
      "      for (int i = 1; i < H; ++i)\n        acc += orc_bf16_to_f32(x[(size_t)t * H + i])", ROUTER_PINS),
+    ("shared expert: weight one half instead of one",
+     "w1[(size_t)t * k1 + k] = 1.0f;", "w1[(size_t)t * k1 + k] = 0.5f;", SHARED_PINS),
+    ("shared expert: applied to the wrong token",
+     "    orc_expert_ffn_w4(x + (size_t)t * H, H, F, s_gu_codes,",
+     "    orc_expert_ffn_w4(x + (size_t)((t + 1) % T) * H, H, F, s_gu_codes,", SHARED_PINS),
     ("combine: routing weight dropped",
      "acc += w[(size_t)t * k + j] * Yrows[((size_t)t * k + j) * H + c];",
      "acc += Yrows[((size_t)t * k + j) * H + c];", METHOD_PINS),
