@@ -261,6 +261,21 @@ MOE_API moe_status moe_route(const float *logits, int T, int E, int k, int32_t *
                              moe_stream_t stream);
 
 /*
+ * moe_route with a shared expert: the same routing of logits [T][E] over the
+ * E routed experts, written to rows of k + 1 entries, the last one the shared
+ * expert (id E, weight 1).  idx, w [T][k+1].  With moe_permute over E + 1
+ * experts and moe_unpermute_combine with k + 1 rows, the layer output is the
+ * routed sum plus the shared expert's row, added last.
+ * Source: a shared expert beside the routed ones ("Drama 3 int4 (drama-rs
+ * format)", table "What's quantized"; "Drama 3 - NVFP4 routed experts",
+ * "Quantization"); weight 1 and the order of the sum are this library's
+ * reading.  Limits: 1 <= k <= min(E, 31), E <= 1023.  T == 0 is a no-op.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE.
+ */
+MOE_API moe_status moe_route_shared(const float *logits, int T, int E, int k, int32_t *idx,
+                                    float *w, moe_stream_t stream);
+
+/*
  * The router linear fused with routing, in one launch: logits[t][e] =
  * sum_k x[t][k] * Wr[e][k] (x bf16 [T][H], Wr bf16 [E][H], fp32 products and
  * sums, no bias), then the routing of moe_route on those logits (idx, w as
@@ -329,8 +344,8 @@ MOE_API moe_status moe_permute(const int32_t *idx, int T, int k, int E, const ui
  * The launch is cooperative: while other work (another stream, another
  * process under MPS) holds SMs, the GPU starts the grid only once every block
  * can run, instead of starting part of it.  The same holds for
- * moe_decode_layer_w4a16, moe_decode_layer_nvfp4 and
- * moe_ffn_w4a16_decode_static.
+ * moe_decode_layer_w4a16, moe_decode_layer_w4a16_shared,
+ * moe_decode_layer_nvfp4 and moe_ffn_w4a16_decode_static.
  */
 MOE_API size_t moe_decode_workspace_bytes(int T, int k, int F);
 MOE_API moe_status moe_ffn_w4a16_decode(const moe_w4_layer *layer, const uint16_t *x,
@@ -359,6 +374,23 @@ MOE_API moe_status moe_decode_layer_w4a16(const moe_w4_layer *layer, const uint1
                                           const float *logits, int T, int k, uint16_t *y,
                                           int32_t *idx, float *w, void *ws, size_t ws_bytes,
                                           moe_stream_t stream);
+
+/*
+ * moe_decode_layer_w4a16 with a shared expert.  `layer` holds E = Er + 1
+ * experts: the Er routed ones, then the shared expert (id Er).  logits fp32
+ * [T][Er]; each token runs its k routed experts and the shared one, and
+ *   y = bf16( (sum over j < k, ascending, of w[t][j] * row(t, j)) + row(t, shared) )
+ * in fp32, as moe_route_shared + moe_unpermute_combine with k + 1 rows.
+ * idx, w [T][k]: optional outputs of the routed selection (both or neither).
+ * Workspace: moe_decode_layer_workspace_bytes(T, k + 1, H, F).  Limits as
+ * for moe_decode_layer_w4a16 with k + 1 in place of k (T*(k+1) <= 256,
+ * k + 1 <= 32, E <= 1024).  Source: the passages of moe_route_shared and
+ * moe_decode_layer_w4a16.
+ */
+MOE_API moe_status moe_decode_layer_w4a16_shared(const moe_w4_layer *layer, const uint16_t *x,
+                                                 const float *logits, int T, int k, uint16_t *y,
+                                                 int32_t *idx, float *w, void *ws, size_t ws_bytes,
+                                                 moe_stream_t stream);
 
 /*
  * The NVFP4 form of moe_decode_layer_w4a16: one launch routes the T tokens,

@@ -67,6 +67,7 @@ SIGNATURES = {
     "moe_unpack_nvfp4": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
     "moe_quantize_nvfp4_rows": (_i, [_vp, _i, _i, _i, _vp, _i, _vp, _vp, _vp, _vp]),
     "moe_route": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
+    "moe_route_shared": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
     "moe_router_route_workspace_bytes": (_sz, [_i, _i]),
     "moe_router_route": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_permute_workspace_bytes": (_sz, [_i, _i, _i]),
@@ -77,6 +78,8 @@ SIGNATURES = {
     "moe_decode_layer_workspace_bytes": (_sz, [_i, _i, _i, _i]),
     "moe_decode_layer_w4a16": (_i, [ctypes.POINTER(moe_w4_layer), _vp, _vp, _i, _i, _vp, _vp, _vp, _vp, _sz,
                                     _vp]),
+    "moe_decode_layer_w4a16_shared": (_i, [ctypes.POINTER(moe_w4_layer), _vp, _vp, _i, _i, _vp, _vp, _vp, _vp,
+                                           _sz, _vp]),
     "moe_decode_layer_nvfp4": (_i, [ctypes.POINTER(moe_nvfp4_layer), _vp, _vp, _i, _i, _vp, _vp, _vp, _vp,
                                     _sz, _vp]),
     "moe_prefill_workspace_bytes": (_sz, [_i, _i]),
@@ -224,6 +227,12 @@ def moe_route(logits, k, idx, w, stream=None):
     _check(lib().moe_route(_p(logits), T, E, k, _p(idx), _p(w), _stream(stream)), "moe_route")
 
 
+def moe_route_shared(logits, k, idx, w, stream=None):
+    """Routing over E experts plus a shared expert: idx, w [T][k+1], column k = (E, 1.0)."""
+    T, E = logits.shape
+    _check(lib().moe_route_shared(_p(logits), T, E, k, _p(idx), _p(w), _stream(stream)), "moe_route_shared")
+
+
 def moe_router_route_workspace_bytes(T, E) -> int:
     return lib().moe_router_route_workspace_bytes(T, E)
 
@@ -277,6 +286,15 @@ def moe_decode_layer_w4a16(layer: moe_w4_layer, x, logits, k, y, ws, idx=None, w
     _check(lib().moe_decode_layer_w4a16(ctypes.byref(layer), _p(x), _p(logits), T, k, _p(y), _p(idx), _p(w),
                                         _p(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "moe_decode_layer_w4a16")
+
+
+def moe_decode_layer_w4a16_shared(layer: moe_w4_layer, x, logits, k, y, ws, idx=None, w=None, stream=None):
+    """One layer in one launch with a shared expert: layer holds the routed
+    experts then the shared one; logits cover the routed experts only."""
+    T = x.shape[0]
+    _check(lib().moe_decode_layer_w4a16_shared(ctypes.byref(layer), _p(x), _p(logits), T, k, _p(y), _p(idx),
+                                               _p(w), _p(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "moe_decode_layer_w4a16_shared")
 
 
 def moe_decode_layer_nvfp4(layer: moe_nvfp4_layer, x, logits, k, y, ws, idx=None, w=None, stream=None):

@@ -68,6 +68,8 @@ struct DecodeArgs {
   uint32_t h_off;            // offset of a B item's h tile inside its stage
   uint32_t h_polls;          // bound of a B item's wait for h (polls of >= 100 ns)
   int starve_gate_up;        // test hook: A items write no h, so B items time out
+  int shared;                // fused form: 1 = the layer's last expert is a shared expert
+                             // (row k - 1 of every token, weight 1); routing scores E - 1
 };
 
 struct DecodeSmem {
@@ -194,16 +196,23 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
   // first weight copies go out as soon as the slots are known.
   if (kFused) {  // warp t routes token t
     if (warp < T) {
+      // with a shared expert the router scores the Er = E - 1 routed experts
+      // and row kr = k - 1 is the shared expert's, weight 1
+      const int kr = k - a.shared, Er = E - a.shared;
       int j_idx;
       float j_w;
-      route_token_warp<PER>(a.logits + (size_t)warp * E, E, k, &j_idx, &j_w);
+      route_token_warp<PER>(a.logits + (size_t)warp * Er, Er, kr, &j_idx, &j_w);
+      if (lane == kr) {  // only reached with a shared expert (kr < k)
+        j_idx = Er;
+        j_w = 1.0f;
+      }
       if (lane < k) {
         ridx[warp * k + lane] = j_idx;
         rw[warp * k + lane] = j_w;
         atomicOr(&emask[j_idx >> 5], 1u << (j_idx & 31));
-        if (blockIdx.x == 0 && a.idx_out) {
-          a.idx_out[warp * k + lane] = j_idx;
-          a.w_out[warp * k + lane] = j_w;
+        if (blockIdx.x == 0 && a.idx_out && lane < kr) {
+          a.idx_out[warp * kr + lane] = j_idx;
+          a.w_out[warp * kr + lane] = j_w;
         }
       }
     }
@@ -677,6 +686,7 @@ static void decode_fill(DecodeArgs &a, const moe_w4_layer *layer, const uint16_t
   a.hbuf = reinterpret_cast<unsigned long long *>(scratch + kDecCtrlBytes);
   a.h_polls = 1u << 20;
   a.starve_gate_up = 0;
+  a.shared = 0;
 }
 
 }  // namespace moe
@@ -725,15 +735,15 @@ extern "C" MOE_API size_t moe_decode_layer_workspace_bytes(int T, int k, int H, 
   return kDecCtrlBytes + sizeof(unsigned long long) * (size_t)T * k * ((size_t)F + (size_t)H);
 }
 
-extern "C" MOE_API moe_status moe_decode_layer_w4a16(const moe_w4_layer *layer, const uint16_t *x,
-                                                     const float *logits, int T, int k,
-                                                     uint16_t *y, int32_t *idx, float *w,
-                                                     void *ws, size_t ws_bytes,
-                                                     moe_stream_t stream) {
+// k: routed experts per token; shared: 1 = the layer's last expert is
+// shared (every token's row k, weight 1), routing over the others
+static moe_status decode_layer_w4(const moe_w4_layer *layer, const uint16_t *x, const float *logits,
+                                  int T, int k, int shared, uint16_t *y, int32_t *idx, float *w,
+                                  void *ws, size_t ws_bytes, moe_stream_t stream) {
   if (!layer || T < 0 || k <= 0) return MOE_ERR_INVALID_ARG;
-  const int E = layer->E, H = layer->H, F = layer->F;
-  if (E <= 0 || H <= 0 || F <= 0 || k > E) return MOE_ERR_INVALID_ARG;
-  if (H % 64 || F % 64 || E > kDecMaxE || T > kDecMaxTok || T * k > kDecMaxRows || k > 32)
+  const int E = layer->E, H = layer->H, F = layer->F, kk = k + shared;
+  if (E <= shared || H <= 0 || F <= 0 || k > E - shared) return MOE_ERR_INVALID_ARG;
+  if (H % 64 || F % 64 || E > kDecMaxE || T > kDecMaxTok || T * kk > kDecMaxRows || kk > 32)
     return MOE_ERR_UNSUPPORTED_SHAPE;
   if (T == 0) return MOE_OK;
   if (!layer->gate_up || !layer->down || !x || !logits || !y) return MOE_ERR_INVALID_ARG;
@@ -742,19 +752,36 @@ extern "C" MOE_API moe_status moe_decode_layer_w4a16(const moe_w4_layer *layer, 
       reinterpret_cast<uintptr_t>(layer->down) % 16 || reinterpret_cast<uintptr_t>(x) % 16 ||
       reinterpret_cast<uintptr_t>(ws) % 16)
     return MOE_ERR_INVALID_ARG;
-  if (!ws || ws_bytes < moe_decode_layer_workspace_bytes(T, k, H, F)) return MOE_ERR_WORKSPACE;
+  if (!ws || ws_bytes < moe_decode_layer_workspace_bytes(T, kk, H, F)) return MOE_ERR_WORKSPACE;
   DecodeArgs a;
-  decode_fill(a, layer, x, nullptr, T, k, nullptr, static_cast<uint8_t *>(ws));
+  decode_fill(a, layer, x, nullptr, T, kk, nullptr, static_cast<uint8_t *>(ws));
+  a.shared = shared;
   a.logits = logits;
   a.y = y;
   a.idx_out = idx;
   a.w_out = w;
   a.ybuf = reinterpret_cast<unsigned long long *>(static_cast<uint8_t *>(ws) + kDecCtrlBytes +
-                                                  sizeof(unsigned long long) * (size_t)T * k * F);
+                                                  sizeof(unsigned long long) * (size_t)T * kk * F);
   a.err = device_error_word();
   if (!a.err) return MOE_ERR_CUDA;
-  if (E <= 256) return decode_launch<kFmtW4, true, 8>(a, true, as_stream(stream));
+  if (E - shared <= 256) return decode_launch<kFmtW4, true, 8>(a, true, as_stream(stream));
   return decode_launch<kFmtW4, true, 32>(a, true, as_stream(stream));
+}
+
+extern "C" MOE_API moe_status moe_decode_layer_w4a16(const moe_w4_layer *layer, const uint16_t *x,
+                                                     const float *logits, int T, int k,
+                                                     uint16_t *y, int32_t *idx, float *w,
+                                                     void *ws, size_t ws_bytes,
+                                                     moe_stream_t stream) {
+  return decode_layer_w4(layer, x, logits, T, k, 0, y, idx, w, ws, ws_bytes, stream);
+}
+
+extern "C" MOE_API moe_status moe_decode_layer_w4a16_shared(const moe_w4_layer *layer,
+                                                            const uint16_t *x, const float *logits,
+                                                            int T, int k, uint16_t *y, int32_t *idx,
+                                                            float *w, void *ws, size_t ws_bytes,
+                                                            moe_stream_t stream) {
+  return decode_layer_w4(layer, x, logits, T, k, 1, y, idx, w, ws, ws_bytes, stream);
 }
 
 extern "C" MOE_API moe_status moe_decode_layer_nvfp4(const moe_nvfp4_layer *layer,

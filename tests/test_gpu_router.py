@@ -61,5 +61,11 @@ def test_router_route_matches_oracle(T, E, H, k):
     gap = srt[:, k - 1] - (srt[:, k] if k < E else -np.inf)
     clear = gap > 2 * bound.max(axis=1)
     assert np.array_equal(idx[clear], ridx[clear])
-    if T >= 16:  # most tokens are clear of near-ties at the k-th place
-        assert clear.mean() > 0.7
+    # the comparison is not vacuous: with the worst-case bound about 15% of
+    # tokens have the k-th gap inside it (order-statistics spacing of the
+    # logits), so most tokens are clear at large T and a quarter at least at
+    # T = 16 (16 samples of that fraction)
+    if T >= 256:
+        assert clear.mean() > 0.75
+    elif T >= 16:
+        assert clear.sum() >= T // 4
