@@ -13,10 +13,15 @@ object adds:
                            tcgen05 grouped FFN (two launches), combine
   nvfp4_prefill_512        the NVFP4 experts on 512 Zipf-routed tokens
   nvfp4_decode_T1          single-layer decode on 40 resident NVFP4 layers
-Each leg carries its own roofline (HBM GB/s or TFLOP/s against the measured
-peak), end-to-end throughput through the C ABI with host buffers, and the CPU
-oracle timed on a bounded sample of the same workload (one core and all
-cores).
+  decode_shared_T1         single-layer decode with a shared expert (weight 1)
+                           beside the 8 routed ones, one launch
+  router_T1/T2048          router linear (bf16 [256][2048]) fused with routing
+  quantize_clip_g64/sym128 the MSE clip-search quantisers (asymmetric g64,
+                           symmetric g128) on 128 MB of fp32 weights per step
+Each leg carries its own roofline (HBM GB/s, TFLOP/s or fp32 ALU ops against
+the measured or derived peak), end-to-end throughput through the C ABI with
+host buffers, and the CPU oracle timed on a bounded sample of the same
+workload (one core and all cores).
 
 Multi-GPU: one process per GPU (torchrun); each rank is an independent
 replica of the workload (the path has no exchange step): barrier + max over
@@ -65,16 +70,32 @@ NVP_WORKLOAD = ("NVFP4 grouped prefill: 512 tokens x top-8 = 4,096 routed rows o
                 "quantisation of the grouped rows, block-scaled tcgen05 grouped FFN, combine; 8 resident layers "
                 "rotated")
 
+SHARED_WORKLOAD = ("single-layer decode with a shared expert: 256 routed experts, top-8, plus one shared expert "
+                   "(weight 1) per token, hidden 2048, expert width 512, 1 token per step; steps rotate over 40 "
+                   "resident int4 layers of 257 experts")
+ROUTER_WORKLOAD = ("router linear + routing: x bf16 [{T}][2048] times a bf16 router [256][2048] (fp32 sums), softmax "
+                   "top-8 with renormalised weights, one launch; steps rotate over 160 router matrices (168 MB)")
+QUANT_WORKLOAD = ("{what}: fp32 weights N(0, 0.02) [16384][2048] (128 MB) per step, 20 clipping ratios "
+                  "1.00 -> 0.81, minimum squared error per group; two input matrices alternate")
+
 # Seeds of the synthetic inputs: weights of the int4 and NVFP4 layer sets,
 # and the activations / logits of each leg (offset by the rank).
 SEED_W4, SEED_NV = 1000, 4000
 SEED_DECODE, SEED_STREAM, SEED_PREFILL, SEED_NVP, SEED_NVD = 1000, 2000, 3000, 4000, 5000
+SEED_SHARED, SEED_ROUTER, SEED_QUANT = 6000, 7000, 8000
+PROJ_ROUTER = 2  # generator stream of a layer's router matrix (experts use 0 and 1)
+# fp32 operations per weight of the clip-search quantisers, counted from the
+# definition: per candidate asym g64 sub, div, rint, max, min, fma, sub, mul,
+# add (9); sym g128 div, rint, add, max, min, sub, mul, sub, mul, add (10)
+CLIP_OPS_PER_WEIGHT = {"clip_g64": 20 * 9, "sym128": 20 * 10}
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of a kernel, from an
 # ncu capture, with the digest of the kernel's sources at capture time.  A
 # digest that no longer matches the sources makes the bench report null.
 KERNEL_SOURCES = {
-    "decode": ["decode.cu", "common.cuh", "route.cuh", "nvfp4.cuh"],
+    "decode": ["decode.cu", "decode_common.cuh", "decode_items.cuh", "common.cuh", "route.cuh", "nvfp4.cuh"],
+    "router": ["router.cu", "route.cuh", "common.cuh"],
+    "quant": ["w4_clip.cu", "common.cuh"],
     "prefill": ["prefill.cu", "tcgen05.cuh", "common.cuh"],
     "prefill_nvfp4": ["prefill_nvfp4.cu", "tcgen05.cuh", "common.cuh", "nvfp4.cuh"],
 }
@@ -228,7 +249,9 @@ def unique_experts(logits: np.ndarray, k: int = TOPK) -> int:
 
 # ---------------------------------------------------------------------------- layers
 def build_layers(L, seed, log):
-    """Resident int4 layers, generated, quantised and packed on the GPU."""
+    """Resident int4 layers, generated, quantised and packed on the GPU.
+    Each layer holds E routed experts and, after them, a shared expert (id
+    E): the routed descriptor covers the first E, the shared one all E + 1."""
     import torch
     import synth
     import quantized_moe_route_b200 as moe
@@ -241,23 +264,24 @@ def build_layers(L, seed, log):
     layers = []
     t0 = time.time()
     for l in range(L):
-        gu = torch.empty(E * gu_b, dtype=torch.uint8, device="cuda")
-        dn = torch.empty(E * d_b, dtype=torch.uint8, device="cuda")
+        gu = torch.empty((E + 1) * gu_b, dtype=torch.uint8, device="cuda")
+        dn = torch.empty((E + 1) * d_b, dtype=torch.uint8, device="cuda")
         for proj, buf, nb, (N, K), kind in ((synth.PROJ_GATE_UP, gu, gu_b, (2 * F, H), moe.MOE_W4_GATE_UP),
                                              (synth.PROJ_DOWN, dn, d_b, (H, F), moe.MOE_W4_PLAIN)):
             G = K // 64
-            for e0 in range(0, E, chunk):
-                w = tmp.view(-1)[: chunk * N * K].view(chunk, N, K)
+            for e0 in range(0, E + 1, chunk):
+                n = min(chunk, E + 1 - e0)
+                w = tmp.view(-1)[: n * N * K].view(n, N, K)
                 synth.cuda_expert_weights(w, seed, l, e0, proj)
-                c = codes.view(-1)[: chunk * N * K].view(chunk * N, K)
-                s = sc.view(-1)[: chunk * N * G].view(chunk * N, G)
-                m = mn.view(-1)[: chunk * N * G].view(chunk * N, G)
-                moe.moe_quantize_w4(w.view(chunk * N, K), c, s, m)
-                for i in range(chunk):
+                c = codes.view(-1)[: n * N * K].view(n * N, K)
+                s = sc.view(-1)[: n * N * G].view(n * N, G)
+                m = mn.view(-1)[: n * N * G].view(n * N, G)
+                moe.moe_quantize_w4(w.view(n * N, K), c, s, m)
+                for i in range(n):
                     e = e0 + i
                     moe.moe_pack_w4(c[i * N:(i + 1) * N], s[i * N:(i + 1) * N], m[i * N:(i + 1) * N], kind,
                                     buf[e * nb:(e + 1) * nb])
-        layers.append((gu, dn, moe.make_layer(E, H, F, gu, dn)))
+        layers.append((gu, dn, moe.make_layer(E, H, F, gu, dn), moe.make_layer(E + 1, H, F, gu, dn)))
     torch.cuda.synchronize()
     del tmp, codes, sc, mn
     log(f"built {L} int4 layers in {time.time() - t0:.1f}s")
@@ -494,15 +518,19 @@ def hbm_roofline(alg_bytes, dur_ms, kernel, traffic_key, src_kernel, extra=None)
 
 
 # ---------------------------------------------------------------------------- legs
-def leg_decode(ctx, fmt, T):
-    """Single-layer decode, T tokens per step, one fused launch per step."""
+def leg_decode(ctx, fmt, T, shared=False):
+    """Single-layer decode, T tokens per step, one fused launch per step
+    (shared: each token also runs the layer's shared expert, weight 1)."""
     import torch
     import quantized_moe_route_b200 as moe
     args, k = ctx.args, TOPK
     layers = ctx.nv_layers() if fmt == "nvfp4" else ctx.w4_layers()
     nl = len(layers)
-    call = moe.moe_decode_layer_nvfp4 if fmt == "nvfp4" else moe.moe_decode_layer_w4a16
-    seed = (SEED_NVD if fmt == "nvfp4" else SEED_DECODE) + ctx.rank
+    call = (moe.moe_decode_layer_nvfp4 if fmt == "nvfp4" else
+            moe.moe_decode_layer_w4a16_shared if shared else moe.moe_decode_layer_w4a16)
+    desc = 3 if shared else 2
+    kk = k + (1 if shared else 0)
+    seed = (SEED_NVD if fmt == "nvfp4" else SEED_SHARED if shared else SEED_DECODE) + ctx.rank
     xs, ls, uniq, host = [], [], [], []
     for l in range(nl):
         x, lg = layer_inputs(seed, l, T)
@@ -511,14 +539,14 @@ def leg_decode(ctx, fmt, T):
         uniq.append(unique_experts(lg))
         host.append(pinned(torch, [x, lg]))
     y = torch.empty((T, H), dtype=torch.int16, device=ctx.dev)
-    ws = torch.zeros(moe.moe_decode_layer_workspace_bytes(T, k, H, F), dtype=torch.uint8, device=ctx.dev)
+    ws = torch.zeros(moe.moe_decode_layer_workspace_bytes(T, kk, H, F), dtype=torch.uint8, device=ctx.dev)
     stream = ctx.stream
 
     def step(i, ev=None):
         l = i % nl
         if ev is not None:
             ev[0].record(stream)
-        call(layers[l][2], xs[l], ls[l], k, y, ws, stream=stream)
+        call(layers[l][desc], xs[l], ls[l], k, y, ws, stream=stream)
         if ev is not None:
             ev[1].record(stream)
 
@@ -538,9 +566,11 @@ def leg_decode(ctx, fmt, T):
     isolated_ms = sum(a.elapsed_time(b) for a, b in evs) / P
     del g
     dur_ms = ms / K
-    alg = sum(uniq[(W + i) % nl] * EXPERT_BYTES + T * H * 2 + T * E * 4 + T * H * 2 for i in range(K)) / K
+    nexp = 1 if shared else 0  # the shared expert's weights, read once per step
+    alg = sum((uniq[(W + i) % nl] + nexp) * EXPERT_BYTES + T * H * 2 + T * E * 4 + T * H * 2
+              for i in range(K)) / K
     kname = f"moe::decode_kernel<{'nvfp4' if fmt == 'nvfp4' else 'int4'}, fused>"
-    roof = hbm_roofline(alg, dur_ms, kname, f"decode_{fmt}_T{T}", "decode",
+    roof = hbm_roofline(alg, dur_ms, kname, f"decode_{fmt}{'_shared' if shared else ''}_T{T}", "decode",
                         {"isolated_launch_us": isolated_ms * 1e3})
 
     xb = T * H * 2
@@ -548,7 +578,7 @@ def leg_decode(ctx, fmt, T):
     def e2e_step(i, din, dout):
         l = i % nl
         x_d, l_d = views(din, [(torch.int16, (T, H)), (torch.float32, (T, E))])
-        call(layers[l][2], x_d, l_d, k, dout, ws, stream=stream)
+        call(layers[l][desc], x_d, l_d, k, dout, ws, stream=stream)
 
     e2e_ms, h2d, d2h = ctx.e2e(e2e_step, host, (T, H), K, W, nl)
     assert h2d == xb + T * E * 4
@@ -556,7 +586,8 @@ def leg_decode(ctx, fmt, T):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ctx.world, "steps": K, "warmup": W,
         "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": DTYPE_NV if fmt == "nvfp4" else DTYPE_W4, "data": "synthetic",
-        "config": {"workload": NV_WORKLOAD if fmt == "nvfp4" else WORKLOAD, "experts": E, "top_k": k, "hidden": H,
+        "config": {"workload": NV_WORKLOAD if fmt == "nvfp4" else SHARED_WORKLOAD if shared else WORKLOAD,
+                   "experts": E, "top_k": k, "hidden": H, "shared_experts": nexp,
                    "expert_width": F, "tokens_per_step": T, "resident_layers": nl, "seed": seed - ctx.rank,
                    "l2": f"inputs larger than L2 ({nl}-layer rotation, {nl * E * EXPERT_BYTES / 1e9:.1f} GB); "
                          f"every resident layer touched before timing",
@@ -806,6 +837,162 @@ def leg_prefill_nvfp4(ctx, T=512, nl=8):
     }
 
 
+def alu_peak():
+    """fp32 operations per second of the SMs' FP32 pipes: 148 SMs x 128
+    lanes x one operation per clock at the maximum SM clock (an FMA counts
+    as one operation, as in the per-weight counts)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            mhz = float(json.load(f)["sm_max_mhz"])
+        kind = "derived: 148 SMs x 128 fp32 lanes x sm_max_mhz from MEASURED_PEAKS.json"
+    except Exception:
+        mhz = 1965.0
+        kind = "derived: 148 SMs x 128 fp32 lanes x 1965 MHz (nominal max clock)"
+    return 148 * 128 * mhz * 1e6 / 1e12, kind
+
+
+def leg_router(ctx, T):
+    """Router linear fused with routing (one launch per step)."""
+    import torch
+    import synth
+    import quantized_moe_route_b200 as moe
+    args, k = ctx.args, TOPK
+    dev, stream = ctx.dev, ctx.stream
+    nw = 160  # 168 MB of router matrices: a step's matrix is never in L2 from an earlier use
+    seed = SEED_ROUTER + ctx.rank
+    tmp = torch.empty((1, E, H), dtype=torch.float32, device=dev)
+    wrs = []
+    for l in range(nw):
+        synth.cuda_expert_weights(tmp, seed, l, 0, PROJ_ROUTER, sigma=1.0 / np.sqrt(H))
+        wrs.append(tmp[0].to(torch.bfloat16).view(torch.int16).clone())
+    del tmp
+    nx = 16 if T >= 1024 else 160
+    host = []
+    xs = []
+    for l in range(nx):
+        x = synth.activations_bf16(seed, l, T, H)
+        xs.append(torch.from_numpy(x.view(np.int16)).to(dev))
+        host.append(pinned(torch, [x]))
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    ws = torch.zeros(moe.moe_router_route_workspace_bytes(T, E), dtype=torch.uint8, device=dev)
+
+    def step(i, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        moe.moe_router_route(xs[i % nx], wrs[i % nw], k, idx, w, ws, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    K, W = args.steps, args.warmup
+    ms, clocks = ctx.timed(step, K, W, max(nx, nw))
+    value = job_throughput(K * T, ctx.world, ms)
+    dur_ms = ms / K
+    alg = T * H * 2 + E * H * 2 + T * E * 4 + T * k * 8  # x, Wr, logits, idx + w
+    flops = 2.0 * T * E * H
+    roof = hbm_roofline(alg, dur_ms, "moe::router_kernel", f"router_T{T}", "router",
+                        {"tflops": flops / (dur_ms / 1e3) / 1e12,
+                         "note": "HBM-bound at both sizes: at T=2048 the bytes take longer than the "
+                                 "contraction at the measured bf16 peak"})
+
+    def e2e_step(i, din, dout):
+        (x_d,) = views(din, [(torch.int16, (T, H))])
+        flat = dout.view(-1)
+        moe.moe_router_route(x_d, wrs[i % nw], k, flat[: 2 * T * k].view(torch.int32).view(T, k),
+                             flat[2 * T * k:].view(torch.float32).view(T, k), ws, stream=stream)
+
+    e2e_ms, h2d, d2h = ctx.e2e(e2e_step, host, (T, 4 * k), K, W, nx)
+    return {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "ms_per_step": dur_ms, "steps": K, "warmup": W,
+        "dtype": "bf16 x and router weights, fp32 sums",
+        "config": {"workload": ROUTER_WORKLOAD.format(T=T), "tokens_per_step": T, "experts": E, "top_k": k,
+                   "hidden": H, "seed": SEED_ROUTER,
+                   "l2": "inputs larger than L2 (160 router matrices rotated, "
+                         f"{nx} token batches of {T * H * 2 / 1e6:.1f} MB rotated)",
+                   "launch": "one kernel per step, CUDA graphs, programmatic dependent launch"},
+        "roofline": roof,
+        "e2e": {"value": job_throughput(K * T, ctx.world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "overlap": "each step's copies run on copy streams beside the neighbouring steps' kernels"},
+        "gpu_launches": K,
+        "clocks": clocks,
+    }
+
+
+def leg_quant(ctx, what):
+    """The clip-search quantisers (offline weight conversion): what =
+    "clip_g64" (asymmetric group 64) or "sym128" (symmetric group 128)."""
+    import torch
+    import synth
+    import quantized_moe_route_b200 as moe
+    args = ctx.args
+    dev, stream = ctx.dev, ctx.stream
+    N, K = 16384, 2048
+    seed = SEED_QUANT + ctx.rank
+    mats, host = [], []
+    tmp = torch.empty((16, 1024, K), dtype=torch.float32, device=dev)
+    for j in range(2):
+        synth.cuda_expert_weights(tmp, seed, j, 0, synth.PROJ_GATE_UP)
+        mats.append(tmp.view(N, K).clone())
+        host.append(mats[-1].cpu().view(torch.uint8).view(-1).pin_memory())
+    del tmp
+    codes = torch.empty((N, K), dtype=torch.uint8, device=dev)
+    gs = 64 if what == "clip_g64" else 128
+    scale = torch.empty((N, K // gs), dtype=torch.int16, device=dev)
+    minv = torch.empty((N, K // gs), dtype=torch.int16, device=dev)
+
+    def quant(w, c, sc, mn):
+        if what == "clip_g64":
+            moe.moe_quantize_w4_clip(w, c, sc, mn, stream=stream)
+        else:
+            moe.moe_quantize_w4_sym128(w, c, sc, stream=stream)
+
+    def step(i, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        quant(mats[i % 2], codes, scale, minv)
+        if ev is not None:
+            ev[1].record(stream)
+
+    Ksteps, W = min(args.steps, 50), args.warmup
+    ms, clocks = ctx.timed(step, Ksteps, W, 2)
+    dur_ms = ms / Ksteps
+    weights = N * K
+    value = job_throughput(Ksteps * weights, ctx.world, ms)
+    ops = CLIP_OPS_PER_WEIGHT[what]
+    peak, peak_kind = alu_peak()
+    achieved = weights * ops / (dur_ms / 1e3) / 1e12
+    hbm = (weights * 4 + weights + 2 * scale.numel() * (2 if what == "clip_g64" else 1)) / (dur_ms / 1e3) / 1e9
+    traffic, tsrc = traffic_of(f"quant_{what}", "quant")
+
+    def e2e_step(i, din, dout):
+        (w_d,) = views(din, [(torch.float32, (N, K))])
+        quant(w_d, dout.view(torch.uint8).view(N, K), scale, minv)
+
+    e2e_ms, h2d, d2h = ctx.e2e(e2e_step, host, (N, K // 2), Ksteps, W, 2)
+    return {
+        "metric": "weights quantised per second vs fp32 ALU roofline", "value": value, "unit": "weights/s",
+        "ms_per_step": dur_ms, "steps": Ksteps, "warmup": W,
+        "dtype": "fp32 weights -> int4 codes + f16 scales (every operation correctly rounded fp32)",
+        "config": {"workload": QUANT_WORKLOAD.format(
+            what="asymmetric group-64 int4 (f16 scale + min)" if what == "clip_g64"
+            else "symmetric group-128 int4 (f16 scale, zero point 8)"),
+            "rows": N, "cols": K, "seed": SEED_QUANT,
+            "l2": "inputs larger than L2 (two 128 MB matrices alternate)",
+            "launch": "one kernel per step, CUDA graphs"},
+        "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tops/s (fp32)",
+                     "frac": achieved / peak, "traffic": traffic, "traffic_source": tsrc,
+                     "kernel": f"moe::clip_search_kernel<{'sym' if what == 'sym128' else 'asym'}>",
+                     "peak_kind": peak_kind, "ops_per_weight": ops, "hbm_gbs": hbm,
+                     "avg_launch_us": dur_ms * 1e3},
+        "e2e": {"value": job_throughput(Ksteps * weights, ctx.world, e2e_ms), "unit": "weights/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "overlap": "each step's copies run on copy streams beside the neighbouring steps' kernels"},
+        "gpu_launches": Ksteps,
+        "clocks": clocks,
+    }
+
+
 # ---------------------------------------------------------------------------- CPU oracle
 def oracle_quantize(w, fmt):
     import oracle
@@ -841,13 +1028,37 @@ def oracle_experts(w_seed, layer, experts, fmt):
 
 
 def oracle_sample(job):
-    """The sample one oracle worker evaluates: a list of (x, logits, experts)
-    token-layers, and the tokens of the leg's unit each evaluation counts for.
+    """The sample one oracle worker evaluates: a list of zero-argument
+    evaluations, and the units of the leg's metric each evaluation counts for.
     job = (kind, fmt, w_seed, in_seed, T, worker)."""
     import oracle
     import synth
     kind, fmt, w_seed, in_seed, T, wi = job
     items = []
+    if kind == "router":  # single tokens of the batch against one router matrix
+        l = wi % 160
+        wr = synth.f32_to_bf16_bits(synth.expert_weights(w_seed, l, 0, PROJ_ROUTER, E, H, sigma=1.0 / np.sqrt(H)))
+        x = synth.activations_bf16(in_seed, wi % (16 if T >= 1024 else 160), T, H)
+        for j in range(4):
+            t = (97 * (4 * wi + j) + 13) % T
+            xt = x[t:t + 1]
+            items.append(lambda xt=xt: oracle.route(oracle.router_logits(xt, wr), TOPK))
+        return items, 1
+    if kind.startswith("quant_"):  # 64 rows of one input matrix
+        w = synth.expert_weights(in_seed, wi % 2, (64 * wi // 1024) % 16, synth.PROJ_GATE_UP, 1024, 2048)
+        r0 = (64 * wi) % 1024
+        rows = np.ascontiguousarray(w[r0:r0 + 64])
+        fn = oracle.quantize_w4_clip if kind == "quant_clip_g64" else oracle.quantize_sym128
+        return [lambda: fn(rows)], rows.size
+    if kind == "shared":
+        for j in range(2):
+            l = (2 * wi + j) % LAYERS
+            x, lg = layer_inputs(in_seed, l, T)
+            idx, _ = oracle.route(lg, TOPK)
+            ex = oracle_experts(w_seed, l, list(idx.ravel()) + [E], fmt)
+            sh = ex.pop(E)
+            items.append(lambda x=x, lg=lg, ex=ex, sh=sh: oracle.moe_forward_w4_shared(x, lg, TOPK, ex, sh))
+        return items, T
     if kind in ("decode", "stream"):
         for j in range(2):
             l = (2 * wi + j) % LAYERS
@@ -857,7 +1068,8 @@ def oracle_sample(job):
             else:
                 x, lg = layer_inputs(in_seed, l, T)
             idx, _ = oracle.route(lg, TOPK)
-            items.append((x, lg, oracle_experts(w_seed, l, idx.ravel(), fmt)))
+            ex = oracle_experts(w_seed, l, idx.ravel(), fmt)
+            items.append(lambda x=x, lg=lg, ex=ex: oracle_forward(x, lg, ex, fmt))
         # a decode step is one layer of T tokens; a stream step is 40 layers
         units = T if kind == "decode" else T / LAYERS
     else:  # prefill: single tokens of the Zipf-routed batch, layer 0
@@ -867,7 +1079,8 @@ def oracle_sample(job):
         idx, _ = oracle.route(lg, TOPK)
         for j in range(2):
             t = (97 * (2 * wi + j) + 13) % T
-            items.append((x[t:t + 1], lg[t:t + 1], oracle_experts(w_seed, 0, idx[t], fmt)))
+            ex = oracle_experts(w_seed, 0, idx[t], fmt)
+            items.append(lambda x=x[t:t + 1], lg=lg[t:t + 1], ex=ex: oracle_forward(x, lg, ex, fmt))
         units = 1
     return items, units
 
@@ -878,11 +1091,9 @@ def oracle_worker(job_budget):
     the one-core figure); touches no GPU."""
     job, deadline = job_budget
     items, units = oracle_sample(job)
-    fmt = job[1]
     n, t0 = 0, time.time()
     while True:
-        x, lg, ex = items[n % len(items)]
-        oracle_forward(x, lg, ex, fmt)
+        items[n % len(items)]()
         n += 1
         if time.time() >= deadline and n >= 1:
             break
@@ -908,7 +1119,12 @@ def cpu_baseline(kind, fmt, w_seed, in_seed, T, seconds, log, unit="tokens/s"):
     what = {"decode": f"token-layer evaluations (T={T}) over 2 sampled layers per process",
             "stream": f"layer evaluations of the 40-layer chain (T={T}, a step = 40 of them) over 2 sampled layers "
                       f"per process",
-            "prefill": f"single tokens of the {T}-token Zipf-routed batch (all 8 experts each), 2 per process"}[kind]
+            "prefill": f"single tokens of the {T}-token Zipf-routed batch (all 8 experts each), 2 per process",
+            "shared": f"token-layer evaluations (T={T}, 8 routed experts + the shared one) over 2 sampled layers "
+                      f"per process",
+            "router": f"single tokens of the {T}-token batch (router linear + routing), 4 per process",
+            "quant_clip_g64": "64 rows x 2048 of the input matrix (asymmetric g64 clip search) per process",
+            "quant_sym128": "64 rows x 2048 of the input matrix (symmetric g128 clip search) per process"}[kind]
     return {"value": allc, "unit": unit, "cores": n, "kind": "oracle",
             "sample": f"{what}; about {seconds:.0f}s per process",
             "single_core": {"value": one, "cores": 1, "sample": f"{what.split(' per process')[0]}, "
@@ -972,6 +1188,16 @@ def run_native(args, log):
     elif wl == "nvfp4-prefill":
         top = leg_prefill_nvfp4(ctx, args.tokens or 512)
         cpu_jobs["top"] = ("prefill", "nvfp4", SEED_NV, SEED_NVP, args.tokens or 512)
+    elif wl == "shared-decode":
+        top = leg_decode(ctx, "w4", args.tokens or 1, shared=True)
+        cpu_jobs["top"] = ("shared", "w4", SEED_W4, SEED_SHARED, args.tokens or 1)
+    elif wl == "router":
+        top = leg_router(ctx, args.tokens or 2048)
+        cpu_jobs["top"] = ("router", "bf16", SEED_ROUTER, SEED_ROUTER, args.tokens or 2048)
+    elif wl in ("quantize-clip", "quantize-sym128"):
+        what = "clip_g64" if wl == "quantize-clip" else "sym128"
+        top = leg_quant(ctx, what)
+        cpu_jobs["top"] = ("quant_" + what, "f32", SEED_QUANT, SEED_QUANT, 0)
     else:
         raise SystemExit(f"unknown workload {wl}")
     if wl == "all":
@@ -984,9 +1210,18 @@ def run_native(args, log):
         cpu_jobs["nvfp4_prefill_512"] = ("prefill", "nvfp4", SEED_NV, SEED_NVP, 512)
         legs["nvfp4_decode_T1"] = leg_decode(ctx, "nvfp4", 1)
         cpu_jobs["nvfp4_decode_T1"] = ("decode", "nvfp4", SEED_NV, SEED_NVD, 1)
+        legs["decode_shared_T1"] = leg_decode(ctx, "w4", 1, shared=True)
+        cpu_jobs["decode_shared_T1"] = ("shared", "w4", SEED_W4, SEED_SHARED, 1)
+        for T in (1, 2048):
+            legs[f"router_T{T}"] = leg_router(ctx, T)
+            cpu_jobs[f"router_T{T}"] = ("router", "bf16", SEED_ROUTER, SEED_ROUTER, T)
+        for what in ("clip_g64", "sym128"):
+            legs[f"quantize_{what}"] = leg_quant(ctx, what)
+            cpu_jobs[f"quantize_{what}"] = ("quant_" + what, "f32", SEED_QUANT, SEED_QUANT, 0)
     if cpu:
         for name, (kind, fmt, ws, xs, T) in cpu_jobs.items():
-            cb = cpu_baseline(kind, fmt, ws, xs, T, sec, log)
+            cb = cpu_baseline(kind, fmt, ws, xs, T, sec, log,
+                              unit="weights/s" if kind.startswith("quant_") else "tokens/s")
             (top if name == "top" else legs[name])["cpu_baseline"] = cb
     if legs:
         top["legs"] = legs
@@ -1005,7 +1240,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="all",
-                    choices=["all", "decode", "stream", "prefill", "nvfp4-decode", "nvfp4-prefill"])
+                    choices=["all", "decode", "stream", "prefill", "nvfp4-decode", "nvfp4-prefill", "shared-decode",
+                             "router", "quantize-clip", "quantize-sym128"])
     ap.add_argument("--tokens", type=int, default=None,
                     help="tokens per step of a single workload (decode 1, prefill 2048, NVFP4 prefill 512)")
     ap.add_argument("--layers", type=int, default=LAYERS,

@@ -283,9 +283,11 @@ MOE_API moe_status moe_route_shared(const float *logits, int T, int E, int k, in
  * workspace).  Source: the router stays bf16 ("Drama 3 int4 (drama-rs
  * format)", table "What's quantized"; "DRAMA-3 MLX expert-only 4-bit",
  * section "Quantization and provenance"); fp32 accumulation and no bias are
- * this library's reading.  The tensor cores sum the products in their own
- * order, so logits can differ from a sequential fp32 sum in the last bits; the
- * selection is made on the logits this call computes.
+ * this library's reading.  The products are summed in the kernel's own
+ * fixed order (fp32 FMAs in a fixed tree up to 16 tokens, the tensor cores
+ * above), so logits can differ from a sequential fp32 sum in the last bits
+ * but not from call to call; the selection is made on the logits this call
+ * computes.
  * Workspace: moe_router_route_workspace_bytes(T, E) bytes, 16-byte aligned,
  * zero-filled before its first use; every call leaves it ready for the next
  * stream-ordered call.  Limits: E % 16 == 0 (E % 64 == 0 above 64), E <=

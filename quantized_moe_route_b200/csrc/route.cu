@@ -44,6 +44,10 @@ static moe_status route_launch(const float *logits, int T, int E, int k, int sha
   return launch_pdl(kern, grid, dim3(threads), 0, s, logits, T, E, k, shared, idx, w);
 }
 
+moe_status route_rows(const float *logits, int T, int E, int k, int32_t *idx, float *w, cudaStream_t stream) {
+  return route_launch(logits, T, E, k, 0, idx, w, reinterpret_cast<moe_stream_t>(stream));
+}
+
 }  // namespace moe
 
 using namespace moe;

@@ -13,6 +13,10 @@ namespace moe {
 
 constexpr int kRouteMaxPerLane = 32;  // E <= 1024
 
+// moe_route's kernel on finished logits (one warp per token), launched with
+// programmatic dependent launch; for other launchers of the library
+moe_status route_rows(const float *logits, int T, int E, int k, int32_t *idx, float *w, cudaStream_t stream);
+
 // One warp, one token.  Lane l owns experts l, l + 32, l + 64, ...
 // (coalesced loads).  Each of the k rounds takes the warp-wide maximum
 // (value, then lowest id) of the not-yet-taken experts with two single-

@@ -39,8 +39,9 @@ def _router(x, wr, k):
     return out
 
 
-@pytest.mark.parametrize("T,E,H,k", [(1, 256, 2048, 8), (16, 256, 2048, 8), (37, 64, 512, 4),
-                                     (2048, 256, 2048, 8), (5, 1024, 256, 8), (3, 16, 64, 2), (70, 48, 128, 3)])
+@pytest.mark.parametrize("T,E,H,k", [(1, 256, 2048, 8), (16, 256, 2048, 8), (17, 256, 2048, 8), (37, 64, 512, 4),
+                                     (2048, 256, 2048, 8), (5, 1024, 256, 8), (3, 16, 64, 2), (70, 48, 128, 3),
+                                     (65, 128, 4096, 4), (300, 1024, 128, 16), (9, 1024, 64, 1)])
 def test_router_route_matches_oracle(T, E, H, k):
     seed = 300 + T + E
     x = synth.activations_bf16(seed, 0, T, H)
