@@ -347,7 +347,8 @@ MOE_API moe_status moe_permute(const int32_t *idx, int T, int k, int E, const ui
  * process under MPS) holds SMs, the GPU starts the grid only once every block
  * can run, instead of starting part of it.  The same holds for
  * moe_decode_layer_w4a16, moe_decode_layer_w4a16_shared,
- * moe_decode_layer_nvfp4 and moe_ffn_w4a16_decode_static.
+ * moe_decode_layer_w4a16_router, moe_decode_layer_nvfp4 and
+ * moe_ffn_w4a16_decode_static.
  */
 MOE_API size_t moe_decode_workspace_bytes(int T, int k, int F);
 MOE_API moe_status moe_ffn_w4a16_decode(const moe_w4_layer *layer, const uint16_t *x,
@@ -393,6 +394,33 @@ MOE_API moe_status moe_decode_layer_w4a16_shared(const moe_w4_layer *layer, cons
                                                  const float *logits, int T, int k, uint16_t *y,
                                                  int32_t *idx, float *w, void *ws, size_t ws_bytes,
                                                  moe_stream_t stream);
+
+/*
+ * The decode layer with the router linear inside the same launch: the kernel
+ * computes logits[t][e] = sum_c x[t][c] * Wr[e][c] (x and Wr bf16 [E - shared]
+ * [H], fp32 FMAs, no bias) for the routed experts, routes on them as
+ * moe_route, and runs the layer as moe_decode_layer_w4a16 (shared = 0) or
+ * moe_decode_layer_w4a16_shared (shared = 1: the layer's last expert is the
+ * shared expert).  Each expert row's logits are summed by one warp: lane l
+ * takes channels 8l .. 8l+7 of every 256 in order, then the 32 lanes' sums
+ * meet in a fixed xor-shuffle tree, so the logits do not change from call to
+ * call; they can differ from moe_router_route's (another order) in the last
+ * bits.  logits fp32 [T][E - shared], idx / w [T][k]: optional outputs
+ * (idx and w both or neither).  Wr 16-byte aligned.
+ * Workspace: moe_decode_layer_router_workspace_bytes(T, k, shared, E, H, F)
+ * (E = layer->E), zero-filled before first use, reusable by stream-ordered
+ * calls.  Limits as for the call it extends.  A wait for a logit that times
+ * out (it cannot while every block is resident) raises
+ * MOE_DEVERR_DECODE_ROUTER_WAIT.  Source: the router stays bf16 ("Drama 3
+ * int4 (drama-rs format)", table "What's quantized"; "DRAMA-3 MLX
+ * expert-only 4-bit", "Quantization and provenance"), and the passages of the
+ * calls it extends.
+ */
+MOE_API size_t moe_decode_layer_router_workspace_bytes(int T, int k, int shared, int E, int H, int F);
+MOE_API moe_status moe_decode_layer_w4a16_router(const moe_w4_layer *layer, const uint16_t *x,
+                                                 const uint16_t *wr, int T, int k, int shared,
+                                                 uint16_t *y, int32_t *idx, float *w, float *logits,
+                                                 void *ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
  * The NVFP4 form of moe_decode_layer_w4a16: one launch routes the T tokens,
@@ -513,6 +541,7 @@ MOE_API moe_status moe_device_error(int *out, moe_stream_t stream);
 
 /* Codes of the device error word. */
 #define MOE_DEVERR_DECODE_H_WAIT 0x101 /* decode: a wait for h or a row output gave up */
+#define MOE_DEVERR_DECODE_ROUTER_WAIT 0x102 /* decode with the router: a wait for a logit gave up */
 #define MOE_DEVERR_PREFILL_WAIT 0x201  /* prefill: a pipeline barrier wait gave up */
 
 /*

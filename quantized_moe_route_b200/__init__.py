@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(HERE, "libmoe.so")
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE = 0, 1, 2
 MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = 3, 4, 5
 MOE_DEVERR_DECODE_H_WAIT, MOE_DEVERR_PREFILL_WAIT = 0x101, 0x201
+MOE_DEVERR_DECODE_ROUTER_WAIT = 0x102
 MOE_W4_PLAIN, MOE_W4_GATE_UP = 0, 1
 
 _lib = None
@@ -80,6 +81,9 @@ SIGNATURES = {
                                     _vp]),
     "moe_decode_layer_w4a16_shared": (_i, [ctypes.POINTER(moe_w4_layer), _vp, _vp, _i, _i, _vp, _vp, _vp, _vp,
                                            _sz, _vp]),
+    "moe_decode_layer_router_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "moe_decode_layer_w4a16_router": (_i, [ctypes.POINTER(moe_w4_layer), _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp,
+                                           _vp, _sz, _vp]),
     "moe_decode_layer_nvfp4": (_i, [ctypes.POINTER(moe_nvfp4_layer), _vp, _vp, _i, _i, _vp, _vp, _vp, _vp,
                                     _sz, _vp]),
     "moe_prefill_workspace_bytes": (_sz, [_i, _i]),
@@ -295,6 +299,20 @@ def moe_decode_layer_w4a16_shared(layer: moe_w4_layer, x, logits, k, y, ws, idx=
     _check(lib().moe_decode_layer_w4a16_shared(ctypes.byref(layer), _p(x), _p(logits), T, k, _p(y), _p(idx),
                                                _p(w), _p(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "moe_decode_layer_w4a16_shared")
+
+
+def moe_decode_layer_router_workspace_bytes(T, k, shared, E, H, F) -> int:
+    return lib().moe_decode_layer_router_workspace_bytes(T, k, shared, E, H, F)
+
+
+def moe_decode_layer_w4a16_router(layer: moe_w4_layer, x, wr, k, y, ws, shared=0, idx=None, w=None, logits=None,
+                                  stream=None):
+    """One layer in one launch from x and the bf16 router weights wr [E - shared][H]:
+    router linear, routing, expert FFN (plus the shared expert), combine."""
+    T = x.shape[0]
+    _check(lib().moe_decode_layer_w4a16_router(ctypes.byref(layer), _p(x), _p(wr), T, k, shared, _p(y), _p(idx),
+                                               _p(w), _p(logits), _p(ws), ws.numel() * ws.element_size(),
+                                               _stream(stream)), "moe_decode_layer_w4a16_router")
 
 
 def moe_decode_layer_nvfp4(layer: moe_nvfp4_layer, x, logits, k, y, ws, idx=None, w=None, stream=None):

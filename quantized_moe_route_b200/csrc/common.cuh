@@ -50,6 +50,7 @@ inline moe_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
 enum : int {
   DEVERR_NONE = 0,
   DEVERR_DECODE_H_WAIT = 0x101,   // decode: down projection waited too long for h
+  DEVERR_DECODE_ROUTER_WAIT = 0x102,  // decode: routing waited too long for a logit
   DEVERR_PREFILL_WAIT = 0x201,    // prefill: a pipeline barrier wait gave up
 };
 int *device_error_word();  // device address of the word on the current device

@@ -47,7 +47,11 @@
 namespace moe {
 
 struct DecodeArgs {
-  const float *logits;       // fused form: router logits [T][E]
+  const float *logits;       // fused form: router logits [T][E] (unless wr)
+  const uint16_t *wr;        // fused int4 form, optional: bf16 router weights [E - shared][H];
+                             // the kernel computes the logits
+  unsigned long long *lbuf;  // with wr: [T][E - shared] words {fp32 logit, epoch}
+  float *logits_out;         // with wr, optional: the computed logits fp32 [T][E - shared]
   uint16_t *y;               // fused form: combined bf16 output [T][H]
   int32_t *idx_out;          // fused form, optional: routing of every token
   float *w_out;
@@ -192,6 +196,61 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
                          pol);
   };
 
+  // ---- router linear (with wr): each CTA computes the logits of its
+  // experts e = blockIdx.x + G * (warp + kDecWarps * i), one warp per expert
+  // row: lane l sums channels 8 l .. 8 l + 7 of every 256 in fp32 FMAs, the
+  // lanes' sums meet in an xor-shuffle tree (a fixed order), and lane t
+  // publishes token t's logit as a word {logit, epoch} for every CTA's
+  // routing below.  All CTAs are resident together (cooperative launch) and
+  // this phase waits on nothing but x, so every word gets written.
+  if (kFused && !kFp4 && a.wr != nullptr) {
+    const int Er = E - a.shared;
+    if (tid == kDecThreads - 1) {
+      const unsigned int ep = ctrl0 + 1u;  // this call's epoch; never 0 (zeroed words never match)
+      misc[2] = (int)(ep == 0u ? 1u : ep);
+    }
+    const int e_first = (int)blockIdx.x + G * warp;
+    if (e_first < Er)  // start the first row's lines on their way to L2 while x lands
+      for (int ln = lane; ln < H / 64; ln += 32)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(a.wr + (size_t)e_first * H + 64 * ln));
+    cp_async_wait_all();
+    __syncthreads();
+    const unsigned int ep = (unsigned int)misc[2];
+    for (int e = e_first; e < Er; e += G * kDecWarps) {
+      float acc[kDecMaxTok];
+#pragma unroll
+      for (int t = 0; t < kDecMaxTok; ++t) acc[t] = 0.f;
+      const uint16_t *row = a.wr + (size_t)e * H;
+      for (int c = 8 * lane; c < H; c += 256) {
+        float wf[8];
+        bf16x8_f32(__ldg(reinterpret_cast<const uint4 *>(row + c)), wf);
+#pragma unroll
+        for (int t = 0; t < kDecMaxTok; ++t) {
+          if (t < T) {
+            float xf[8];
+            bf16x8_f32(*reinterpret_cast<const uint4 *>(x_s + (size_t)t * H + c), xf);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[t] = __fmaf_rn(xf[i], wf[i], acc[t]);
+          }
+        }
+      }
+      float mine = 0.f;
+#pragma unroll
+      for (int t = 0; t < kDecMaxTok; ++t) {
+        if (t < T) {
+          float v = acc[t];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+          if (lane == t) mine = v;
+        }
+      }
+      if (lane < T) {
+        a.lbuf[(size_t)lane * Er + e] = ((unsigned long long)__float_as_uint(mine) << 32) | ep;
+        if (a.logits_out) a.logits_out[(size_t)lane * Er + e] = mine;
+      }
+    }
+  }
+
   // ---- routing table.  Unique experts in increasing id ("slots"); the
   // first weight copies go out as soon as the slots are known.
   if (kFused) {  // warp t routes token t
@@ -199,9 +258,45 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
       // with a shared expert the router scores the Er = E - 1 routed experts
       // and row kr = k - 1 is the shared expert's, weight 1
       const int kr = k - a.shared, Er = E - a.shared;
+      uint32_t key[PER];
+      if (!kFp4 && a.wr != nullptr) {
+        // this token's logit words, all requested at once, then each one
+        // polled again until it carries this call's epoch (bounded)
+        const unsigned int ep = (unsigned int)misc[2];
+        const unsigned long long *lw = a.lbuf + (size_t)warp * Er;
+        unsigned long long wv[PER];
+#pragma unroll
+        for (int i = 0; i < PER; ++i) wv[i] = lane + 32 * i < Er ? ld_relaxed_u64(lw + lane + 32 * i) : 0ull;
+        bool ok = true;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+          const int e = lane + 32 * i;
+          if (e < Er) {
+            uint32_t spins = 0;
+            while (ok && (unsigned int)(wv[i] & 0xFFFFFFFFull) != ep) {
+              if (++spins > (1u << 22)) {
+                ok = false;  // the logit is used as read; the error word tells the caller
+                atomicExch(a.err, DEVERR_DECODE_ROUTER_WAIT);
+                break;
+              }
+              __nanosleep(32);
+              wv[i] = ld_relaxed_u64(lw + e);
+            }
+            key[i] = route_key(__uint_as_float((unsigned int)(wv[i] >> 32)));
+          } else {
+            key[i] = 0u;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+          const int e = lane + 32 * i;
+          key[i] = e < Er ? route_key(a.logits[(size_t)warp * Er + e]) : 0u;
+        }
+      }
       int j_idx;
       float j_w;
-      route_token_warp<PER>(a.logits + (size_t)warp * Er, Er, kr, &j_idx, &j_w);
+      route_token_keys<PER>(key, kr, &j_idx, &j_w);
       if (lane == kr) {  // only reached with a shared expert (kr < k)
         j_idx = Er;
         j_w = 1.0f;
@@ -222,7 +317,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
     ridx[tid] = e;
     atomicOr(&emask[e >> 5], 1u << (e & 31));
   }
-  if (tid == kDecThreads - 1) {
+  if (tid == kDecThreads - 1 && !(kFused && !kFp4 && a.wr != nullptr)) {  // (set above with wr)
     const unsigned int ep = ctrl0 + 1u;  // this call's epoch; never 0 (zeroed words never match)
     misc[2] = (int)(ep == 0u ? 1u : ep);
   }
@@ -687,6 +782,9 @@ static void decode_fill(DecodeArgs &a, const moe_w4_layer *layer, const uint16_t
   a.h_polls = 1u << 20;
   a.starve_gate_up = 0;
   a.shared = 0;
+  a.wr = nullptr;
+  a.lbuf = nullptr;
+  a.logits_out = nullptr;
 }
 
 }  // namespace moe
@@ -736,27 +834,37 @@ extern "C" MOE_API size_t moe_decode_layer_workspace_bytes(int T, int k, int H, 
 }
 
 // k: routed experts per token; shared: 1 = the layer's last expert is
-// shared (every token's row k, weight 1), routing over the others
+// shared (every token's row k, weight 1), routing over the others.
+// Exactly one of logits (given) and wr (router weights: the kernel computes
+// the logits, optionally copied to logits_out) is non-null.
 static moe_status decode_layer_w4(const moe_w4_layer *layer, const uint16_t *x, const float *logits,
-                                  int T, int k, int shared, uint16_t *y, int32_t *idx, float *w,
-                                  void *ws, size_t ws_bytes, moe_stream_t stream) {
-  if (!layer || T < 0 || k <= 0) return MOE_ERR_INVALID_ARG;
+                                  const uint16_t *wr, float *logits_out, int T, int k, int shared,
+                                  uint16_t *y, int32_t *idx, float *w, void *ws, size_t ws_bytes,
+                                  moe_stream_t stream) {
+  if (!layer || T < 0 || k <= 0 || shared < 0 || shared > 1) return MOE_ERR_INVALID_ARG;
   const int E = layer->E, H = layer->H, F = layer->F, kk = k + shared;
   if (E <= shared || H <= 0 || F <= 0 || k > E - shared) return MOE_ERR_INVALID_ARG;
   if (H % 64 || F % 64 || E > kDecMaxE || T > kDecMaxTok || T * kk > kDecMaxRows || kk > 32)
     return MOE_ERR_UNSUPPORTED_SHAPE;
   if (T == 0) return MOE_OK;
-  if (!layer->gate_up || !layer->down || !x || !logits || !y) return MOE_ERR_INVALID_ARG;
+  if (!layer->gate_up || !layer->down || !x || (!logits == !wr) || !y) return MOE_ERR_INVALID_ARG;
   if ((idx == nullptr) != (w == nullptr)) return MOE_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(layer->gate_up) % 16 ||
       reinterpret_cast<uintptr_t>(layer->down) % 16 || reinterpret_cast<uintptr_t>(x) % 16 ||
-      reinterpret_cast<uintptr_t>(ws) % 16)
+      reinterpret_cast<uintptr_t>(ws) % 16 || reinterpret_cast<uintptr_t>(wr) % 16)
     return MOE_ERR_INVALID_ARG;
-  if (!ws || ws_bytes < moe_decode_layer_workspace_bytes(T, kk, H, F)) return MOE_ERR_WORKSPACE;
+  const size_t need = wr ? moe_decode_layer_router_workspace_bytes(T, k, shared, E, H, F)
+                         : moe_decode_layer_workspace_bytes(T, kk, H, F);
+  if (!ws || ws_bytes < need) return MOE_ERR_WORKSPACE;
   DecodeArgs a;
   decode_fill(a, layer, x, nullptr, T, kk, nullptr, static_cast<uint8_t *>(ws));
   a.shared = shared;
   a.logits = logits;
+  a.wr = wr;
+  a.logits_out = logits_out;
+  a.lbuf = wr ? reinterpret_cast<unsigned long long *>(static_cast<uint8_t *>(ws) +
+                                                      moe_decode_layer_workspace_bytes(T, kk, H, F))
+              : nullptr;
   a.y = y;
   a.idx_out = idx;
   a.w_out = w;
@@ -773,7 +881,8 @@ extern "C" MOE_API moe_status moe_decode_layer_w4a16(const moe_w4_layer *layer, 
                                                      uint16_t *y, int32_t *idx, float *w,
                                                      void *ws, size_t ws_bytes,
                                                      moe_stream_t stream) {
-  return decode_layer_w4(layer, x, logits, T, k, 0, y, idx, w, ws, ws_bytes, stream);
+  if (!logits) return MOE_ERR_INVALID_ARG;
+  return decode_layer_w4(layer, x, logits, nullptr, nullptr, T, k, 0, y, idx, w, ws, ws_bytes, stream);
 }
 
 extern "C" MOE_API moe_status moe_decode_layer_w4a16_shared(const moe_w4_layer *layer,
@@ -781,7 +890,24 @@ extern "C" MOE_API moe_status moe_decode_layer_w4a16_shared(const moe_w4_layer *
                                                             int T, int k, uint16_t *y, int32_t *idx,
                                                             float *w, void *ws, size_t ws_bytes,
                                                             moe_stream_t stream) {
-  return decode_layer_w4(layer, x, logits, T, k, 1, y, idx, w, ws, ws_bytes, stream);
+  if (!logits) return MOE_ERR_INVALID_ARG;
+  return decode_layer_w4(layer, x, logits, nullptr, nullptr, T, k, 1, y, idx, w, ws, ws_bytes, stream);
+}
+
+extern "C" MOE_API size_t moe_decode_layer_router_workspace_bytes(int T, int k, int shared, int E, int H,
+                                                                  int F) {
+  if (T <= 0 || k <= 0 || shared < 0 || shared > 1 || E <= shared || H <= 0 || F <= 0) return 0;
+  return moe_decode_layer_workspace_bytes(T, k + shared, H, F) +
+         sizeof(unsigned long long) * (size_t)T * (size_t)(E - shared);
+}
+
+extern "C" MOE_API moe_status moe_decode_layer_w4a16_router(const moe_w4_layer *layer, const uint16_t *x,
+                                                            const uint16_t *wr, int T, int k, int shared,
+                                                            uint16_t *y, int32_t *idx, float *w,
+                                                            float *logits, void *ws, size_t ws_bytes,
+                                                            moe_stream_t stream) {
+  if (!wr) return MOE_ERR_INVALID_ARG;
+  return decode_layer_w4(layer, x, nullptr, wr, logits, T, k, shared, y, idx, w, ws, ws_bytes, stream);
 }
 
 extern "C" MOE_API moe_status moe_decode_layer_nvfp4(const moe_nvfp4_layer *layer,

@@ -63,6 +63,16 @@ __device__ __forceinline__ int warp_inclusive_scan(int v) {
   return v;
 }
 
+// eight bf16 (16 bytes) -> fp32, exact
+__device__ __forceinline__ void bf16x8_f32(const uint4 &v, float f[8]) {
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(u[i] << 16);
+    f[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
+  }
+}
+
 __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long *p) {
   unsigned long long v;
   asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");

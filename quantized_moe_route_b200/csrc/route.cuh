@@ -36,16 +36,11 @@ __device__ __forceinline__ float route_key_value(uint32_t key) {
   return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
 }
 
+// The selection from the lanes' keys: key[i] is expert lane + 32 i's
+// route_key (0 past the last expert).
 template <int PER>
-__device__ __forceinline__ void route_token_warp(const float *__restrict__ l, int E, int k,
-                                                 int *idx_j, float *w_j) {
+__device__ __forceinline__ void route_token_keys(const uint32_t (&key)[PER], int k, int *idx_j, float *w_j) {
   const int lane = threadIdx.x & 31;
-  uint32_t key[PER];
-#pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    const int e = lane + 32 * i;
-    key[i] = e < E ? route_key(l[e]) : 0u;
-  }
   uint32_t taken = 0;  // bit i: expert lane + 32 i already selected
   // local best of the untaken entries: entries visited in increasing id and
   // strict > keeps the lowest id among equal keys; key 0 = nothing left
@@ -83,6 +78,19 @@ __device__ __forceinline__ void route_token_warp(const float *__restrict__ l, in
   }
   *idx_j = my_idx;
   *w_j = my_w / denom;
+}
+
+template <int PER>
+__device__ __forceinline__ void route_token_warp(const float *__restrict__ l, int E, int k,
+                                                 int *idx_j, float *w_j) {
+  const int lane = threadIdx.x & 31;
+  uint32_t key[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = lane + 32 * i;
+    key[i] = e < E ? route_key(l[e]) : 0u;
+  }
+  route_token_keys<PER>(key, k, idx_j, w_j);
 }
 
 }  // namespace moe
