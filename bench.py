@@ -15,6 +15,8 @@ object adds:
   nvfp4_decode_T1          single-layer decode on 40 resident NVFP4 layers
   decode_shared_T1         single-layer decode with a shared expert (weight 1)
                            beside the 8 routed ones, one launch
+  decode_router_T1         single-layer decode with the router linear inside
+                           the same launch (x and the bf16 router in)
   router_T1/T2048          router linear (bf16 [256][2048]) fused with routing
   quantize_clip_g64/sym128 the MSE clip-search quantisers (asymmetric g64,
                            symmetric g128) on 128 MB of fp32 weights per step
@@ -75,6 +77,9 @@ SHARED_WORKLOAD = ("single-layer decode with a shared expert: 256 routed experts
                    "resident int4 layers of 257 experts")
 ROUTER_WORKLOAD = ("router linear + routing: x bf16 [{T}][2048] times a bf16 router [256][2048] (fp32 sums), softmax "
                    "top-8 with renormalised weights, one launch; steps rotate over 160 router matrices (168 MB)")
+RDEC_WORKLOAD = ("single-layer decode with the router inside: x bf16 [{T}][2048] and a bf16 router [256][2048] in, "
+                 "logits, top-8 routing, 256 int4 experts (expert width 512) and combine in one launch; steps rotate "
+                 "over 40 resident layers (18.1 GB of experts, 40 router matrices)")
 QUANT_WORKLOAD = ("{what}: fp32 weights N(0, 0.02) [16384][2048] (128 MB) per step, 20 clipping ratios "
                   "1.00 -> 0.81, minimum squared error per group; two input matrices alternate")
 
@@ -82,7 +87,7 @@ QUANT_WORKLOAD = ("{what}: fp32 weights N(0, 0.02) [16384][2048] (128 MB) per st
 # and the activations / logits of each leg (offset by the rank).
 SEED_W4, SEED_NV = 1000, 4000
 SEED_DECODE, SEED_STREAM, SEED_PREFILL, SEED_NVP, SEED_NVD = 1000, 2000, 3000, 4000, 5000
-SEED_SHARED, SEED_ROUTER, SEED_QUANT = 6000, 7000, 8000
+SEED_SHARED, SEED_ROUTER, SEED_QUANT, SEED_RDEC = 6000, 7000, 8000, 9000
 PROJ_ROUTER = 2  # generator stream of a layer's router matrix (experts use 0 and 1)
 # fp32 operations per weight of the clip-search quantisers, counted from the
 # definition: per candidate asym g64 sub, div, rint, max, min, fma, sub, mul,
@@ -837,6 +842,75 @@ def leg_prefill_nvfp4(ctx, T=512, nl=8):
     }
 
 
+def leg_decode_router(ctx, T):
+    """Single-layer decode with the router linear in the same launch: x and
+    the layer's bf16 router matrix in, y out."""
+    import torch
+    import synth
+    import quantized_moe_route_b200 as moe
+    args, k = ctx.args, TOPK
+    layers = ctx.w4_layers()
+    nl = len(layers)
+    dev, stream = ctx.dev, ctx.stream
+    seed = SEED_RDEC + ctx.rank
+    tmp = torch.empty((1, E, H), dtype=torch.float32, device=dev)
+    wrs, xs, host = [], [], []
+    for l in range(nl):
+        synth.cuda_expert_weights(tmp, seed, l, 0, PROJ_ROUTER, sigma=1.0 / np.sqrt(H))
+        wrs.append(tmp[0].to(torch.bfloat16).view(torch.int16).clone())
+        x = synth.activations_bf16(seed, l, T, H)
+        xs.append(torch.from_numpy(x.view(np.int16)).to(dev))
+        host.append(pinned(torch, [x]))
+    del tmp
+    y = torch.empty((T, H), dtype=torch.int16, device=dev)
+    ws = torch.zeros(moe.moe_decode_layer_router_workspace_bytes(T, k, 0, E, H, F), dtype=torch.uint8, device=dev)
+    # the experts each layer's call selects (for the byte count), from one untimed call per layer
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    uniq = []
+    for l in range(nl):
+        moe.moe_decode_layer_w4a16_router(layers[l][2], xs[l], wrs[l], k, y, ws, idx=idx, w=w, stream=stream)
+        stream.synchronize()
+        uniq.append(len(np.unique(idx.cpu().numpy())))
+
+    def step(i, ev=None):
+        l = i % nl
+        if ev is not None:
+            ev[0].record(stream)
+        moe.moe_decode_layer_w4a16_router(layers[l][2], xs[l], wrs[l], k, y, ws, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    K, W = args.steps, args.warmup
+    ms, clocks = ctx.timed(step, K, W, nl)
+    value = job_throughput(K * T, ctx.world, ms)
+    dur_ms = ms / K
+    alg = sum(uniq[(W + i) % nl] * EXPERT_BYTES + E * H * 2 + T * H * 2 + T * H * 2 for i in range(K)) / K
+    roof = hbm_roofline(alg, dur_ms, "moe::decode_kernel<int4, fused> (router inside)", f"decode_router_T{T}",
+                        "decode", {"router_bytes_per_launch": E * H * 2})
+
+    def e2e_step(i, din, dout):
+        (x_d,) = views(din, [(torch.int16, (T, H))])
+        moe.moe_decode_layer_w4a16_router(layers[i % nl][2], x_d, wrs[i % nl], k, dout, ws, stream=stream)
+
+    e2e_ms, h2d, d2h = ctx.e2e(e2e_step, host, (T, H), K, W, nl)
+    return {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "ms_per_step": dur_ms, "steps": K, "warmup": W,
+        "dtype": DTYPE_W4 + "; bf16 router, fp32 logits",
+        "config": {"workload": RDEC_WORKLOAD.format(T=T), "tokens_per_step": T, "experts": E, "top_k": k,
+                   "hidden": H, "expert_width": F, "resident_layers": nl, "seed": SEED_RDEC,
+                   "l2": f"inputs larger than L2 ({nl}-layer rotation); every resident layer touched before timing",
+                   "launch": "one kernel per step (router linear + route + FFN + combine), CUDA graphs, "
+                             "programmatic dependent launch"},
+        "roofline": roof,
+        "e2e": {"value": job_throughput(K * T, ctx.world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "overlap": "each step's copies run on copy streams beside the neighbouring steps' kernels"},
+        "gpu_launches": K,
+        "clocks": clocks,
+    }
+
+
 def alu_peak():
     """fp32 operations per second of the SMs' FP32 pipes: 148 SMs x 128
     lanes x one operation per clock at the maximum SM clock (an FMA counts
@@ -1050,6 +1124,16 @@ def oracle_sample(job):
         rows = np.ascontiguousarray(w[r0:r0 + 64])
         fn = oracle.quantize_w4_clip if kind == "quant_clip_g64" else oracle.quantize_sym128
         return [lambda: fn(rows)], rows.size
+    if kind == "router_decode":  # router linear + one layer, 2 sampled token-layers
+        for j in range(2):
+            l = (2 * wi + j) % LAYERS
+            wr = synth.f32_to_bf16_bits(synth.expert_weights(in_seed, l, 0, PROJ_ROUTER, E, H, sigma=1.0 / np.sqrt(H)))
+            x = synth.activations_bf16(in_seed, l, T, H)
+            lg = oracle.router_logits(x, wr)
+            idx, _ = oracle.route(lg, TOPK)
+            ex = oracle_experts(w_seed, l, idx.ravel(), fmt)
+            items.append(lambda x=x, wr=wr, ex=ex: oracle.moe_forward_w4(x, oracle.router_logits(x, wr), TOPK, ex))
+        return items, T
     if kind == "shared":
         for j in range(2):
             l = (2 * wi + j) % LAYERS
@@ -1123,6 +1207,8 @@ def cpu_baseline(kind, fmt, w_seed, in_seed, T, seconds, log, unit="tokens/s"):
             "shared": f"token-layer evaluations (T={T}, 8 routed experts + the shared one) over 2 sampled layers "
                       f"per process",
             "router": f"single tokens of the {T}-token batch (router linear + routing), 4 per process",
+            "router_decode": f"token-layer evaluations (T={T}, router linear + routing + 8 experts + combine) over "
+                             f"2 sampled layers per process",
             "quant_clip_g64": "64 rows x 2048 of the input matrix (asymmetric g64 clip search) per process",
             "quant_sym128": "64 rows x 2048 of the input matrix (symmetric g128 clip search) per process"}[kind]
     return {"value": allc, "unit": unit, "cores": n, "kind": "oracle",
@@ -1191,6 +1277,9 @@ def run_native(args, log):
     elif wl == "shared-decode":
         top = leg_decode(ctx, "w4", args.tokens or 1, shared=True)
         cpu_jobs["top"] = ("shared", "w4", SEED_W4, SEED_SHARED, args.tokens or 1)
+    elif wl == "router-decode":
+        top = leg_decode_router(ctx, args.tokens or 1)
+        cpu_jobs["top"] = ("router_decode", "w4", SEED_W4, SEED_RDEC, args.tokens or 1)
     elif wl == "router":
         top = leg_router(ctx, args.tokens or 2048)
         cpu_jobs["top"] = ("router", "bf16", SEED_ROUTER, SEED_ROUTER, args.tokens or 2048)
@@ -1212,6 +1301,8 @@ def run_native(args, log):
         cpu_jobs["nvfp4_decode_T1"] = ("decode", "nvfp4", SEED_NV, SEED_NVD, 1)
         legs["decode_shared_T1"] = leg_decode(ctx, "w4", 1, shared=True)
         cpu_jobs["decode_shared_T1"] = ("shared", "w4", SEED_W4, SEED_SHARED, 1)
+        legs["decode_router_T1"] = leg_decode_router(ctx, 1)
+        cpu_jobs["decode_router_T1"] = ("router_decode", "w4", SEED_W4, SEED_RDEC, 1)
         for T in (1, 2048):
             legs[f"router_T{T}"] = leg_router(ctx, T)
             cpu_jobs[f"router_T{T}"] = ("router", "bf16", SEED_ROUTER, SEED_ROUTER, T)
@@ -1241,7 +1332,7 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="all",
                     choices=["all", "decode", "stream", "prefill", "nvfp4-decode", "nvfp4-prefill", "shared-decode",
-                             "router", "quantize-clip", "quantize-sym128"])
+                             "router", "router-decode", "quantize-clip", "quantize-sym128"])
     ap.add_argument("--tokens", type=int, default=None,
                     help="tokens per step of a single workload (decode 1, prefill 2048, NVFP4 prefill 512)")
     ap.add_argument("--layers", type=int, default=LAYERS,

@@ -78,7 +78,7 @@ struct DecodeArgs {
 
 struct DecodeSmem {
   // byte offsets into dynamic shared memory
-  uint32_t stages, x, xsum, hsum, bars, meta, total;
+  uint32_t stages, x, xsum, hsum, bars, rbars, meta, total;
 };
 
 
@@ -113,6 +113,7 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int fmt, int T, int H, 
   L.xsum = take(fmt == kFmtW4 ? (uint32_t)T * (H / 64) * 4 : 2u * T * 4, 16);
   L.hsum = take(fmt == kFmtW4 ? 2u * T * (F / 64) * 4 : 2u * 2u * T * 4, 16);
   L.bars = take((uint32_t)nstages * 8, 8);
+  L.rbars = take(kDecWarps * 8, 8);  // router-row copies, one barrier per warp
   L.meta = take(3600 * 4, 16);  // routing tables + 256 x 8 row-set words
   L.total = o;
   return L;
@@ -154,8 +155,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
   const uint32_t stripA = (uint32_t)Gh * kBlkBytes, stripB = (uint32_t)Gf * kBlkBytes;
   const int G = gridDim.x;
 
+  uint64_t *rbars = reinterpret_cast<uint64_t *>(smem + L.rbars);
   if (tid == 0) {
     for (int s = 0; s < a.nstages; ++s) mbar_init(&bars[s], 1);
+    for (int w = 0; w < kDecWarps; ++w) mbar_init(&rbars[w], 1);
     fence_mbar_init();
   }
   if (tid < kDecMaxTok) ident[tid] = tid;
@@ -198,8 +201,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
 
   // ---- router linear (with wr): each CTA computes the logits of its
   // experts e = blockIdx.x + G * (warp + kDecWarps * i), one warp per expert
-  // row: lane l sums channels 8 l .. 8 l + 7 of every 256 in fp32 FMAs, the
-  // lanes' sums meet in an xor-shuffle tree (a fixed order), and lane t
+  // row: lane l sums channels 8 l .. 8 l + 7 of every 256, in channel order,
+  // in fp32 FMAs, the lanes' sums meet in an xor-shuffle tree (a fixed
+  // order), and lane t
   // publishes token t's logit as a word {logit, epoch} for every CTA's
   // routing below.  All CTAs are resident together (cooperative launch) and
   // this phase waits on nothing but x, so every word gets written.
@@ -209,46 +213,74 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
       const unsigned int ep = ctrl0 + 1u;  // this call's epoch; never 0 (zeroed words never match)
       misc[2] = (int)(ep == 0u ? 1u : ep);
     }
+    // a warp's row comes into shared memory by one bulk copy (the stage
+    // buffers are idle until the first weight copy, and 16 warps x 2 H bytes
+    // fit in two stages); the first row's copy starts before waiting for x
     const int e_first = (int)blockIdx.x + G * warp;
-    if (e_first < Er)  // start the first row's lines on their way to L2 while x lands
-      for (int ln = lane; ln < H / 64; ln += 32)
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(a.wr + (size_t)e_first * H + 64 * ln));
+    uint8_t *rowbuf = smem + L.stages + (size_t)warp * H * 2;
+    auto fetch_row = [&](int e) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&rbars[warp], (uint32_t)H * 2u);
+        bulk_g2s(rowbuf, a.wr + (size_t)e * H, (uint32_t)H * 2u, &rbars[warp]);
+      }
+    };
+    if (e_first < Er) fetch_row(e_first);
     cp_async_wait_all();
     __syncthreads();
     const unsigned int ep = (unsigned int)misc[2];
+    uint32_t rpar = 0;
     for (int e = e_first; e < Er; e += G * kDecWarps) {
-      float acc[kDecMaxTok];
+      if (e != e_first) {
+        __syncwarp();  // every lane is done with the previous row
+        fence_proxy_async_smem();
+        fetch_row(e);
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&rbars[warp], rpar, 1u << 22))) {
+        if (lane == 0) atomicExch(a.err, DEVERR_DECODE_ROUTER_WAIT);
+        break;  // the row never came: its words stay unwritten, and the routing's bounded waits give up
+      }
+      rpar ^= 1u;
+      // tokens in groups of four (a loop over groups keeps the code short:
+      // tokens past T cost issue slots even when predicated off)
+      for (int t0 = 0; t0 < T; t0 += 4) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int c = 8 * lane; c < H; c += 256) {
+          float wf[8];
+          bf16x8_f32(*reinterpret_cast<const uint4 *>(rowbuf + (size_t)c * 2), wf);
 #pragma unroll
-      for (int t = 0; t < kDecMaxTok; ++t) acc[t] = 0.f;
-      const uint16_t *row = a.wr + (size_t)e * H;
-      for (int c = 8 * lane; c < H; c += 256) {
-        float wf[8];
-        bf16x8_f32(__ldg(reinterpret_cast<const uint4 *>(row + c)), wf);
+          for (int tt = 0; tt < 4; ++tt) {
+            if (t0 + tt < T) {
+              float xf[8];
+              bf16x8_f32(*reinterpret_cast<const uint4 *>(x_s + (size_t)(t0 + tt) * H + c), xf);
 #pragma unroll
-        for (int t = 0; t < kDecMaxTok; ++t) {
-          if (t < T) {
-            float xf[8];
-            bf16x8_f32(*reinterpret_cast<const uint4 *>(x_s + (size_t)t * H + c), xf);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[t] = __fmaf_rn(xf[i], wf[i], acc[t]);
+              for (int i = 0; i < 8; ++i) acc[tt] = __fmaf_rn(xf[i], wf[i], acc[tt]);
+            }
           }
         }
-      }
-      float mine = 0.f;
+        float mine = 0.f;
 #pragma unroll
-      for (int t = 0; t < kDecMaxTok; ++t) {
-        if (t < T) {
-          float v = acc[t];
+        for (int tt = 0; tt < 4; ++tt) {
+          if (t0 + tt < T) {
+            float v = acc[tt];
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
-          if (lane == t) mine = v;
+            for (int o = 16; o > 0; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+            if (lane == tt) mine = v;
+          }
+        }
+        if (lane < 4 && t0 + lane < T) {
+          const int t = t0 + lane;
+          a.lbuf[(size_t)t * Er + e] = ((unsigned long long)__float_as_uint(mine) << 32) | ep;
+          if (a.logits_out) a.logits_out[(size_t)t * Er + e] = mine;
+          // every CTA polls these words: push them out now (without the
+          // fence they reached the pollers microseconds later; the h and row
+          // words below measured slower with one)
+          __threadfence();
         }
       }
-      if (lane < T) {
-        a.lbuf[(size_t)lane * Er + e] = ((unsigned long long)__float_as_uint(mine) << 32) | ep;
-        if (a.logits_out) a.logits_out[(size_t)lane * Er + e] = mine;
-      }
     }
+    // the rows were read by the generic proxy; the stages' next writers are
+    // the weight copies (async proxy)
+    fence_proxy_async_smem();
   }
 
   // ---- routing table.  Unique experts in increasing id ("slots"); the
@@ -267,26 +299,27 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
         unsigned long long wv[PER];
 #pragma unroll
         for (int i = 0; i < PER; ++i) wv[i] = lane + 32 * i < Er ? ld_relaxed_u64(lw + lane + 32 * i) : 0ull;
-        bool ok = true;
+        // every round reloads all of the lane's words still from an earlier
+        // call, together
+        uint32_t spins = 0;
+        while (true) {
+          uint32_t pending = 0;
 #pragma unroll
-        for (int i = 0; i < PER; ++i) {
-          const int e = lane + 32 * i;
-          if (e < Er) {
-            uint32_t spins = 0;
-            while (ok && (unsigned int)(wv[i] & 0xFFFFFFFFull) != ep) {
-              if (++spins > (1u << 22)) {
-                ok = false;  // the logit is used as read; the error word tells the caller
-                atomicExch(a.err, DEVERR_DECODE_ROUTER_WAIT);
-                break;
-              }
-              __nanosleep(32);
-              wv[i] = ld_relaxed_u64(lw + e);
-            }
-            key[i] = route_key(__uint_as_float((unsigned int)(wv[i] >> 32)));
-          } else {
-            key[i] = 0u;
+          for (int i = 0; i < PER; ++i)
+            if (lane + 32 * i < Er && (unsigned int)(wv[i] & 0xFFFFFFFFull) != ep) pending |= 1u << i;
+          if (!pending) break;
+          if (++spins > (1u << 22)) {  // the logits are used as read; the error word tells the caller
+            atomicExch(a.err, DEVERR_DECODE_ROUTER_WAIT);
+            break;
           }
+          __nanosleep(32);
+#pragma unroll
+          for (int i = 0; i < PER; ++i)
+            if ((pending >> i) & 1u) wv[i] = ld_relaxed_u64(lw + lane + 32 * i);
         }
+#pragma unroll
+        for (int i = 0; i < PER; ++i)
+          key[i] = lane + 32 * i < Er ? route_key(__uint_as_float((unsigned int)(wv[i] >> 32))) : 0u;
       } else {
 #pragma unroll
         for (int i = 0; i < PER; ++i) {
@@ -697,6 +730,8 @@ static moe_status decode_launch(DecodeArgs &a, bool pdl, cudaStream_t stream) {
   while (nst > 2 && decode_smem_layout(kFmt, T, H, F, nst, a.stage_bytes).total > cap) nst -= 2;
   const DecodeSmem L = decode_smem_layout(kFmt, T, H, F, nst, a.stage_bytes);
   if (L.total > cap) return MOE_ERR_UNSUPPORTED_SHAPE;
+  // the router rows (one per warp) are staged in the idle stage buffers
+  if (a.wr && (size_t)nst * a.stage_bytes < (size_t)kDecWarps * 2u * (size_t)H) return MOE_ERR_UNSUPPORTED_SHAPE;
   a.nstages = nst;
   // per device: the shared-memory opt-in and the CTAs per SM it allows
   // (host threads may race here; both values are idempotent)
