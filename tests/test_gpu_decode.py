@@ -155,8 +155,8 @@ def test_decode_with_an_sm_held_by_another_stream():
     cooperative, and while a kernel on another stream holds one SM (and all
     its shared memory) for about a second, the grid waits for the SM, runs
     whole, and gives the oracle's result with no device error.  The fused
-    layer kernel waits only inside its clusters, so it runs beside the held
-    SM and gives the oracle's result too."""
+    layer kernel is launched the same way and gives the oracle's result
+    too."""
     import gpu_hold
     E, H, F, T, k, seed = 256, 2048, 512, 1, 8, 91
     x = synth.activations_bf16(seed, 0, T, H)
