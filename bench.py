@@ -105,7 +105,31 @@ KERNEL_SOURCES = {
     "prefill_nvfp4": ["prefill_nvfp4.cu", "tcgen05.cuh", "common.cuh", "nvfp4.cuh"],
 }
 TRAFFIC = {
-    # key: (kernel, workload) -> {"bytes": per launch (or per launch pair), "sha": digest, "how": ...}
+    # key -> {"bytes": DRAM read + write of the captured launch, "alg": its algorithmic bytes,
+    #         "sha": digest of the kernel's sources, "how": the capture}.  A leg's traffic is
+    # bytes / alg x the leg's algorithmic bytes per launch (traffic grows with the unique
+    # experts a launch streams; the captures are smaller cases of the same kernel).
+    "decode_w4_T1": {"bytes": 14255872, "alg": 14164992, "sha": "29425667925c1440",
+                     "how": "profiles/decode_kernel_single_layer_T1.md, 2 resident layers"},
+    "decode_w4_shared_T1": {"bytes": 16021504, "alg": 15934464, "sha": "29425667925c1440",
+                            "how": "profiles/decode_kernel_single_layer_T1.md, shared expert, 2 resident layers"},
+    "decode_router_T1": {"bytes": 15303936, "alg": 15213440, "sha": "29425667925c1440",
+                         "how": "profiles/decode_kernel_single_layer_T1.md, router inside, 2 resident layers"},
+    "decode_w4_T16": {"bytes": 186604544, "alg": 182403072, "sha": "29425667925c1440",
+                      "how": "profiles/decode_kernel_single_layer_T1.md, stream kernel at 16 tokens, "
+                             "2 resident layers"},
+    "decode_nvfp4_T1": {"bytes": 14292224, "alg": 14164992, "sha": "29425667925c1440",
+                        "how": "profiles/decode_kernel_nvfp4_single_layer_T1.md, 2 resident layers"},
+    "prefill_w4_2048": {"bytes": 314900992, "sha": "45646a7528abf117",
+                        "how": "profiles/prefill_kernel_grouped_2048tok.md, gate/up + down launch pair"},
+    "router_T2048": {"bytes": 11555584, "alg": 11665408, "sha": "9739658a7ea06e4b",
+                     "how": "profiles/router_kernels_T1_T2048.md, GEMM + routing launches"},
+    "router_T1": {"bytes": 1082368, "alg": 1053760, "sha": "9739658a7ea06e4b",
+                  "how": "profiles/router_kernels_T1_T2048.md"},
+    "quant_clip_g64": {"bytes": 154823168, "sha": "c8f14825edeba35f",
+                       "how": "profiles/clip_search_kernel_128MB.md"},
+    "quant_sym128": {"bytes": 154248192, "sha": "c8f14825edeba35f",
+                     "how": "profiles/clip_search_kernel_128MB.md"},
 }
 
 
@@ -118,8 +142,9 @@ def sources_sha(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
-def traffic_of(key: str, kernel: str):
-    """(bytes, source note): the captured figure if the kernel's sources still
+def traffic_of(key: str, kernel: str, alg=None):
+    """(bytes per launch, source note): the captured figure, scaled to the
+    leg's algorithmic bytes when both are known, if the kernel's sources still
     have the digest they had at capture time, else (None, why)."""
     rec = TRAFFIC.get(key)
     sha = sources_sha(kernel)
@@ -127,6 +152,9 @@ def traffic_of(key: str, kernel: str):
         return None, f"not captured for the current sources (sha {sha})"
     if rec["sha"] != sha:
         return None, f"stale: captured on sources {rec['sha']}, current {sha}"
+    if alg is not None and rec.get("alg"):
+        return rec["bytes"] / rec["alg"] * alg, (f"ncu capture ({rec['how']}) on sources {sha}: "
+                                                 f"{rec['bytes']} B for {rec['alg']} algorithmic B, scaled")
     return rec["bytes"], f"ncu capture ({rec['how']}) on sources {sha}"
 
 
@@ -513,7 +541,7 @@ def views(buf, specs):
 def hbm_roofline(alg_bytes, dur_ms, kernel, traffic_key, src_kernel, extra=None):
     peak, peak_kind = hbm_peak()
     achieved = alg_bytes / (dur_ms / 1e3) / 1e9
-    traffic, tsrc = traffic_of(traffic_key, src_kernel)
+    traffic, tsrc = traffic_of(traffic_key, src_kernel, alg_bytes)
     r = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
          "traffic": traffic, "traffic_source": tsrc, "kernel": kernel, "peak_kind": peak_kind,
          "alg_bytes_per_launch": alg_bytes, "avg_launch_us": dur_ms * 1e3}
@@ -687,6 +715,7 @@ def leg_prefill(ctx, T=2048, nl=4):
     import quantized_moe_route_b200 as moe
     args, k = ctx.args, TOPK
     layers = ctx.w4_layers()[:nl]
+    nl = len(layers)
     seed = SEED_PREFILL + ctx.rank
     xs, ls, host, _ = _prefill_inputs(seed, T, nl, ctx)
     R = T * k
@@ -766,6 +795,7 @@ def leg_prefill_nvfp4(ctx, T=512, nl=8):
     import quantized_moe_route_b200 as moe
     args, k = ctx.args, TOPK
     layers = ctx.nv_layers()[:nl]
+    nl = len(layers)
     seed = SEED_NVP + ctx.rank
     xs, ls, host, uniq = _prefill_inputs(seed, T, nl, ctx)
     R = T * k
@@ -964,7 +994,8 @@ def leg_router(ctx, T):
     dur_ms = ms / K
     alg = T * H * 2 + E * H * 2 + T * E * 4 + T * k * 8  # x, Wr, logits, idx + w
     flops = 2.0 * T * E * H
-    roof = hbm_roofline(alg, dur_ms, "moe::router_kernel", f"router_T{T}", "router",
+    kname = "moe::router_gemv_kernel" if T <= 16 else "moe::router_mma_kernel + moe::route_kernel (one call)"
+    roof = hbm_roofline(alg, dur_ms, kname, f"router_T{T}", "router",
                         {"tflops": flops / (dur_ms / 1e3) / 1e12,
                          "note": "HBM-bound at both sizes: at T=2048 the bytes take longer than the "
                                  "contraction at the measured bf16 peak"})
@@ -988,7 +1019,7 @@ def leg_router(ctx, T):
         "e2e": {"value": job_throughput(K * T, ctx.world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "overlap": "each step's copies run on copy streams beside the neighbouring steps' kernels"},
-        "gpu_launches": K,
+        "gpu_launches": K * (1 if T <= 16 else 2),
         "clocks": clocks,
     }
 
