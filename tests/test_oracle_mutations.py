@@ -50,7 +50,7 @@ MUTATIONS = [
      "u += wu * xf[i];\n    }\n    h[n] = g / (1.0f + expf(-g)) * u;",
      "u += wu * xf[i];\n    }\n    h[n] = u / (1.0f + expf(-u)) * g;", METHOD_PINS),
     ("int4 FFN: down weights transposed",
-     "d_codes[(size_t)c * F + n]", "d_codes[(size_t)n * H + c]", METHOD_PINS),
+     "orc_dequant_one(d_codes[(size_t)c * F + n]", "orc_dequant_one(d_codes[(size_t)n * H + c]", METHOD_PINS),
     ("route: ties go to the higher expert id",
      "if (best < 0 || l[e] > l[best]) best = e;", "if (best < 0 || l[e] >= l[best]) best = e;", METHOD_PINS),
     ("route: weights not renormalised over the selected experts",
