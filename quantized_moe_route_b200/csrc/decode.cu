@@ -370,11 +370,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs a) {
     if (lane == 0) {
       misc[0] = U;
       misc[1] = 0;
-      const int nA = U * (F / 16), nItems = nA + U * (H / kDecOutRows);
-      const int myCount = (int)blockIdx.x < nItems ? (nItems - 1 - (int)blockIdx.x) / G + 1 : 0;
-      const uint64_t pol = policy_evict_first();
-      for (int q = 0; q < min(myCount, a.nstages); ++q) issue(blockIdx.x + q * G, nA, q, pol);
     }
+    // the CTA's first nstages items: lane q issues item q's copy into stage q
+    // (the copies leave together instead of one after another)
+    const int nA = U * (F / 16), nItems = nA + U * (H / kDecOutRows);
+    const int myCount = (int)blockIdx.x < nItems ? (nItems - 1 - (int)blockIdx.x) / G + 1 : 0;
+    if (lane < min(myCount, a.nstages)) issue(blockIdx.x + lane * G, nA, lane, policy_evict_first());
   }
   if (!kFp4) cp_async_wait_all();  // this thread's x copies
   __syncthreads();

@@ -38,9 +38,67 @@ __device__ __forceinline__ float route_key_value(uint32_t key) {
 
 // The selection from the lanes' keys: key[i] is expert lane + 32 i's
 // route_key (0 past the last expert).
+//
+// Eight entries per lane (E <= 256): each lane first sorts its entries by
+// (key larger first, id smaller first) with a 19-comparator merge network,
+// so a round's winner only shifts its list; the winner is the one lane whose
+// head equals the warp maximum (a ballot), or, when several heads are equal,
+// the lowest id among them (a second reduction).  The same selection as the
+// general form, with a shorter dependent chain per round.  (A butterfly
+// merge of the lanes' sorted lists, five exchange steps of eight 64-bit
+// values, measured slower than these k rounds.)
 template <int PER>
 __device__ __forceinline__ void route_token_keys(const uint32_t (&key)[PER], int k, int *idx_j, float *w_j) {
   const int lane = threadIdx.x & 31;
+  if constexpr (PER == 8) {
+    uint64_t c[8];  // key << 8 | (255 - i): larger is earlier
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c[i] = ((uint64_t)key[i] << 8) | (uint64_t)(255 - i);
+    auto cas = [&](int a, int b) {  // c[a] >= c[b] afterwards
+      const uint64_t hi = c[a] > c[b] ? c[a] : c[b], lo = c[a] > c[b] ? c[b] : c[a];
+      c[a] = hi;
+      c[b] = lo;
+    };
+    cas(0, 1); cas(2, 3); cas(4, 5); cas(6, 7);
+    cas(0, 2); cas(1, 3); cas(4, 6); cas(5, 7);
+    cas(1, 2); cas(5, 6);
+    cas(0, 4); cas(1, 5); cas(2, 6); cas(3, 7);
+    cas(2, 4); cas(3, 5);
+    cas(1, 2); cas(3, 4); cas(5, 6);
+    float top = 0.f, denom = 0.f, my_w = 0.f;
+    int my_idx = 0;
+    for (int j = 0; j < k; ++j) {
+      const uint32_t hk = (uint32_t)(c[0] >> 8);
+      const uint32_t hid = (uint32_t)lane + 32u * (255u - (uint32_t)(c[0] & 0xFFu));
+      const uint32_t kmax = __reduce_max_sync(0xffffffffu, hk);
+      const uint32_t hit = __ballot_sync(0xffffffffu, hk == kmax);
+      uint32_t ri;
+      int wl;
+      if ((hit & (hit - 1u)) == 0u) {  // one lane holds the maximum
+        wl = __ffs(hit) - 1;
+        ri = __shfl_sync(0xffffffffu, hid, wl);
+      } else {  // equal keys: the lowest id
+        ri = __reduce_min_sync(0xffffffffu, hk == kmax ? hid : 0xffffffffu);
+        wl = (int)(ri & 31u);
+      }
+      if (lane == wl) {
+#pragma unroll
+        for (int i = 0; i < 7; ++i) c[i] = c[i + 1];
+        c[7] = 0ull;
+      }
+      const float rv = route_key_value(kmax);
+      if (j == 0) top = rv;
+      const float ex = expf(rv - top);
+      denom += ex;
+      if (lane == j) {
+        my_idx = (int)ri;
+        my_w = ex;
+      }
+    }
+    *idx_j = my_idx;
+    *w_j = my_w / denom;
+    return;
+  }
   uint32_t taken = 0;  // bit i: expert lane + 32 i already selected
   // local best of the untaken entries: entries visited in increasing id and
   // strict > keeps the lowest id among equal keys; key 0 = nothing left
