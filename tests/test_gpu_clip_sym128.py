@@ -27,13 +27,30 @@ def _weights_with_edge_groups(seed, N, K):
     w[1, :128] = 0.0125                                     # constant group
     w[2, :64] = np.tile(np.arange(16), 4) * np.float32(2.0 ** -8) - np.float32(0.03125)  # exact asym group
     w[3, :128] = synth.expert_weights(seed, 0, 1, 0, 1, 128)[0] * 40  # wide-range group
+    # quotients exactly on half-integers at ratio 1.0 (ties to even): asymmetric
+    # m = -0.5, s = 0.0625; symmetric amax = 0.46875, s = 2 amax / 15 = 0.0625
+    k = np.arange(64) % 15
+    w[4, :64] = np.float32(-0.5) + (k + np.float32(0.5)) * np.float32(0.0625)
+    w[4, 0], w[4, 63] = np.float32(-0.5), np.float32(0.4375)
+    j = np.arange(128) % 8
+    w[5, :128] = np.where(np.arange(128) % 2 == 0, 1, -1) * (j + np.float32(0.5)) * np.float32(0.0625)
+    w[5, 0] = np.float32(0.46875)
     return w
 
 
-def test_clip_quantiser_bit_exact_with_oracle():
+def _on_device(w, offset):
+    """w on the device starting `offset` floats into a buffer (offset 1: not 16-byte aligned)."""
+    buf = torch.empty(w.size + 4, dtype=torch.float32, device="cuda")
+    d = buf[offset:offset + w.size].view(*w.shape)
+    d.copy_(torch.from_numpy(w))
+    return d
+
+
+@pytest.mark.parametrize("offset", [0, 1])
+def test_clip_quantiser_bit_exact_with_oracle(offset):
     w = _weights_with_edge_groups(61, 64, 1024)
     c, s, m = oracle.quantize_w4_clip(w)
-    dw = torch.from_numpy(w).cuda()
+    dw = _on_device(w, offset)
     gc = torch.empty((64, 1024), dtype=torch.uint8, device="cuda")
     gs = torch.empty((64, 16), dtype=torch.int16, device="cuda")
     gm = torch.empty((64, 16), dtype=torch.int16, device="cuda")
@@ -43,10 +60,11 @@ def test_clip_quantiser_bit_exact_with_oracle():
     assert np.array_equal(to_u16(gs), s) and np.array_equal(to_u16(gm), m)
 
 
-def test_sym128_quantiser_bit_exact_with_oracle():
+@pytest.mark.parametrize("offset", [0, 1])
+def test_sym128_quantiser_bit_exact_with_oracle(offset):
     w = _weights_with_edge_groups(62, 64, 1024)
     c, s = oracle.quantize_sym128(w)
-    dw = torch.from_numpy(w).cuda()
+    dw = _on_device(w, offset)
     gc = torch.empty((64, 1024), dtype=torch.uint8, device="cuda")
     gs = torch.empty((64, 8), dtype=torch.int16, device="cuda")
     moe.moe_quantize_w4_sym128(dw, gc, gs)
