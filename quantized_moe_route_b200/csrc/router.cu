@@ -20,7 +20,8 @@
 // tokens x 64 experts (BM = 64 from 256 tokens up, so every router row is
 // read T / 64 times; 16 below, for more CTAs): m16n8k16 bf16 MMAs with
 // ldmatrix fragments, fp32 accumulation, K in chunks of 64 channels staged
-// through shared memory by cp.async with several chunks in flight.  Routing
+// through shared memory by cp.async with 8 (64-token tiles) or 6 chunks in
+// flight.  Routing
 // in the GEMM's last CTA per tile would serialise BM tokens on four warps;
 // the separate launch routes every token in parallel.
 #include <atomic>
@@ -350,7 +351,7 @@ extern "C" MOE_API moe_status moe_router_route(const uint16_t *x, const uint16_t
   moe_status st;
   const int by = (E + 63) / 64;
   if (T >= 256) {
-    constexpr int ST = 4, BM = 64;
+    constexpr int ST = 8, BM = 64;
     const size_t smem = (size_t)ST * (BM + 64) * kRtLd * 2;
     auto kern = router_mma_kernel<2, 4, 2, 2, ST>;
     static std::atomic<unsigned long long> done{0};
