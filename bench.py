@@ -109,22 +109,22 @@ TRAFFIC = {
     #         "sha": digest of the kernel's sources, "how": the capture}.  A leg's traffic is
     # bytes / alg x the leg's algorithmic bytes per launch (traffic grows with the unique
     # experts a launch streams; the captures are smaller cases of the same kernel).
-    "decode_w4_T1": {"bytes": 14255872, "alg": 14164992, "sha": "29425667925c1440",
+    "decode_w4_T1": {"bytes": 14255616, "alg": 14164992, "sha": "43e8b20b61872d94",
                      "how": "profiles/decode_kernel_single_layer_T1.md, 2 resident layers"},
-    "decode_w4_shared_T1": {"bytes": 16021504, "alg": 15934464, "sha": "29425667925c1440",
+    "decode_w4_shared_T1": {"bytes": 16020992, "alg": 15934464, "sha": "43e8b20b61872d94",
                             "how": "profiles/decode_kernel_single_layer_T1.md, shared expert, 2 resident layers"},
-    "decode_router_T1": {"bytes": 15303936, "alg": 15213440, "sha": "29425667925c1440",
+    "decode_router_T1": {"bytes": 15303168, "alg": 15213440, "sha": "43e8b20b61872d94",
                          "how": "profiles/decode_kernel_single_layer_T1.md, router inside, 2 resident layers"},
-    "decode_w4_T16": {"bytes": 186604544, "alg": 182403072, "sha": "29425667925c1440",
+    "decode_w4_T16": {"bytes": 185648128, "alg": 182403072, "sha": "43e8b20b61872d94",
                       "how": "profiles/decode_kernel_single_layer_T1.md, stream kernel at 16 tokens, "
                              "2 resident layers"},
-    "decode_nvfp4_T1": {"bytes": 14292224, "alg": 14164992, "sha": "29425667925c1440",
+    "decode_nvfp4_T1": {"bytes": 14292480, "alg": 14164992, "sha": "43e8b20b61872d94",
                         "how": "profiles/decode_kernel_nvfp4_single_layer_T1.md, 2 resident layers"},
     "prefill_w4_2048": {"bytes": 314900992, "sha": "45646a7528abf117",
                         "how": "profiles/prefill_kernel_grouped_2048tok.md, gate/up + down launch pair"},
-    "router_T2048": {"bytes": 11555584, "alg": 11665408, "sha": "9739658a7ea06e4b",
+    "router_T2048": {"bytes": 11567360, "alg": 11665408, "sha": "96de99454fcdc218",
                      "how": "profiles/router_kernels_T1_T2048.md, GEMM + routing launches"},
-    "router_T1": {"bytes": 1082368, "alg": 1053760, "sha": "9739658a7ea06e4b",
+    "router_T1": {"bytes": 1094144, "alg": 1053760, "sha": "96de99454fcdc218",
                   "how": "profiles/router_kernels_T1_T2048.md"},
     "quant_clip_g64": {"bytes": 154823168, "sha": "c8f14825edeba35f",
                        "how": "profiles/clip_search_kernel_128MB.md"},
