@@ -20,7 +20,7 @@
  *   - softmax routing with renormalised top-k over the router logits, and the
  *     router-weighted combine (the router is bf16 per "Drama 3 int4",
  *     "What's quantized"; top-k = 8, renormalisation and the lowest-index tie
- *     break are the readings this build takes where the pages are silent).
+ *     break are the readings taken where the pages are silent).
  *   - NVFP4 experts: packed E2M1 codes, one E4M3 scale per 16 input channels,
  *     one FP32 global scale per matrix, gate and up sharing it, dynamic
  *     per-token activation scales ("Drama 3 - NVFP4 routed experts",
@@ -392,8 +392,8 @@ ORC_API void orc_combine(const float *Yrows, const float *w, int T, int k, int H
  * weight 1.  The pages list a shared expert beside the routed ones ("Drama 3
  * int4 (drama-rs format)", table "What's quantized"; "Drama 3 - NVFP4 routed
  * experts", section "Quantization"); weight 1, its place after the routed
- * sum, and its int4 storage (in the routed experts' format) are this build's
- * reading.  idx/w receive the k routed choices; y_rows (optional) [T][k+1][H]
+ * sum, and its int4 storage (in the routed experts' format) are the reading
+ * taken here.  idx/w receive the k routed choices; y_rows (optional) [T][k+1][H]
  * the rows.  Parity: pinned (zero shared weights give the routed-only result;
  * zero routed weights give the shared expert alone; the composition of the
  * pinned FFN and combine). */
@@ -434,7 +434,7 @@ ORC_API void orc_moe_forward_w4_shared(const uint16_t *x, const float *logits, i
 /* keeps bf16 weights ("Drama 3 int4 (drama-rs format)", table "What's       */
 /* quantized": embeddings, router, norms bf16 / f32; "DRAMA-3 MLX            */
 /* expert-only 4-bit", section "Quantization and provenance": routers retain */
-/* source BF16); fp32 accumulation and no bias are this build's reading.     */
+/* source BF16); fp32 accumulation and no bias are the reading taken here.  */
 /* Parity: pinned (one-hot rows select a channel of x exactly; a float64     */
 /* matmul within the fp32 summation bound; linearity in x).                  */
 /* ------------------------------------------------------------------------ */
