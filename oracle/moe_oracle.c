@@ -25,6 +25,13 @@
  *     one FP32 global scale per matrix, gate and up sharing it, dynamic
  *     per-token activation scales ("Drama 3 - NVFP4 routed experts",
  *     section "Quantization", bullets 2 and 4).
+ *   - the MSE clip search over 20 clipping ratios 1.00 -> 0.81 ("Drama 3 int4
+ *     (drama-rs format)", "What's quantized"; "drama-3-w4a16", "How it was
+ *     made") for the asymmetric group-64 format and for the symmetric
+ *     group-128 format with zero point 8 ("drama-3-w4a16", "At a glance").
+ *   - the bf16 router linear (logits = Wr x) and a shared expert beside the
+ *     routed ones ("Drama 3 int4 (drama-rs format)", "What's quantized";
+ *     "Drama 3 - NVFP4 routed experts", "Quantization").
  *
  * Precision: the FFN accumulates in fp32 with k ascending, dequantises with
  * one fp32 fused multiply-add (q*s + m, single rounding), and rounds the
