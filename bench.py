@@ -118,6 +118,10 @@ TRAFFIC = {
     "decode_w4_T16": {"bytes": 185648128, "alg": 182403072, "sha": "43e8b20b61872d94",
                       "how": "profiles/decode_kernel_single_layer_T1.md, stream kernel at 16 tokens, "
                              "2 resident layers"},
+    "decode_w4_T4": {"bytes": 55533312, "alg": 54890496, "sha": "43e8b20b61872d94",
+                     "how": "profiles/decode_kernel_single_layer_T1.md, stream kernel at 4 tokens, 2 resident layers"},
+    "prefill_nvfp4_512": {"bytes": 144929536, "alg": 169852928, "sha": "6795a7bcc7dffc35",
+                          "how": "profiles/prefill_nvfp4_kernel_grouped_512tok.md, the FFN call's three launches"},
     "decode_nvfp4_T1": {"bytes": 14292480, "alg": 14164992, "sha": "43e8b20b61872d94",
                         "how": "profiles/decode_kernel_nvfp4_single_layer_T1.md, 2 resident layers"},
     "prefill_w4_2048": {"bytes": 314900992, "sha": "45646a7528abf117",
