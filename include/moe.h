@@ -276,11 +276,15 @@ MOE_API moe_status moe_route_shared(const float *logits, int T, int E, int k, in
                                     float *w, moe_stream_t stream);
 
 /*
- * The router linear fused with routing, in one launch: logits[t][e] =
- * sum_k x[t][k] * Wr[e][k] (x bf16 [T][H], Wr bf16 [E][H], fp32 products and
- * sums, no bias), then the routing of moe_route on those logits (idx, w as
- * there).  logits fp32 [T][E] is an optional output (NULL: kept in the
- * workspace).  Source: the router stays bf16 ("Drama 3 int4 (drama-rs
+ * The router linear fused with routing: logits[t][e] = sum_k x[t][k] *
+ * Wr[e][k] (x bf16 [T][H], Wr bf16 [E][H], fp32 products and sums, no bias),
+ * then the routing of moe_route on those logits (idx, w as there).  Up to 16
+ * tokens one launch does both (the last CTA to finish its logits routes);
+ * above, a tensor-core GEMM launch is followed by moe_route's kernel, chained
+ * by programmatic dependent launch.  logits fp32 [T][E] is an optional
+ * output (NULL: kept in the workspace).  For a decode layer,
+ * moe_decode_layer_w4a16_router computes the router inside the layer's own
+ * launch instead.  Source: the router stays bf16 ("Drama 3 int4 (drama-rs
  * format)", table "What's quantized"; "DRAMA-3 MLX expert-only 4-bit",
  * section "Quantization and provenance"); fp32 accumulation and no bias are
  * this library's reading.  The products are summed in the kernel's own
