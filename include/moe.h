@@ -103,7 +103,8 @@ MOE_API moe_status moe_quantize_w4(const float *w, int N, int K, uint8_t *codes,
  * the rounded m) and coded by nearest rounding; the candidate with the
  * smallest fp32 sum over the group, in channel order, of (q*s + m - w)^2 wins,
  * ties to the larger ratio.  p = 1 is exactly moe_quantize_w4's choice, so
- * no group gets a larger squared error.  Bit-exact with the reference.
+ * no group gets a larger squared error.  Every step is one correctly rounded
+ * fp32 operation, so the choice and the codes do not depend on the device.
  * Source: "Drama 3 int4 (drama-rs format)", table "What's quantized" (MSE
  * clip search); "drama-3-w4a16", section "How it was made" (20 clipping
  * ratios 1.0 -> 0.81 by minimum squared error).  Errors as moe_quantize_w4.
