@@ -20,13 +20,26 @@ symmetric, group 128, GPTQ packing).
 - The symmetric group-128 FFN equals, bit for bit, the (pinned) asymmetric
   group-64 FFN of the same weights written as scale s and min -8 s.
 """
+import os
+
 import numpy as np
 import pytest
 
 import oracle
 import synth
 
-RATIOS = [np.float32(100 - i) / np.float32(100) for i in range(20)]
+def _page_figure(key):
+    with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "page_figures.txt")) as f:
+        for line in f:
+            parts = line.split("|")[0].split()
+            if len(parts) == 2 and parts[0] == key:
+                return float(parts[1])
+    raise KeyError(key)
+
+
+# the page's schedule: 20 ratios from 1.00 down to 0.81 in steps of 0.01
+RATIOS = [np.float32(100 - i) / np.float32(100) for i in range(int(_page_figure("clip_ratio_count")))]
+assert float(RATIOS[0]) == _page_figure("clip_ratio_first") and abs(float(RATIOS[-1]) - _page_figure("clip_ratio_last")) < 1e-6
 
 
 def f16(bits):
@@ -138,7 +151,8 @@ def test_sym128_gaussian_error_matches_the_page():
         c, s = oracle.quantize_sym128(w)
         deq = (c.astype(np.float64) - 8) * np.repeat(f16(s), 128, 1)
         errs.append(np.linalg.norm(deq - w) / np.linalg.norm(w))
-    assert 0.095 < np.mean(errs) < 0.108, errs
+    page = _page_figure("sym128_mean_rel_error")
+    assert 0.92 * page < np.mean(errs) < 1.05 * page, errs
 
 
 def test_sym128_ffn_equals_the_asymmetric_ffn_of_the_same_weights():
